@@ -1,0 +1,7 @@
+"""Seeded synthetic workloads for relative-position attention.
+
+This package only draws random numbers and shapes them into the inputs of
+one attention layer.  It holds none of the attention arithmetic: both the
+CUDA library's tests/benchmarks and the CPU oracle consume what it returns.
+"""
+from .workloads import CONFIGS, Workload, make_workload, small_workload  # noqa: F401
