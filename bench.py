@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of one exact relative-position attention layer on B200.
+
+A step is one forward + backward of the layer (projection, fused attention,
+two-pass backward, relation-table gradients) over one batch of synthetic
+input.  Workload: Shaw truncated map clip 64 (129 relation rows) with both
+the q.aQ and k.aK terms, B=1, H=12, N=8192, d=64, fp16 -- the 8K x 12-head
+x d64 layer the paper digest reports its headline speed-ups on.
+
+Metric: useful TFLOP/s of the layer (forward 4 B H N^2 d + backward
+10 B H N^2 d, plus the relation projections 2 (fwd) / 4 (bwd) B H N R d per
+term), with the inputs resident in HBM, L2 flushed before every step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With --gpus N > 1 (launched under torch.distributed.run) every rank runs an
+independent replica of the layer on its own batch (weak scaling; the layer
+has no cross-rank exchange), timed on the device as the max over ranks.
+`--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "shaw_clip64_n8192"
+
+
+def useful_flops(w, R_exp):
+    """Useful FLOPs of one forward and one backward (FlashAttention convention)."""
+    cf = 0.5 if w.causal else 1.0
+    BH, N, d = w.B * w.H, w.N, w.d
+    nterms = int(w.aq is not None) + int(w.ak is not None)
+    fwd = 4.0 * BH * N * N * d * cf + 2.0 * BH * N * R_exp * d * nterms
+    bwd = 10.0 * BH * N * N * d * cf + 4.0 * BH * N * R_exp * d * nterms
+    return fwd, bwd
+
+
+def kernel_flops(w):
+    """Tensor-core FLOPs each attention kernel's algorithm performs per launch."""
+    cf = 0.5 if w.causal else 1.0
+    base = 2.0 * w.B * w.H * w.N * w.N * w.d * cf    # one N x N x d GEMM
+    return {"fwd_attention": 2 * base, "bwd_dq": 3 * base, "bwd_dkdv": 4 * base}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"bf16_tflops": j["bf16_tflops"], "bf16_tflops_sustained": j.get("bf16_tflops_sustained"),
+                "hbm_gbs": j["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_relative_position_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(phase):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernels."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    ent = j.get("kernels", {}).get(phase)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, R_exp, seconds=15.0, block=256):
+    """The fp64 oracle on the host cores over blocks of query rows of head 0."""
+    import numpy as np
+    import oracle as orc
+    from threadpoolctl import threadpool_info
+    f64 = lambda t: None if t is None else t.double().numpy()
+    q, k, v, do = (f64(getattr(w, n)[0, 0]) for n in ("q", "k", "v", "do"))
+    aq = None if w.aq is None else f64(w.aq if w.aq.dim() == 2 else w.aq[0])
+    ak = None if w.ak is None else f64(w.ak if w.ak.dim() == 2 else w.ak[0])
+    bv = None if w.b is None else f64(w.b[0])
+    kl = None if w.key_len is None else int(w.key_len[0])
+    m = orc.MapDesc(w.map_kind, w.clip, w.num_buckets, w.max_distance, w.bidirectional)
+    t0 = time.perf_counter()
+    rows_done = 0
+    r0 = 0
+    while time.perf_counter() - t0 < seconds:
+        rows = np.arange(r0, min(w.N, r0 + block))
+        orc.head_block_step(q, k, v, do, aq, ak, bv, w.tau, m, w.causal, kl, rows)
+        rows_done += len(rows)
+        r0 = (r0 + block) % w.N
+    dt = time.perf_counter() - t0
+    fwd, bwd = useful_flops(w, R_exp)
+    flops = (fwd + bwd) / (w.B * w.H * w.N) * rows_done
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle forward+backward of {rows_done} query rows ({rows_done // block} blocks of "
+                      f"{block}) of head 0 against all {w.N} keys, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 CPU oracle, one block of query rows per step."""
+    from synth import make_workload
+    import numpy as np
+    import oracle as orc
+    from threadpoolctl import threadpool_info
+    if rank != 0:
+        return
+    w = make_workload(WORKLOAD)
+    m = orc.MapDesc(w.map_kind, w.clip, w.num_buckets, w.max_distance, w.bidirectional)
+    elo, ehi = orc.expanded_bounds(m, w.N)
+    R_exp = ehi - elo + 1
+    f64 = lambda t: None if t is None else t.double().numpy()
+    q, k, v, do = (f64(getattr(w, n)[0, 0]) for n in ("q", "k", "v", "do"))
+    aq, ak = f64(w.aq), f64(w.ak)
+    block = 128
+
+    def step(i):
+        rows = np.arange((i * block) % w.N, (i * block) % w.N + block)
+        orc.head_block_step(q, k, v, do, aq, ak, None, w.tau, m, False, None, rows)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    fwd, bwd = useful_flops(w, R_exp)
+    flops_step = (fwd + bwd) / (w.B * w.H * w.N) * block
+    value = flops_step * args.steps / dt / 1e12
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    sample = (f"fp64 oracle forward+backward of one block of {block} query rows of head 0 against all {w.N} keys "
+              f"per step")
+    line = {"impl": "reference", "metric": "useful TFLOP/s of one rel-pos attention layer (fwd+bwd)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, **{k_: v_ for k_, v_ in w.describe().items() if k_ != "workload"}},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import exact_relative_position_b200 as rp
+    from synth import make_workload
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    w = make_workload(args.workload, seed=rank)
+    m = rp.RelPosMap(w.map_kind, w.clip, w.num_buckets, w.max_distance, w.bidirectional)
+    elo, ehi = rp.expanded_bounds(m, w.N)
+    R_exp = ehi - elo + 1
+    fwd_flops, bwd_flops = useful_flops(w, R_exp)
+    out_f32 = w.dtype == torch.bfloat16
+
+    d = lambda t: None if t is None else t.to(dev).contiguous()
+    q, k, v, do, aq, ak, b, kl = (d(getattr(w, n)) for n in ("q", "k", "v", "do", "aq", "ak", "b", "key_len"))
+    o = torch.empty(q.shape, device=dev, dtype=torch.float32 if out_f32 else q.dtype)
+    lse = torch.empty(q.shape[:3], device=dev, dtype=torch.float32)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+             None if aq is None else torch.empty(aq.shape, device=dev, dtype=torch.float32),
+             None if ak is None else torch.empty(ak.shape, device=dev, dtype=torch.float32),
+             None if b is None else torch.empty(b.shape, device=dev, dtype=torch.float32))
+    fws, bws = rp.workspace_size(q, aq, ak, b, w.tau, m, causal=w.causal, key_len=kl, out_f32=out_f32)
+    ws = torch.empty(max(fws, bws), device=dev, dtype=torch.uint8)
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)   # 256 MiB > 126 MB L2
+    kw = dict(tau=w.tau, map=m, causal=w.causal, key_len=kl)
+
+    def fwd():
+        rp.relpos_attn_fwd(q, k, v, aq, ak, b, out_f32=out_f32, workspace=ws, o=o, lse=lse, **kw)
+
+    def bwd():
+        rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, workspace=ws, grads=grads, **kw)
+
+    torch.cuda.reset_peak_memory_stats(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    input_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, do, aq, ak, b) if t is not None)
+
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    launches0 = rp.kernel_launches()
+    rp.profile_start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        flush.zero_()
+        ev[s][0].record(stream)
+        fwd()
+        ev[s][1].record(stream)
+        bwd()
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    phases = rp.profile_stop()
+    launches = rp.kernel_launches() - launches0
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev)
+    t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev)
+    t_step = t_fwd + t_bwd
+    if world > 1:
+        tt = torch.tensor([t_step, t_fwd, t_bwd], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step, t_fwd, t_bwd = tt.tolist()
+    peak_mem = torch.cuda.max_memory_allocated(dev)
+
+    # ---- end-to-end through the public API with host buffers
+    pin = lambda t: None if t is None else t.cpu().pin_memory()
+    hq, hk, hv, hdo, haq, hak, hb = (pin(t) for t in (q, k, v, do, aq, ak, b))
+    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory()] + \
+             [None if g is None else torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in grads]
+    e2e_steps = max(3, min(args.steps, 20))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, haq, hak, hb) if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h if t is not None)
+    e2e_ms = 0.0
+    for s in range(e2e_steps + 1):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for dst, src in zip((q, k, v, do, aq, ak, b), (hq, hk, hv, hdo, haq, hak, hb)):
+            if src is not None:
+                dst.copy_(src, non_blocking=True)
+        fwd()
+        bwd()
+        for dst, src in zip(outs_h, (o,) + grads):
+            if src is not None:
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if s > 0:
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms /= e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = tt.item()
+
+    if rank == 0:
+        peaks = load_peaks()
+        kf = kernel_flops(w)
+        cand = {ph: v for ph, v in phases.items() if ph in kf}
+        dom = max(cand, key=lambda ph: cand[ph][2]) if cand else None
+        roof = None
+        if dom:
+            calls, nk, tot = cand[dom]
+            avg_ms = tot / max(calls, 1)
+            achieved = kf[dom] / (avg_ms * 1e-3) / 1e12
+            tr = traffic_for(dom)
+            roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": tr,
+                    "peak_source": f"{peaks['source']} dense bf16 (burst); fp16 has the same nominal rate",
+                    "avg_launch_ms": avg_ms, "algorithmic_flops_per_launch": kf[dom]}
+        step_flops = (fwd_flops + bwd_flops) * world
+        ms = t_step / args.steps
+        value = step_flops / (ms * 1e-3) / 1e12
+        line = {
+            "metric": "useful TFLOP/s of one rel-pos attention layer (fwd+bwd), 8K x 12h x d64 fp16",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp16" if w.dtype == torch.float16 else "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, **{k_: v_ for k_, v_ in w.describe().items() if k_ != "workload"},
+                       "R_exp": R_exp, "l2": "flushed (256 MiB write) before every step",
+                       "parallelism": f"replicas x{world}"},
+            "passes": {
+                "fwd_ms": t_fwd / args.steps, "bwd_ms": t_bwd / args.steps,
+                "fwd_tflops": fwd_flops / (t_fwd / args.steps * 1e-3) / 1e12,
+                "bwd_tflops": bwd_flops / (t_bwd / args.steps * 1e-3) / 1e12,
+                "fwd_frac_of_peak": fwd_flops / (t_fwd / args.steps * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "bwd_frac_of_peak": bwd_flops / (t_bwd / args.steps * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            },
+            "phases_ms_per_step": {ph: v[2] / args.steps for ph, v in phases.items()},
+            "peak_mem_extra_bytes": int(peak_mem - input_bytes),
+            "roofline": roof,
+            "e2e": {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "wall_s_timed_region": wall,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, R_exp, seconds=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,41 @@
+"""Exact relative-position attention for B200 (sm_100a).
+
+    S_ij = tau (q_i.k_j + q_i.aQ_phi(i,j) + k_j.aK_phi(i,j) + b_phi(i,j)) + M_ij
+
+Shaw (truncated), Transformer-XL (identity), DeBERTa (log buckets) and T5
+(buckets) relative attention, forward and backward, computed by the CUDA
+library behind the C ABI in include/relpos_attn.h.  PyTorch supplies device
+memory and streams only.
+"""
+from ._binding import (  # noqa: F401
+    RelPosError, RelPosMap, debug_phi, debug_phi_device, debug_tile_plan, debug_tile_plan_device,
+    expanded_bounds, lib, relpos_attn_bwd, relpos_attn_fwd, table_rows, workspace_size,
+)
+
+import torch
+
+
+class RelPosAttention(torch.autograd.Function):
+    """Autograd wrapper: O = attention(q, k, v, aq, ak, b) through the CUDA library."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, aq, ak, b, tau, rmap, causal, key_len):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, lse = relpos_attn_fwd(q, k, v, aq, ak, b, tau=tau, map=rmap, causal=causal, key_len=key_len)
+        ctx.save_for_backward(q, k, v, o, lse, aq, ak, b, key_len)
+        ctx.cfg = (tau, rmap, causal)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse, aq, ak, b, key_len = ctx.saved_tensors
+        tau, rmap, causal = ctx.cfg
+        dq, dk, dv, daq, dak, db = relpos_attn_bwd(do.contiguous(), q, k, v, o, lse, aq, ak, b, tau=tau, map=rmap,
+                                                   causal=causal, key_len=key_len)
+        cast = lambda g, t: None if g is None else g.to(t.dtype)
+        return dq, dk, dv, cast(daq, aq), cast(dak, ak), db, None, None, None, None
+
+
+def relpos_attention(q, k, v, aq=None, ak=None, b=None, *, tau, map, causal=False, key_len=None):
+    """Differentiable exact relative-position attention (CUDA only)."""
+    return RelPosAttention.apply(q, k, v, aq, ak, b, tau, map, causal, key_len)

@@ -1,0 +1,463 @@
+// api.cu -- the C ABI (include/relpos_attn.h): argument validation, the host
+// planner (expanded offset range, projection group geometry, workspace
+// layout) and the launch sequence of the forward and backward passes.
+//
+// Forward  (digest of "Fast and Exact Relative-Position Attention via
+//           Structure-Aware Kernels", pipeline section):
+//   tables -> projection Z^Q, Z^K over reachable columns -> fused attention.
+// Backward (two-pass backward, Eq. (4)):
+//   tables -> projection -> D -> Q-parallel pass (dQ, dZ^Q) -> K-parallel pass
+//   (dK, dV, dZ^K) -> relation GEMMs, split sums and bucket fold.
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "kernels.cuh"
+
+#define RELPOS_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace relpos {
+static std::atomic<long long> g_kernel_launches{0};
+void note_launch(int n) { g_kernel_launches += n; }
+}  // namespace relpos
+
+using namespace relpos;
+
+namespace {
+
+// ---- optional per-phase event timing (relpos_profile_start / _stop)
+enum Phase { PH_TABLES, PH_PROJ, PH_FWD, PH_PREP, PH_DQ, PH_DKDV, PH_FOLD, PH_RELGRAD, PH_COUNT };
+const char* const kPhaseNames[PH_COUNT] = {"tables", "projection", "fwd_attention", "bwd_prep",
+                                           "bwd_dq", "bwd_dkdv", "fold_ranges", "relation_grads"};
+struct PhaseEvent {
+  int phase, kernels;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<PhaseEvent> g_prof_events;
+
+template <typename F>
+cudaError_t run_phase(int ph, cudaStream_t s, F&& f) {
+  if (!g_prof_on.load()) return f();
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return f();
+  const long long before = g_kernel_launches.load();
+  cudaEventRecord(a, s);
+  const cudaError_t e = f();
+  cudaEventRecord(b, s);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_events.push_back({ph, (int)(g_kernel_launches.load() - before), a, b});
+  return e;
+}
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return RELPOS_ERR_CUDA;
+}
+
+constexpr int kMaxN = 1 << 22;
+
+int check_map(const relpos_map_desc* m) {
+  if (!m) return RELPOS_ERR_INVALID_ARG;
+  switch (m->kind) {
+    case RELPOS_MAP_TRUNCATED:
+      return (m->clip >= 0 && m->clip <= kMaxN) ? RELPOS_OK : RELPOS_ERR_INVALID_ARG;
+    case RELPOS_MAP_IDENTITY:
+      return RELPOS_OK;
+    case RELPOS_MAP_BUCKET_T5: {
+      const int h = m->bidirectional ? m->num_buckets / 2 : m->num_buckets;
+      if (m->num_buckets < 2 || m->num_buckets > 65536 || h < 2) return RELPOS_ERR_INVALID_ARG;
+      if (m->max_distance <= h / 2) return RELPOS_ERR_INVALID_ARG;
+      return RELPOS_OK;
+    }
+    case RELPOS_MAP_BUCKET_LOG: {
+      if (m->num_buckets < 2 || m->num_buckets > 65536) return RELPOS_ERR_INVALID_ARG;
+      if (m->max_distance - 1 <= m->num_buckets / 2) return RELPOS_ERR_INVALID_ARG;
+      return RELPOS_OK;
+    }
+    default:
+      return RELPOS_ERR_UNSUPPORTED;
+  }
+}
+
+int rows_of(const relpos_map_desc& m, int N) {
+  switch (m.kind) {
+    case RELPOS_MAP_TRUNCATED: return 2 * m.clip + 1;
+    case RELPOS_MAP_IDENTITY: return 2 * N - 1;
+    case RELPOS_MAP_BUCKET_T5: return m.num_buckets;
+    default: return 2 * m.num_buckets;
+  }
+}
+
+// Leading / trailing runs of offsets that share one row (see header).
+void bounds_of(const relpos_map_desc& m, int N, int* lo, int* hi) {
+  if (m.kind == RELPOS_MAP_IDENTITY) { *lo = 1 - N; *hi = N - 1; return; }
+  if (m.kind == RELPOS_MAP_TRUNCATED) {
+    *lo = std::max(-m.clip, 1 - N);
+    *hi = std::min(m.clip, N - 1);
+    if (*hi < *lo) *hi = *lo;
+    // clip 0: every offset maps to row 0; the leading run covers everything
+    if (m.clip == 0) { *lo = N - 1; *hi = N - 1; }
+    return;
+  }
+  const int p0 = phi_of(m, N, 1 - N);
+  int d = 1 - N;
+  while (d + 1 <= N - 1 && phi_of(m, N, d + 1) == p0) ++d;
+  *lo = d;
+  const int p1 = phi_of(m, N, N - 1);
+  d = N - 1;
+  while (d - 1 >= 1 - N && phi_of(m, N, d - 1) == p1) --d;
+  *hi = std::max(d, *lo);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Layout {
+  size_t gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
+  size_t dsum, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
+  int R, Hq, expand, nsq, nsk, nsb;
+};
+
+int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
+  if (!a) return RELPOS_ERR_INVALID_ARG;
+  if (a->d != kHeadDim) return RELPOS_ERR_UNSUPPORTED;
+  if (a->dtype != RELPOS_F16 && a->dtype != RELPOS_BF16) return RELPOS_ERR_UNSUPPORTED;
+  if (a->out_dtype != a->dtype && a->out_dtype != RELPOS_F32) return RELPOS_ERR_UNSUPPORTED;
+  if (a->B < 1 || a->H < 1 || a->N < 1 || a->N > kMaxN) return RELPOS_ERR_INVALID_ARG;
+  if ((long long)a->B * a->H > 65535) return RELPOS_ERR_INVALID_ARG;
+  if (a->mask & ~(RELPOS_MASK_CAUSAL | RELPOS_MASK_KEY_PADDING)) return RELPOS_ERR_UNSUPPORTED;
+  if (!(a->tau == a->tau) || a->tau > 3.0e38f || a->tau < -3.0e38f) return RELPOS_ERR_INVALID_ARG;
+  int st = check_map(&a->map);
+  if (st) return st;
+  memset(p, 0, sizeof(*p));
+  memset(L, 0, sizeof(*L));
+  const int N = a->N;
+  p->B = a->B; p->H = a->H; p->N = N;
+  bounds_of(a->map, N, &p->E_lo, &p->E_hi);
+  p->Rexp = p->E_hi - p->E_lo + 1;
+  p->nT = (N + kTile - 1) / kTile;
+  p->grouped = p->Rexp > N + kTile - 1;
+  p->causal = (a->mask & RELPOS_MASK_CAUSAL) != 0;
+  p->padding = (a->mask & RELPOS_MASK_KEY_PADDING) != 0;
+  p->tau = a->tau;
+  const bool aq = a->aq != nullptr, ak = a->ak != nullptr, bb = a->b != nullptr;
+  const long long zq_head = head_elems(*p, 0), zk_head = head_elems(*p, 1);
+  p->zq_head = (aq || bb) ? zq_head : 0;
+  p->zk_head = ak ? zk_head : 0;
+  L->R = rows_of(a->map, N);
+  L->Hq = a->table_per_head ? a->H : 1;
+  L->expand = a->map.kind == RELPOS_MAP_BUCKET_T5 || a->map.kind == RELPOS_MAP_BUCKET_LOG;
+  const size_t BH = (size_t)a->B * a->H;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = up256(off + bytes); return o; };
+  L->gq = take(sizeof(GroupInfo) * p->nT);
+  L->gk = take(sizeof(GroupInfo) * p->nT);
+  L->phi = take(sizeof(int) * p->Rexp);
+  L->fold_lo = take(sizeof(int) * L->R);
+  L->fold_hi = take(sizeof(int) * L->R);
+  L->bexp = bb ? take(sizeof(float) * a->H * p->Rexp) : 0;
+  L->aqe = (aq && L->expand) ? take((size_t)2 * L->Hq * p->Rexp * 64) : 0;
+  L->ake = (ak && L->expand) ? take((size_t)2 * L->Hq * p->Rexp * 64) : 0;
+  L->zq = aq ? take(sizeof(float) * BH * p->zq_head) : 0;
+  L->zk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
+  L->fwd_end = off;
+  L->dsum = take(sizeof(float) * BH * N);
+  L->dzq = (aq || bb) ? take(sizeof(float) * BH * p->zq_head) : 0;
+  L->dzk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
+  L->dqacc = aq ? take(sizeof(float) * BH * N * 64) : 0;
+  L->dkacc = ak ? take(sizeof(float) * BH * N * 64) : 0;
+  const int nE = (p->Rexp + 63) / 64;
+  const long long items = a->table_per_head ? (long long)a->B * p->nT : (long long)BH * p->nT;
+  auto pick = [](long long want, long long items_) {
+    long long s = std::max(1LL, want);
+    s = std::min(s, items_);
+    s = std::min(s, 256LL);
+    return (int)std::max(1LL, s);
+  };
+  L->nsq = pick(296LL / ((long long)nE * L->Hq), items);
+  L->nsk = L->nsq;
+  L->nsb = pick(296LL / ((long long)((p->Rexp + 255) / 256) * a->H), (long long)a->B * p->nT);
+  L->daqp = aq ? take(sizeof(float) * (size_t)L->nsq * L->Hq * p->Rexp * 64) : 0;
+  L->dakp = ak ? take(sizeof(float) * (size_t)L->nsk * L->Hq * p->Rexp * 64) : 0;
+  L->dbp = bb ? take(sizeof(float) * (size_t)L->nsb * a->H * p->Rexp) : 0;
+  L->bwd_end = off;
+  return RELPOS_OK;
+}
+
+int check_fwd_ptrs(const relpos_fwd_args* a) {
+  if (!a->q || !a->k || !a->v || !a->o || !a->lse) return RELPOS_ERR_INVALID_ARG;
+  if ((a->mask & RELPOS_MASK_KEY_PADDING) && !a->key_len) return RELPOS_ERR_INVALID_ARG;
+  const void* al[] = {a->q, a->k, a->v, a->o, a->aq, a->ak};
+  for (const void* x : al)
+    if (x && !aligned16(x)) return RELPOS_ERR_INVALID_ARG;
+  return RELPOS_OK;
+}
+
+// Resolve workspace regions and the expanded-table pointers; launch the
+// table builder and the projections (shared by forward and backward).
+int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Tensors& t, cudaStream_t s) {
+  memset(&t, 0, sizeof(t));
+  GroupInfo* gq = reinterpret_cast<GroupInfo*>(ws + L.gq);
+  GroupInfo* gk = reinterpret_cast<GroupInfo*>(ws + L.gk);
+  p.gq = gq;
+  p.gk = gk;
+  p.key_len = a->key_len;
+  t.q = a->q; t.k = a->k; t.v = a->v;
+  t.o = a->o; t.o_f32 = a->out_dtype == RELPOS_F32; t.lse = a->lse;
+  t.is_bf16 = a->dtype == RELPOS_BF16;
+  t.table_per_head = a->table_per_head;
+  t.R = L.R;
+  int* phi_exp = reinterpret_cast<int*>(ws + L.phi);
+  t.phi_exp = phi_exp;
+  t.fold_lo = reinterpret_cast<int*>(ws + L.fold_lo);
+  t.fold_hi = reinterpret_cast<int*>(ws + L.fold_hi);
+  if (a->b) t.b_exp = reinterpret_cast<float*>(ws + L.bexp);
+  // expanded-table row e <-> offset E_lo + e
+  long long row0 = 0;
+  if (a->map.kind == RELPOS_MAP_TRUNCATED) row0 = (long long)p.E_lo + a->map.clip;
+  else if (a->map.kind == RELPOS_MAP_IDENTITY) row0 = (long long)p.E_lo + a->N - 1;
+  const size_t esz = 2;
+  if (a->aq) {
+    if (L.expand) { t.aq_exp = ws + L.aqe; t.aq_hs = (long long)p.Rexp * 64; }
+    else { t.aq_exp = static_cast<const uint8_t*>(a->aq) + row0 * 64 * esz; t.aq_hs = (long long)L.R * 64; }
+    t.zq = reinterpret_cast<float*>(ws + L.zq);
+  }
+  if (a->ak) {
+    if (L.expand) { t.ak_exp = ws + L.ake; t.ak_hs = (long long)p.Rexp * 64; }
+    else { t.ak_exp = static_cast<const uint8_t*>(a->ak) + row0 * 64 * esz; t.ak_hs = (long long)L.R * 64; }
+    t.zk = reinterpret_cast<float*>(ws + L.zk);
+  }
+  cudaError_t e = run_phase(PH_TABLES, s, [&] {
+    return launch_build_tables(p, a->map, gq, gk, phi_exp, L.R, a->aq, a->ak, a->table_per_head, ws + L.aqe,
+                               ws + L.ake, a->b, const_cast<float*>(t.b_exp), t.is_bf16, L.expand, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (a->aq || a->ak) {
+    e = run_phase(PH_PROJ, s, [&] { return launch_projection(p, t, s); });
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return RELPOS_OK;
+}
+
+}  // namespace
+
+RELPOS_EXPORT int relpos_table_rows(const relpos_map_desc* map, int32_t N, int32_t* R_out) {
+  if (!map || !R_out || N < 1 || N > kMaxN) return RELPOS_ERR_INVALID_ARG;
+  const int st = check_map(map);
+  if (st) return st;
+  *R_out = rows_of(*map, N);
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_expanded_bounds(const relpos_map_desc* map, int32_t N, int32_t* e_lo, int32_t* e_hi) {
+  if (!map || !e_lo || !e_hi || N < 1 || N > kMaxN) return RELPOS_ERR_INVALID_ARG;
+  const int st = check_map(map);
+  if (st) return st;
+  bounds_of(*map, N, e_lo, e_hi);
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_workspace_size(const relpos_fwd_args* a, size_t* fwd_bytes, size_t* bwd_bytes) {
+  Plan p;
+  Layout L;
+  const int st = make_plan(a, &p, &L);
+  if (st) return st;
+  if (fwd_bytes) *fwd_bytes = L.fwd_end;
+  if (bwd_bytes) *bwd_bytes = L.bwd_end;
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_attn_fwd(const relpos_fwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream) {
+  Plan p;
+  Layout L;
+  int st = make_plan(a, &p, &L);
+  if (st) return st;
+  st = check_fwd_ptrs(a);
+  if (st) return st;
+  if (!workspace || ws_bytes < L.fwd_end || (reinterpret_cast<uintptr_t>(workspace) & 255)) return RELPOS_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Tensors t;
+  st = prepare(a, p, L, static_cast<uint8_t*>(workspace), t, s);
+  if (st) return st;
+  const cudaError_t e = run_phase(PH_FWD, s, [&] { return launch_forward(p, t, s); });
+  if (e != cudaSuccess) return cuda_fail(e);
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, size_t ws_bytes, relpos_stream_t stream) {
+  if (!g) return RELPOS_ERR_INVALID_ARG;
+  const relpos_fwd_args* a = &g->fwd;
+  Plan p;
+  Layout L;
+  int st = make_plan(a, &p, &L);
+  if (st) return st;
+  st = check_fwd_ptrs(a);
+  if (st) return st;
+  if (!g->dout || !g->dq || !g->dk || !g->dv) return RELPOS_ERR_INVALID_ARG;
+  if ((a->aq && !g->daq) || (a->ak && !g->dak) || (a->b && !g->db)) return RELPOS_ERR_INVALID_ARG;
+  const void* al[] = {g->dout, g->dq, g->dk, g->dv, g->daq, g->dak, g->db};
+  for (const void* x : al)
+    if (x && !aligned16(x)) return RELPOS_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < L.bwd_end || (reinterpret_cast<uintptr_t>(workspace) & 255)) return RELPOS_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  Tensors t;
+  st = prepare(a, p, L, ws, t, s);
+  if (st) return st;
+  t.dout = g->dout;
+  t.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  t.dq = g->dq; t.dk = g->dk; t.dv = g->dv;
+  t.daq = g->daq; t.dak = g->dak; t.db = g->db;
+  const size_t BH = (size_t)a->B * a->H;
+  cudaError_t e;
+  if (a->aq || a->b) {
+    t.dzq = reinterpret_cast<float*>(ws + L.dzq);
+    e = cudaMemsetAsync(t.dzq, 0, sizeof(float) * BH * p.zq_head, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (a->ak) {
+    t.dzk = reinterpret_cast<float*>(ws + L.dzk);
+    e = cudaMemsetAsync(t.dzk, 0, sizeof(float) * BH * p.zk_head, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (a->aq) { t.dq_acc = reinterpret_cast<float*>(ws + L.dqacc); t.daq_part = reinterpret_cast<float*>(ws + L.daqp); }
+  if (a->ak) { t.dk_acc = reinterpret_cast<float*>(ws + L.dkacc); t.dak_part = reinterpret_cast<float*>(ws + L.dakp); }
+  if (a->b) t.db_part = reinterpret_cast<float*>(ws + L.dbp);
+  t.nsplit_q = L.nsq; t.nsplit_k = L.nsk; t.nsplit_b = L.nsb;
+  if ((e = run_phase(PH_PREP, s, [&] { return launch_bwd_prep(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  if ((e = run_phase(PH_DQ, s, [&] { return launch_bwd_dq(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  if ((e = run_phase(PH_DKDV, s, [&] { return launch_bwd_dkdv(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  if (a->aq || a->ak || a->b) {
+    e = run_phase(PH_FOLD, s, [&] { return launch_fold_ranges(p, t.phi_exp, L.R, t.fold_lo, t.fold_hi, s); });
+    if (e != cudaSuccess) return cuda_fail(e);
+    if ((e = run_phase(PH_RELGRAD, s, [&] { return launch_relgrad(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  }
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT const char* relpos_status_string(int status) {
+  switch (status) {
+    case RELPOS_OK: return "ok";
+    case RELPOS_ERR_INVALID_ARG: return "invalid argument";
+    case RELPOS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RELPOS_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case RELPOS_ERR_CUDA: return "CUDA error (see relpos_last_cuda_error)";
+    case RELPOS_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+RELPOS_EXPORT int relpos_last_cuda_error(void) { return g_last_cuda_error; }
+
+RELPOS_EXPORT int relpos_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& ev : g_prof_events) {
+    cudaEventDestroy(ev.a);
+    cudaEventDestroy(ev.b);
+  }
+  g_prof_events.clear();
+  g_prof_on = true;
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_profile_stop(relpos_phase_stat* stats, int32_t max_stats, int32_t* n_stats) {
+  g_prof_on = false;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  relpos_phase_stat agg[PH_COUNT];
+  memset(agg, 0, sizeof(agg));
+  int status = RELPOS_OK;
+  for (auto& ev : g_prof_events) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(ev.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, ev.a, ev.b);
+    if (e != cudaSuccess) status = cuda_fail(e);
+    agg[ev.phase].calls += 1;
+    agg[ev.phase].kernels += ev.kernels;
+    agg[ev.phase].total_ms += ms;
+    cudaEventDestroy(ev.a);
+    cudaEventDestroy(ev.b);
+  }
+  g_prof_events.clear();
+  int n = 0;
+  for (int ph = 0; ph < PH_COUNT; ++ph) {
+    if (agg[ph].calls == 0) continue;
+    strncpy(agg[ph].name, kPhaseNames[ph], sizeof(agg[ph].name) - 1);
+    if (stats && n < max_stats) stats[n] = agg[ph];
+    ++n;
+  }
+  if (n_stats) *n_stats = n;
+  return status;
+}
+
+RELPOS_EXPORT int64_t relpos_kernel_launches(void) { return g_kernel_launches.load(); }
+
+RELPOS_EXPORT int relpos_debug_phi(const relpos_map_desc* map, int32_t N, int32_t* phi_host) {
+  if (!map || !phi_host || N < 1 || N > 46340) return RELPOS_ERR_INVALID_ARG;
+  const int st = check_map(map);
+  if (st) return st;
+  std::vector<int> by_delta(2 * (size_t)N - 1);
+  for (int d = 1 - N; d <= N - 1; ++d) by_delta[d + N - 1] = phi_of(*map, N, d);
+  for (int i = 0; i < N; ++i)
+    for (int j = 0; j < N; ++j) phi_host[(size_t)i * N + j] = by_delta[j - i + N - 1];
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_debug_phi_device(const relpos_map_desc* map, int32_t N, int32_t* phi_dev, relpos_stream_t stream) {
+  if (!map || !phi_dev || N < 1 || N > kMaxN) return RELPOS_ERR_INVALID_ARG;
+  const int st = check_map(map);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_debug_phi(*map, N, phi_dev, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return e == cudaSuccess ? RELPOS_OK : cuda_fail(e);
+}
+
+RELPOS_EXPORT int relpos_debug_tile_plan(const relpos_map_desc* map, int32_t B, int32_t N, int32_t mask,
+                                         const int32_t* key_len_host, int32_t* classes_host, int32_t* segs_host) {
+  if (!map || !classes_host || !segs_host || B < 1 || N < 1 || N > kMaxN) return RELPOS_ERR_INVALID_ARG;
+  if (mask & ~(RELPOS_MASK_CAUSAL | RELPOS_MASK_KEY_PADDING)) return RELPOS_ERR_UNSUPPORTED;
+  if ((mask & RELPOS_MASK_KEY_PADDING) && !key_len_host) return RELPOS_ERR_INVALID_ARG;
+  const int st = check_map(map);
+  if (st) return st;
+  int lo, hi;
+  bounds_of(*map, N, &lo, &hi);
+  const int nT = (N + kTile - 1) / kTile;
+  const int causal = (mask & RELPOS_MASK_CAUSAL) != 0;
+  for (int b = 0; b < B; ++b) {
+    const int nkv = (mask & RELPOS_MASK_KEY_PADDING) ? key_len_host[b] : N;
+    for (int qi = 0; qi < nT; ++qi) {
+      for (int kj = 0; kj < nT; ++kj)
+        classes_host[((size_t)b * nT + qi) * nT + kj] = tile_class(qi, kj, N, nkv, causal, lo, hi);
+      int sg[4];
+      tile_segments(qi, nT, N, nkv, causal, lo, hi, sg);
+      for (int c = 0; c < 4; ++c) segs_host[((size_t)b * nT + qi) * 4 + c] = sg[c];
+    }
+  }
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_debug_tile_plan_device(const relpos_map_desc* map, int32_t B, int32_t N, int32_t mask,
+                                                const int32_t* key_len_dev, int32_t* classes_dev, int32_t* segs_dev,
+                                                relpos_stream_t stream) {
+  if (!map || !classes_dev || !segs_dev || B < 1 || N < 1 || N > kMaxN) return RELPOS_ERR_INVALID_ARG;
+  if (mask & ~(RELPOS_MASK_CAUSAL | RELPOS_MASK_KEY_PADDING)) return RELPOS_ERR_UNSUPPORTED;
+  if ((mask & RELPOS_MASK_KEY_PADDING) && !key_len_dev) return RELPOS_ERR_INVALID_ARG;
+  const int st = check_map(map);
+  if (st) return st;
+  int lo, hi;
+  bounds_of(*map, N, &lo, &hi);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_debug_tile_plan(B, N, (mask & RELPOS_MASK_CAUSAL) != 0,
+                                         (mask & RELPOS_MASK_KEY_PADDING) ? key_len_dev : nullptr, lo, hi,
+                                         classes_dev, segs_dev, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return e == cudaSuccess ? RELPOS_OK : cuda_fail(e);
+}

@@ -1,0 +1,197 @@
+// common.cuh -- shared definitions of the relative-position attention library:
+// offset maps, the expanded (bucket -> truncated) form, projection group
+// geometry and the tile plan.  Host and device use the same functions, so the
+// planner and the kernels agree by construction.
+//
+// Source: digest page of "Fast and Exact Relative-Position Attention via
+// Structure-Aware Kernels" -- Eq. (1)-(3), sections "grouped reachable range"
+// and "constant tiles and the saturated region".
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/relpos_attn.h"
+
+#define RP_HD __host__ __device__ __forceinline__
+
+namespace relpos {
+
+constexpr int kTile = RELPOS_TILE;   // tile edge and projection group size (128)
+constexpr int kHeadDim = 64;
+constexpr double kGuard = 1e-9;      // exact integer crossings of the log formulas round as in exact arithmetic
+
+RP_HD int imin(int a, int b) { return a < b ? a : b; }
+RP_HD int imax(int a, int b) { return a > b ? a : b; }
+RP_HD int iclamp(int x, int lo, int hi) { return imin(imax(x, lo), hi); }
+RP_HD int round_up4(int x) { return (x + 3) & ~3; }
+
+// ---------------------------------------------------------------------------
+// Offset maps phi(delta), delta = j - i.
+// ---------------------------------------------------------------------------
+
+// T5 buckets: half of the buckets per direction when bidirectional; within a
+// half of size h, magnitudes below h/2 are exact and larger ones fall into
+// h/2 + floor(ln(n/(h/2)) / ln(max_distance/(h/2)) * (h/2)) capped at h-1.
+RP_HD int phi_t5(int delta, int num_buckets, int max_distance, int bidirectional) {
+  int h = num_buckets, base = 0, n;
+  if (bidirectional) {
+    h = num_buckets / 2;
+    base = delta > 0 ? h : 0;
+    n = delta < 0 ? -delta : delta;
+  } else {
+    n = delta < 0 ? -delta : 0;
+  }
+  const int exact = h / 2;
+  if (n < exact) return base + n;
+  const double x = log((double)n / (double)exact) / log((double)max_distance / (double)exact) *
+                   (double)(h - exact);
+  const int large = exact + (int)floor(x + kGuard);
+  return base + imin(large, h - 1);
+}
+
+// DeBERTa log buckets: |delta| <= mid = num_buckets/2 keeps the offset, beyond
+// it sign * (mid + ceil(ln(n/mid) / ln((max_distance-1)/mid) * (mid-1)));
+// the row is that position + num_buckets clamped to [0, 2 num_buckets).
+RP_HD int phi_log(int delta, int num_buckets, int max_distance) {
+  const int mid = num_buckets / 2;
+  const int n = delta < 0 ? -delta : delta;
+  int pos = delta;
+  if (n > mid) {
+    const double x = log((double)n / (double)mid) / log((double)(max_distance - 1) / (double)mid) *
+                     (double)(mid - 1);
+    const int lp = mid + (int)ceil(x - kGuard);
+    pos = delta < 0 ? -lp : lp;
+  }
+  return iclamp(pos + num_buckets, 0, 2 * num_buckets - 1);
+}
+
+RP_HD int phi_of(const relpos_map_desc& m, int N, int delta) {
+  switch (m.kind) {
+    case RELPOS_MAP_TRUNCATED: return iclamp(delta, -m.clip, m.clip) + m.clip;
+    case RELPOS_MAP_IDENTITY: return delta + N - 1;
+    case RELPOS_MAP_BUCKET_T5: return phi_t5(delta, m.num_buckets, m.max_distance, m.bidirectional);
+    default: return phi_log(delta, m.num_buckets, m.max_distance);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Plan passed by value to every kernel.
+// ---------------------------------------------------------------------------
+
+// Projection geometry of one 128-row group: its rows store the expanded
+// columns [e0, e0 + W) with a row stride of S floats, starting `base` floats
+// into the (batch, head) slice.
+struct GroupInfo {
+  int e0, W, S, pad;
+  long long base;
+};
+
+struct Plan {
+  int B, H, N;
+  int E_lo, E_hi, Rexp;     // expanded offset range [E_lo, E_hi]; expanded row e = clamp(delta) - E_lo
+  int nT;                   // number of 128-row tiles / groups
+  int grouped;              // 1: per-group reachable columns; 0: every row stores all Rexp columns
+  int causal, padding;
+  float tau;
+  long long zq_head, zk_head;   // floats per (batch, head) of Z^Q / Z^K (0 when absent)
+  const GroupInfo* gq;          // device [nT]
+  const GroupInfo* gk;          // device [nT]
+  const int* key_len;           // device [B] or null
+};
+
+// Reachable expanded columns of query group g (key_side = 0) or key group g
+// (key_side = 1): a query i reaches delta in [-i, N-1-i], a key j reaches
+// [j-(N-1), j]; causal keeps delta <= 0.
+RP_HD void group_columns(const Plan& p, int key_side, int g, int* e0, int* W) {
+  if (!p.grouped) { *e0 = 0; *W = p.Rexp; return; }
+  const int r0 = g * kTile, n = imin(kTile, p.N - r0);
+  int lo, hi;
+  if (!key_side) { lo = -(r0 + n - 1); hi = p.N - 1 - r0; }
+  else { lo = r0 - (p.N - 1); hi = r0 + n - 1; }
+  if (p.causal) hi = imin(hi, 0);
+  lo = imax(lo, p.E_lo);
+  hi = imin(hi, p.E_hi);
+  if (hi < lo) hi = lo;
+  *e0 = lo - p.E_lo;
+  *W = hi - lo + 1;
+}
+
+// Fills GroupInfo for group g (prefix sum over the preceding groups).
+RP_HD GroupInfo group_info(const Plan& p, int key_side, int g) {
+  GroupInfo gi;
+  long long base = 0;
+  for (int t = 0; t < g; ++t) {
+    int e0, W;
+    group_columns(p, key_side, t, &e0, &W);
+    base += (long long)imin(kTile, p.N - t * kTile) * round_up4(W);
+  }
+  group_columns(p, key_side, g, &gi.e0, &gi.W);
+  gi.S = round_up4(gi.W);
+  gi.pad = 0;
+  gi.base = base;
+  return gi;
+}
+
+RP_HD long long head_elems(const Plan& p, int key_side) {
+  if (p.nT == 0) return 0;
+  GroupInfo last = group_info(p, key_side, p.nT - 1);
+  return last.base + (long long)imin(kTile, p.N - (p.nT - 1) * kTile) * last.S;
+}
+
+// ---------------------------------------------------------------------------
+// Tile plan: the two comparisons of a tile's offset range with (E_lo, E_hi).
+// ---------------------------------------------------------------------------
+RP_HD int tile_class(int qi, int kj, int N, int nkv, int causal, int E_lo, int E_hi) {
+  const int i0 = qi * kTile, i1 = imin(i0 + kTile, N) - 1;
+  const int j0 = kj * kTile, j1 = imin(j0 + kTile, N) - 1;
+  if (j0 >= nkv || (causal && j0 > i1)) return RELPOS_TILE_MASKED;
+  const int j1v = imin(j1, nkv - 1);
+  if (j1v - i0 <= E_lo) return RELPOS_TILE_CONST_LO;
+  if (j0 - i1 >= E_hi) return RELPOS_TILE_CONST_HI;
+  return RELPOS_TILE_BAND;
+}
+
+// Segments of query tile qi: key tiles [0, lo_end) are CONST_LO, [lo_end,
+// band_end) BAND, [band_end, live_end) CONST_HI, [live_end, nT) MASKED.
+// Classes are monotone in kj (the offset range grows with kj and the
+// masked tiles are the tail), so the bounds come from counting.
+RP_HD void tile_segments(int qi, int nT, int N, int nkv, int causal, int E_lo, int E_hi, int seg[4]) {
+  int nlo = 0, nband = 0, nhi = 0;
+  for (int kj = 0; kj < nT; ++kj) {
+    const int c = tile_class(qi, kj, N, nkv, causal, E_lo, E_hi);
+    nlo += c == RELPOS_TILE_CONST_LO;
+    nband += c == RELPOS_TILE_BAND;
+    nhi += c == RELPOS_TILE_CONST_HI;
+  }
+  seg[0] = nlo;
+  seg[1] = nlo + nband;
+  seg[2] = nlo + nband + nhi;
+  seg[3] = nT;
+}
+
+template <typename T> struct DT;
+template <> struct DT<__half> {
+  static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+  static __device__ __forceinline__ __half from_f(float x) { return __float2half_rn(x); }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+template <> struct DT<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+}  // namespace relpos

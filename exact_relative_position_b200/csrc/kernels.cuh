@@ -1,0 +1,56 @@
+// kernels.cuh -- launch wrappers of the library's kernels (one translation
+// unit per kernel family) and the parameter blocks they take.
+#pragma once
+
+#include "common.cuh"
+
+namespace relpos {
+
+// Device pointers of one forward/backward call, resolved into the workspace.
+struct Tensors {
+  const void *q, *k, *v;
+  const void *aq_exp, *ak_exp;   // expanded tables, [Hq][Rexp][64] (Hq = H or 1), or null
+  int table_per_head;
+  long long aq_hs, ak_hs;        // head stride (elements) of the expanded tables when per head
+  const float* b_exp;            // [H][Rexp] or null
+  float *zq, *zk;                // projections (grouped layout), or null
+  void* o;
+  int o_f32;
+  float* lse;
+  // backward
+  const void* dout;
+  float* dsum;                   // D_i = sum_c dO_ic O_ic, [B,H,N]
+  float *dzq, *dzk;              // offset-sharded relation gradients (same layout as zq/zk)
+  void *dq, *dk, *dv;
+  float *dq_acc, *dk_acc;        // fp32 [B,H,N,64] before the relation-GEMM epilogue (or null)
+  float *daq_part, *dak_part;    // [nsplit][Hq][Rexp][64] partial table gradients
+  float* db_part;                // [nsplit][H][Rexp]
+  int nsplit_q, nsplit_k, nsplit_b;
+  float *daq_exp, *dak_exp, *db_exp_grad;   // summed expanded-table gradients
+  const int* phi_exp;            // [Rexp] expanded row -> original table row
+  int* fold_lo;                  // [R] first expanded row of each table row
+  int* fold_hi;                  // [R] one past its last expanded row
+  int R;
+  float *daq, *dak, *db;         // final outputs
+  int is_bf16;
+};
+
+// Counts kernel launches (process-wide, reported by relpos_kernel_launches).
+void note_launch(int n);
+
+cudaError_t launch_build_tables(const Plan& p, const relpos_map_desc& map, GroupInfo* gq, GroupInfo* gk,
+                                int* phi_exp, int R, const void* aq, const void* ak, int table_per_head,
+                                void* aq_exp, void* ak_exp, const float* b, float* b_exp, int is_bf16,
+                                int expand_tables, cudaStream_t s);
+cudaError_t launch_fold_ranges(const Plan& p, const int* phi_exp, int R, int* fold_lo, int* fold_hi, cudaStream_t s);
+cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_forward(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_bwd_dkdv(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_relgrad(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_debug_phi(const relpos_map_desc& map, int N, int* out, cudaStream_t s);
+cudaError_t launch_debug_tile_plan(int B, int N, int causal, const int* key_len, int E_lo, int E_hi,
+                                   int* classes, int* segs, cudaStream_t s);
+
+}  // namespace relpos

@@ -1,0 +1,407 @@
+// relation.cu -- relation-table side of exact relative-position attention
+// (digest of "Fast and Exact Relative-Position Attention via Structure-Aware
+// Kernels": Eq. (3), "grouped reachable range", "constant tiles and the
+// saturated region" and the table-gradient GEMMs of the backward section).
+//
+//  * tables:      group geometry, expanded row -> table row map, expanded
+//                 bias and (for bucketed maps) the expanded aQ/aK tables in
+//                 which every bucket row is copied once per offset it covers.
+//  * projection:  Z = X A_exp^T for every 128-row group over its reachable
+//                 columns only (dense tensor-core GEMM, K = head dim).
+//  * relgrad:     dQ += dZ^Q A_exp and dK += dZ^K A_exp (row epilogue),
+//                 dA_exp = sum dZ^T X per fixed split of (batch, head, group),
+//                 db_exp = column sums of dZ^Q, then a deterministic final
+//                 pass that sums the splits in order and folds the copy
+//                 columns of a bucket back into that bucket in ascending
+//                 offset order.  No atomics.
+#include "kernels.cuh"
+#include "warp_mma.cuh"
+
+namespace relpos {
+
+namespace {
+
+// ------------------------------------------------------------------ tables
+__global__ void groups_kernel(const Plan p, GroupInfo* gq, GroupInfo* gk) {
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= p.nT) return;
+  gq[g] = group_info(p, 0, g);
+  gk[g] = group_info(p, 1, g);
+}
+
+__global__ void phi_exp_kernel(const relpos_map_desc map, const int N, const int E_lo, const int Rexp, int* phi_exp) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < Rexp) phi_exp[e] = phi_of(map, N, E_lo + e);
+}
+
+__global__ void bias_exp_kernel(const relpos_map_desc map, const int N, const int E_lo, const int Rexp, const int R,
+                                const int H, const float* __restrict__ b, float* __restrict__ b_exp) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)H * Rexp) return;
+  const int h = (int)(idx / Rexp), e = (int)(idx - (long long)h * Rexp);
+  b_exp[idx] = b[(size_t)h * R + phi_of(map, N, E_lo + e)];
+}
+
+// Copy of table row phi(E_lo + e) into expanded row e (16-byte chunks).
+__global__ void table_exp_kernel(const relpos_map_desc map, const int N, const int E_lo, const int Rexp, const int R,
+                                 const int Hq, const uint4* __restrict__ src, uint4* __restrict__ dst) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long total = (long long)Hq * Rexp * 8;
+  if (idx >= total) return;
+  const int c = (int)(idx & 7);
+  const long long row = idx >> 3;
+  const int h = (int)(row / Rexp), e = (int)(row - (long long)h * Rexp);
+  const int r = phi_of(map, N, E_lo + e);
+  dst[idx] = src[((size_t)h * R + r) * 8 + c];
+}
+
+__global__ void fold_mark_kernel(const int* __restrict__ phi_exp, const int Rexp, int* fold_lo, int* fold_hi) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= Rexp) return;
+  const int r = phi_exp[e];
+  if (e == 0 || phi_exp[e - 1] != r) fold_lo[r] = e;
+  if (e == Rexp - 1 || phi_exp[e + 1] != r) fold_hi[r] = e + 1;
+}
+
+// ------------------------------------------------------------------ projection
+// Z[b,h, group g rows, columns e0 + [c0, c0 + 64)] = X_rows A_exp[e0 + c0 ..]^T
+constexpr int kProjSmem = 128 * 128 + 64 * 128;
+
+template <typename T>
+__global__ void __launch_bounds__(256) projection_kernel(const Plan p, const int key_side, const T* __restrict__ X,
+                                                         const T* __restrict__ A, const long long a_hs,
+                                                         float* __restrict__ Z, const long long z_head) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
+  const int h = bh % p.H;
+  const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
+  const int c0 = chunk * 64;
+  if (c0 >= gi.W) return;
+  const int r0 = g * kTile;
+  const uint32_t sX = smem_u32(smem), sA = sX + 128 * 128;
+  const T* Xh = X + (size_t)bh * p.N * 64;
+  const T* Ah = A + (size_t)h * a_hs + (size_t)(gi.e0 + c0) * 64;
+  load_tile_async<128, 256>(sX, Xh, r0, p.N, tid);
+  load_tile_async<64, 256>(sA, Ah, 0, gi.W - c0, tid);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  uint32_t xa[4][4];
+  load_a_frags(sX, warp * 16, lane, xa);
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  mma_abt<T, 8>(acc, xa, sA, 0, lane);
+  const int g8 = lane >> 2, tq = lane & 3;
+  float* Zg = Z + (size_t)bh * z_head + gi.base;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const int rr = warp * 16 + g8 + 8 * hf;
+    if (r0 + rr >= p.N) continue;
+    float* zrow = Zg + (long long)rr * gi.S;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int col = c0 + nt * 8 + 2 * tq;
+      if (col < gi.W) *reinterpret_cast<float2*>(zrow + col) = make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ relgrad rows
+// out[rows of group g] = acc_in[rows] + dZ_g[rows, :W] A_exp[e0 .. e0 + W)   (tf32 tensor cores)
+constexpr int kRowPitchA = 36;   // floats, dZ chunk [128][32]
+constexpr int kRowPitchB = 72;   // floats, table chunk [32][64]
+
+template <typename T>
+__global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
+                                                           const long long z_head, const T* __restrict__ A,
+                                                           const long long a_hs, const float* __restrict__ acc_in,
+                                                           T* __restrict__ out) {
+  __shared__ float As[128 * kRowPitchA];
+  __shared__ float Bs[32 * kRowPitchB];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.x, bh = blockIdx.y, h = bh % p.H;
+  const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
+  const int r0 = g * kTile;
+  const int nrows = imin(kTile, p.N - r0);
+  const float* Zg = dZ + (size_t)bh * z_head + gi.base;
+  const T* Ah = A + (size_t)h * a_hs + (size_t)gi.e0 * 64;
+  const int g8 = lane >> 2, tq = lane & 3;
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  for (int c0 = 0; c0 < gi.W; c0 += 32) {
+    for (int idx = tid; idx < 128 * 32; idx += 256) {
+      const int r = idx >> 5, c = idx & 31;
+      As[r * kRowPitchA + c] = (r < nrows && c0 + c < gi.W) ? Zg[(long long)r * gi.S + c0 + c] : 0.f;
+    }
+    for (int idx = tid; idx < 32 * 64; idx += 256) {
+      const int r = idx >> 6, c = idx & 63;
+      Bs[r * kRowPitchB + c] = (c0 + r < gi.W) ? DT<T>::to_f(Ah[(size_t)(c0 + r) * 64 + c]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const int rb = warp * 16;
+      const uint32_t a0 = to_tf32(As[(rb + g8) * kRowPitchA + ks * 8 + tq]);
+      const uint32_t a1 = to_tf32(As[(rb + g8 + 8) * kRowPitchA + ks * 8 + tq]);
+      const uint32_t a2 = to_tf32(As[(rb + g8) * kRowPitchA + ks * 8 + tq + 4]);
+      const uint32_t a3 = to_tf32(As[(rb + g8 + 8) * kRowPitchA + ks * 8 + tq + 4]);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const uint32_t b0 = to_tf32(Bs[(ks * 8 + tq) * kRowPitchB + nt * 8 + g8]);
+        const uint32_t b1 = to_tf32(Bs[(ks * 8 + tq + 4) * kRowPitchB + nt * 8 + g8]);
+        mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    __syncthreads();
+  }
+  const size_t off = (size_t)bh * p.N * 64;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const int rr = warp * 16 + g8 + 8 * hf;
+    if (rr >= nrows) continue;
+    const size_t ro = off + (size_t)(r0 + rr) * 64;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int c = nt * 8 + 2 * tq;
+      const float2 base = *reinterpret_cast<const float2*>(acc_in + ro + c);
+      *reinterpret_cast<uint32_t*>(out + ro + c) = DT<T>::pack(base.x + acc[nt][2 * hf], base.y + acc[nt][2 * hf + 1]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ table partials
+// part[s][hq][c0 + m][:] = sum over the split's (batch, head, group) items, in
+// order, of dZ_g[rows, c0 + m - e0] X[rows, :]   (tf32 tensor cores)
+template <typename T>
+__global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
+                                                         const long long z_head, const T* __restrict__ X,
+                                                         const int per_head, const int nsplit,
+                                                         float* __restrict__ part) {
+  __shared__ float Zs[32 * kRowPitchB];   // [rows][e]
+  __shared__ float Xs[32 * kRowPitchB];   // [rows][d]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c0 = blockIdx.x * 64, hq = blockIdx.y, s = blockIdx.z;
+  const int Hq = per_head ? p.H : 1;
+  const long long nitems = per_head ? (long long)p.B * p.nT : (long long)p.B * p.H * p.nT;
+  const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
+  const int g8 = lane >> 2, tq = lane & 3;
+  const int eb = (warp & 3) * 16, db = (warp >> 2) * 32;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  for (long long it = it0; it < it1; ++it) {
+    int bh, g;
+    if (per_head) {
+      const int b = (int)(it / p.nT);
+      g = (int)(it - (long long)b * p.nT);
+      bh = b * p.H + hq;
+    } else {
+      bh = (int)(it / p.nT);
+      g = (int)(it - (long long)bh * p.nT);
+    }
+    const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
+    if (c0 + 64 <= gi.e0 || c0 >= gi.e0 + gi.W) continue;   // block-uniform
+    const int r0 = g * kTile, nrows = imin(kTile, p.N - r0);
+    const float* Zg = dZ + (size_t)bh * z_head + gi.base;
+    const T* Xg = X + (size_t)bh * p.N * 64 + (size_t)r0 * 64;
+    for (int rc = 0; rc < nrows; rc += 32) {
+      for (int idx = tid; idx < 32 * 64; idx += 256) {
+        const int r = idx >> 6, c = idx & 63;
+        const int col = c0 + c - gi.e0;
+        const bool ok = (rc + r < nrows) && col >= 0 && col < gi.W;
+        Zs[r * kRowPitchB + c] = ok ? Zg[(long long)(rc + r) * gi.S + col] : 0.f;
+        Xs[r * kRowPitchB + c] = (rc + r < nrows) ? DT<T>::to_f(Xg[(size_t)(rc + r) * 64 + c]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint32_t a0 = to_tf32(Zs[(ks * 8 + tq) * kRowPitchB + eb + g8]);
+        const uint32_t a1 = to_tf32(Zs[(ks * 8 + tq) * kRowPitchB + eb + g8 + 8]);
+        const uint32_t a2 = to_tf32(Zs[(ks * 8 + tq + 4) * kRowPitchB + eb + g8]);
+        const uint32_t a3 = to_tf32(Zs[(ks * 8 + tq + 4) * kRowPitchB + eb + g8 + 8]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          const uint32_t b0 = to_tf32(Xs[(ks * 8 + tq) * kRowPitchB + db + nt * 8 + g8]);
+          const uint32_t b1 = to_tf32(Xs[(ks * 8 + tq + 4) * kRowPitchB + db + nt * 8 + g8]);
+          mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
+        }
+      }
+      __syncthreads();
+    }
+  }
+  float* P = part + ((size_t)s * Hq + hq) * (size_t)p.Rexp * 64;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const int e = c0 + eb + g8 + 8 * hf;
+    if (e >= p.Rexp) continue;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int d = db + nt * 8 + 2 * tq;
+      *reinterpret_cast<float2*>(P + (size_t)e * 64 + d) = make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+    }
+  }
+}
+
+// db_part[s][h][e] = sum over the split's (batch, group) items of column e of dZ^Q.
+__global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const float* __restrict__ dZ, const long long z_head,
+                                                        const int nsplit, float* __restrict__ part) {
+  const int e = blockIdx.x * 256 + threadIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const long long nitems = (long long)p.B * p.nT;
+  const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
+  float acc = 0.f;
+  if (e < p.Rexp) {
+    for (long long it = it0; it < it1; ++it) {
+      const int b = (int)(it / p.nT), g = (int)(it - (long long)b * p.nT);
+      const GroupInfo gi = p.gq[g];
+      const int col = e - gi.e0;
+      if (col < 0 || col >= gi.W) continue;
+      const int nrows = imin(kTile, p.N - g * kTile);
+      const float* Zg = dZ + (size_t)(b * p.H + h) * z_head + gi.base + col;
+      for (int r = 0; r < nrows; ++r) acc += Zg[(long long)r * gi.S];
+    }
+    part[((size_t)s * p.H + h) * p.Rexp + e] = acc;
+  }
+}
+
+// out[hq][r][c] = sum_{e in fold range of r, ascending} sum_{s ascending} part[s][hq][e][c]
+__global__ void fold_kernel(const float* __restrict__ part, const int nsplit, const int Hq, const int Rexp, const int R,
+                            const int C, const int* __restrict__ fold_lo, const int* __restrict__ fold_hi,
+                            float* __restrict__ out) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)Hq * R * C) return;
+  const int c = (int)(idx % C);
+  const long long hr = idx / C;
+  const int r = (int)(hr % R), hq = (int)(hr / R);
+  float acc = 0.f;
+  for (int e = fold_lo[r]; e < fold_hi[r]; ++e) {
+    float se = 0.f;
+    for (int s = 0; s < nsplit; ++s) se += part[(((size_t)s * Hq + hq) * Rexp + e) * C + c];
+    acc += se;
+  }
+  out[idx] = acc;
+}
+
+// ------------------------------------------------------------------ debug
+__global__ void debug_phi_kernel(const relpos_map_desc map, const int N, int* out) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < 2 * N - 1) out[t] = phi_of(map, N, t - (N - 1));
+}
+
+__global__ void debug_plan_kernel(const int B, const int N, const int causal, const int* key_len, const int E_lo,
+                                  const int E_hi, int* classes, int* segs) {
+  const int nT = (N + kTile - 1) / kTile;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)B * nT * nT) return;
+  const int kj = (int)(idx % nT);
+  const int qi = (int)((idx / nT) % nT);
+  const int b = (int)(idx / ((long long)nT * nT));
+  const int nkv = key_len ? key_len[b] : N;
+  classes[idx] = tile_class(qi, kj, N, nkv, causal, E_lo, E_hi);
+  if (kj == 0) {
+    int sg[4];
+    tile_segments(qi, nT, N, nkv, causal, E_lo, E_hi, sg);
+    for (int c = 0; c < 4; ++c) segs[((size_t)b * nT + qi) * 4 + c] = sg[c];
+  }
+}
+
+inline unsigned nblk(long long n, int t) { return (unsigned)((n + t - 1) / t); }
+
+}  // namespace
+
+cudaError_t launch_build_tables(const Plan& p, const relpos_map_desc& map, GroupInfo* gq, GroupInfo* gk, int* phi_exp,
+                                int R, const void* aq, const void* ak, int table_per_head, void* aq_exp, void* ak_exp,
+                                const float* b, float* b_exp, int is_bf16, int expand_tables, cudaStream_t s) {
+  (void)is_bf16;
+  { groups_kernel<<<nblk(p.nT, 128), 128, 0, s>>>(p, gq, gk); note_launch(1); }
+  { phi_exp_kernel<<<nblk(p.Rexp, 256), 256, 0, s>>>(map, p.N, p.E_lo, p.Rexp, phi_exp); note_launch(1); }
+  if (b) { bias_exp_kernel<<<nblk((long long)p.H * p.Rexp, 256), 256, 0, s>>>(map, p.N, p.E_lo, p.Rexp, R, p.H, b, b_exp); note_launch(1); }
+  if (expand_tables) {
+    const int Hq = table_per_head ? p.H : 1;
+    const long long n = (long long)Hq * p.Rexp * 8;
+    if (aq) { table_exp_kernel<<<nblk(n, 256), 256, 0, s>>>(map, p.N, p.E_lo, p.Rexp, R, Hq, (const uint4*)aq, (uint4*)aq_exp); note_launch(1); }
+    if (ak) { table_exp_kernel<<<nblk(n, 256), 256, 0, s>>>(map, p.N, p.E_lo, p.Rexp, R, Hq, (const uint4*)ak, (uint4*)ak_exp); note_launch(1); }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold_ranges(const Plan& p, const int* phi_exp, int R, int* fold_lo, int* fold_hi, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(fold_lo, 0, sizeof(int) * R, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(fold_hi, 0, sizeof(int) * R, s);
+  if (e != cudaSuccess) return e;
+  { fold_mark_kernel<<<nblk(p.Rexp, 256), 256, 0, s>>>(phi_exp, p.Rexp, fold_lo, fold_hi); note_launch(1); }
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(projection_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kProjSmem);
+  if (e != cudaSuccess) return e;
+  // widest group decides the chunk count; narrower groups exit early
+  int wq = 0, wk = 0;
+  if (!p.grouped) { wq = wk = p.Rexp; }
+  else { wq = wk = p.N + kTile - 1; }
+  if (t.zq && t.aq_exp) {
+    dim3 grid((wq + 63) / 64, p.nT, p.B * p.H);
+    { projection_kernel<T><<<grid, 256, kProjSmem, s>>>(p, 0, (const T*)t.q, (const T*)t.aq_exp,
+                                                      t.table_per_head ? t.aq_hs : 0, t.zq, p.zq_head); note_launch(1); }
+  }
+  if (t.zk && t.ak_exp) {
+    dim3 grid((wk + 63) / 64, p.nT, p.B * p.H);
+    { projection_kernel<T><<<grid, 256, kProjSmem, s>>>(p, 1, (const T*)t.k, (const T*)t.ak_exp,
+                                                      t.table_per_head ? t.ak_hs : 0, t.zk, p.zk_head); note_launch(1); }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s) {
+  return t.is_bf16 ? projection_typed<__nv_bfloat16>(p, t, s) : projection_typed<__half>(p, t, s);
+}
+
+template <typename T>
+static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
+  const int Hq = t.table_per_head ? p.H : 1;
+  const int nE = (p.Rexp + 63) / 64;
+  if (t.aq_exp) {
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, 0, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
+                                                                t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
+    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, 0, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
+                                                                   t.table_per_head, t.nsplit_q, t.daq_part); note_launch(1); }
+    { fold_kernel<<<nblk((long long)Hq * t.R * 64, 256), 256, 0, s>>>(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64,
+                                                                     t.fold_lo, t.fold_hi, t.daq); note_launch(1); }
+  }
+  if (t.ak_exp) {
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, 0, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
+                                                                t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
+    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, 0, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
+                                                                   t.table_per_head, t.nsplit_k, t.dak_part); note_launch(1); }
+    { fold_kernel<<<nblk((long long)Hq * t.R * 64, 256), 256, 0, s>>>(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64,
+                                                                     t.fold_lo, t.fold_hi, t.dak); note_launch(1); }
+  }
+  if (t.b_exp) {
+    { bias_part_kernel<<<dim3((p.Rexp + 255) / 256, p.H, t.nsplit_b), 256, 0, s>>>(p, t.dzq, p.zq_head, t.nsplit_b, t.db_part); note_launch(1); }
+    { fold_kernel<<<nblk((long long)p.H * t.R, 256), 256, 0, s>>>(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1,
+                                                                 t.fold_lo, t.fold_hi, t.db); note_launch(1); }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_relgrad(const Plan& p, const Tensors& t, cudaStream_t s) {
+  return t.is_bf16 ? relgrad_typed<__nv_bfloat16>(p, t, s) : relgrad_typed<__half>(p, t, s);
+}
+
+cudaError_t launch_debug_phi(const relpos_map_desc& map, int N, int* out, cudaStream_t s) {
+  { debug_phi_kernel<<<nblk(2LL * N - 1, 256), 256, 0, s>>>(map, N, out); note_launch(1); }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_tile_plan(int B, int N, int causal, const int* key_len, int E_lo, int E_hi, int* classes,
+                                   int* segs, cudaStream_t s) {
+  const int nT = (N + kTile - 1) / kTile;
+  { debug_plan_kernel<<<nblk((long long)B * nT * nT, 256), 256, 0, s>>>(B, N, causal, key_len, E_lo, E_hi, classes, segs); note_launch(1); }
+  return cudaGetLastError();
+}
+
+}  // namespace relpos

@@ -1,0 +1,211 @@
+/*
+ * relpos_attn.h -- C ABI of the B200 (sm_100a) exact relative-position
+ * attention library.
+ *
+ * The operation is the unified additive score of "Fast and Exact
+ * Relative-Position Attention via Structure-Aware Kernels" (digest page,
+ * Eq. (1)):
+ *
+ *   S_ij = tau * ( q_i.k_j + q_i.aQ_phi(i,j) + k_j.aK_phi(i,j) + b_phi(i,j) ) + M_ij
+ *   O    = softmax_j(S) V,   LSE_i = log sum_j exp(S_ij)
+ *
+ * computed without any N x N tensor in device memory: the relation terms
+ * are projected to scalars Z^Q = Q aQ^T, Z^K = K aK^T over each 128-row
+ * group's reachable offsets (Eq. (2)-(3), "grouped reachable range"), added
+ * to the score tiles on chip, and differentiated per offset with a single
+ * writer per gradient entry (Eq. (4), "backward ... without atomics").
+ * Bucketed maps are expanded to an equivalent truncated map whose copy
+ * columns are summed back into their bucket ("constant tiles and the
+ * saturated region").
+ *
+ * Conventions shared by every entry point
+ *  - Offsets are delta = j - i (key position minus query position).
+ *  - Every pointer named "device" must point to CUDA device memory owned
+ *    by the caller; the library never allocates or frees device memory.
+ *    Pointers named "host" point to host memory owned by the caller.
+ *  - Tensors are dense row-major; [B,H,N,d] means the last index is
+ *    contiguous.  Device pointers to 16-bit tensors must be 16-byte aligned.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default)
+ *    and runs asynchronously; nothing synchronises the host except the
+ *    calls marked "synchronous".
+ *  - Return value: RELPOS_OK (0) or a negative relpos_status.  On an error
+ *    that is detected before any launch nothing is enqueued.  No C++
+ *    exception crosses this interface.
+ *  - Identical inputs give bit-identical outputs (no atomics anywhere).
+ */
+#ifndef RELPOS_ATTN_H_
+#define RELPOS_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* relpos_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  RELPOS_OK = 0,
+  RELPOS_ERR_INVALID_ARG = -1,    /* null required pointer, bad size, misaligned pointer */
+  RELPOS_ERR_UNSUPPORTED = -2,    /* head dim other than 64, unknown dtype/map/mask */
+  RELPOS_ERR_WORKSPACE = -3,      /* workspace null or smaller than relpos_workspace_size */
+  RELPOS_ERR_CUDA = -4,           /* a CUDA call failed; see relpos_last_cuda_error() */
+  RELPOS_ERR_TIMEOUT = -5         /* a kernel's bounded wait expired (device status word) */
+} relpos_status;
+
+/* Offset maps (digest, experimental setup: Shaw truncated, Transformer-XL
+ * identity, T5 buckets, DeBERTa log buckets). */
+typedef enum {
+  RELPOS_MAP_TRUNCATED = 0,   /* phi = clamp(delta, -clip, clip) + clip; R = 2 clip + 1 */
+  RELPOS_MAP_IDENTITY = 1,    /* phi = delta + N - 1; R = 2N - 1 */
+  RELPOS_MAP_BUCKET_T5 = 2,   /* T5 buckets (num_buckets, max_distance, bidirectional); R = num_buckets */
+  RELPOS_MAP_BUCKET_LOG = 3   /* DeBERTa log buckets (num_buckets = span k, max_distance = max
+                                 position); R = 2 num_buckets */
+} relpos_map_kind;
+
+typedef struct {
+  int32_t kind;           /* relpos_map_kind */
+  int32_t clip;           /* TRUNCATED: clip distance c >= 0 */
+  int32_t num_buckets;    /* BUCKET_T5 / BUCKET_LOG */
+  int32_t max_distance;   /* BUCKET_T5 / BUCKET_LOG */
+  int32_t bidirectional;  /* BUCKET_T5: 1 = bidirectional, 0 = causal-style one-sided */
+} relpos_map_desc;
+
+/* Additive mask M (bit flags; M = -inf where masked, 0 elsewhere). */
+typedef enum {
+  RELPOS_MASK_NONE = 0,
+  RELPOS_MASK_CAUSAL = 1,       /* masks j > i */
+  RELPOS_MASK_KEY_PADDING = 2   /* masks j >= key_len[b] */
+} relpos_mask_flags;
+
+typedef enum { RELPOS_F16 = 0, RELPOS_BF16 = 1, RELPOS_F32 = 2 } relpos_dtype;
+
+/* Tile classes of the tile plan (digest, "constant tiles and the saturated region"). */
+typedef enum {
+  RELPOS_TILE_MASKED = 0,    /* no kept cell: skipped */
+  RELPOS_TILE_CONST_LO = 1,  /* every cell has delta <= E_lo: one shared low-saturated row */
+  RELPOS_TILE_BAND = 2,      /* intersects the band: per-score gather */
+  RELPOS_TILE_CONST_HI = 3   /* every cell has delta >= E_hi: one shared high-saturated row */
+} relpos_tile_class;
+
+/* Tile edge of the tile plan and group size of the projections. */
+#define RELPOS_TILE 128
+
+typedef struct {
+  int32_t B, H, N, d;        /* d must be 64 */
+  int32_t dtype;             /* RELPOS_F16 or RELPOS_BF16: q, k, v, aq, ak (and dout, dq, dk, dv) */
+  int32_t out_dtype;         /* O: same as dtype, or RELPOS_F32 */
+  float tau;                 /* score scale */
+  relpos_map_desc map;
+  int32_t mask;              /* relpos_mask_flags */
+  int32_t table_per_head;    /* 0: aq/ak are [R,d] shared by all heads; 1: [H,R,d] */
+  const int32_t* key_len;    /* device [B], each in [0, N]; required iff mask has KEY_PADDING */
+  const void* q;             /* device [B,H,N,d] dtype */
+  const void* k;             /* device [B,H,N,d] dtype */
+  const void* v;             /* device [B,H,N,d] dtype */
+  const void* aq;            /* device [R,d] / [H,R,d] dtype, or NULL (term absent) */
+  const void* ak;            /* device [R,d] / [H,R,d] dtype, or NULL (term absent) */
+  const float* b;            /* device [H,R] float32, or NULL (term absent) */
+  void* o;                   /* device [B,H,N,d] out_dtype: output (forward) / input (backward) */
+  float* lse;                /* device [B,H,N] float32, natural log: output (fwd) / input (bwd);
+                                -inf for a row whose keys are all masked (its O row is 0) */
+} relpos_fwd_args;
+
+typedef struct {
+  relpos_fwd_args fwd;       /* the forward's inputs, plus its O and LSE (read) */
+  const void* dout;          /* device [B,H,N,d] dtype: upstream gradient dO */
+  void* dq;                  /* device [B,H,N,d] dtype, overwritten */
+  void* dk;                  /* device [B,H,N,d] dtype, overwritten */
+  void* dv;                  /* device [B,H,N,d] dtype, overwritten */
+  float* daq;                /* device float32, shape of aq; required iff aq != NULL; overwritten */
+  float* dak;                /* device float32, shape of ak; required iff ak != NULL; overwritten */
+  float* db;                 /* device [H,R] float32; required iff b != NULL; overwritten */
+} relpos_bwd_args;
+
+/* Number of rows R of a relation table for `map` at sequence length N (host only).
+ * Errors: INVALID_ARG for null pointers or N < 1, UNSUPPORTED for an unknown kind. */
+int relpos_table_rows(const relpos_map_desc* map, int32_t N, int32_t* R_out);
+
+/* Saturation bounds of the expanded truncated map (host only, digest "constant
+ * tiles and the saturated region"): every reachable offset <= *e_lo maps to one
+ * row, every offset >= *e_hi to one row; the expanded table has one row per
+ * offset in [*e_lo, *e_hi]. */
+int relpos_expanded_bounds(const relpos_map_desc* map, int32_t N, int32_t* e_lo, int32_t* e_hi);
+
+/* Workspace bytes needed by relpos_attn_fwd / relpos_attn_bwd for these
+ * arguments (pointers are not read; only sizes, map, mask and which of
+ * aq/ak/b are non-NULL).  The workspace holds the projections Z^Q/Z^K
+ * (O(B H N R_reach), never N x N for non-identity maps), the expanded
+ * tables, and in backward the offset-sharded gradients. */
+int relpos_workspace_size(const relpos_fwd_args* a, size_t* fwd_bytes, size_t* bwd_bytes);
+
+/* Forward: writes a->o and a->lse.  workspace: device, >= fwd_bytes, 256-byte
+ * aligned, contents on entry ignored.  Errors: INVALID_ARG, UNSUPPORTED,
+ * WORKSPACE, CUDA. */
+int relpos_attn_fwd(const relpos_fwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream);
+
+/* Backward (digest: two-pass backward, Eq. (4)): from dO and the forward's O
+ * and LSE, writes dq, dk, dv and the table gradients daq/dak/db.  Shared
+ * tables receive the sum over batch and heads, per-head tables the sum over
+ * batch, both in a fixed order.  workspace: device, >= bwd_bytes. */
+int relpos_attn_bwd(const relpos_bwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream);
+
+/* Human-readable text of a relpos_status (static storage). */
+const char* relpos_status_string(int status);
+
+/* The last cudaError_t seen by this thread inside the library (0 = none). */
+int relpos_last_cuda_error(void);
+
+/* --- measurement ---------------------------------------------------------- */
+
+/* Per-phase device time collected between relpos_profile_start and
+ * relpos_profile_stop.  Phases: "tables", "projection", "fwd_attention",
+ * "bwd_prep", "bwd_dq", "bwd_dkdv", "fold_ranges", "relation_grads". */
+typedef struct {
+  char name[32];
+  int32_t calls;       /* times the phase ran */
+  int32_t kernels;     /* kernels it launched in total */
+  float total_ms;      /* summed device time (CUDA events on the caller's stream) */
+} relpos_phase_stat;
+
+/* Starts bracketing every phase the library enqueues with CUDA events
+ * (host-side bookkeeping only; the events add a few microseconds per phase).
+ * Clears earlier statistics. */
+int relpos_profile_start(void);
+
+/* Stops collecting, waits for the recorded events (synchronous) and copies up
+ * to max_stats phase statistics into stats (host array).  *n_stats receives
+ * the number of phases seen. */
+int relpos_profile_stop(relpos_phase_stat* stats, int32_t max_stats, int32_t* n_stats);
+
+/* Number of kernels this library has launched in this process so far. */
+int64_t relpos_kernel_launches(void);
+
+/* --- parity exports (used by the tests) --------------------------------- */
+
+/* phi(i, j) for all N x N cells computed on the host. phi_host: host [N*N] int32. */
+int relpos_debug_phi(const relpos_map_desc* map, int32_t N, int32_t* phi_host);
+
+/* phi(j - i) for the 2N-1 offsets delta = 1-N .. N-1, computed by the same
+ * device code the expansion kernel uses. phi_dev: device [2N-1] int32.
+ * Synchronous. */
+int relpos_debug_phi_device(const relpos_map_desc* map, int32_t N, int32_t* phi_dev, relpos_stream_t stream);
+
+/* Tile plan on the host: classes host int32 [B][nT][nT] and segments host
+ * int32 [B][nT][4] = (end of CONST_LO run, end of BAND run, end of live
+ * tiles, nT) with nT = ceil(N / RELPOS_TILE).  key_len_host: host [B] or NULL. */
+int relpos_debug_tile_plan(const relpos_map_desc* map, int32_t B, int32_t N, int32_t mask,
+                           const int32_t* key_len_host, int32_t* classes_host, int32_t* segs_host);
+
+/* The same tile plan computed by the device code the kernels use; arguments
+ * as above but key_len, classes and segs are device pointers.  Synchronous. */
+int relpos_debug_tile_plan_device(const relpos_map_desc* map, int32_t B, int32_t N, int32_t mask,
+                                  const int32_t* key_len_dev, int32_t* classes_dev, int32_t* segs_dev,
+                                  relpos_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RELPOS_ATTN_H_ */

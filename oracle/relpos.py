@@ -404,3 +404,111 @@ def backward(q, k, v, do, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None
                 db[h] += g["db"]
     res["daq"], res["dak"], res["db"] = daq, dak, db
     return res
+
+
+# ----------------------------------------------------------------------------
+# Sampled evaluation for sequence lengths where whole N x N matrices per head
+# are too large to keep: the definitions above applied to chosen query rows
+# (dQ) and chosen key columns (dK, dV).  Every query row of the forward is
+# independent, so O and LSE of all rows are produced row-chunk by row-chunk.
+# ----------------------------------------------------------------------------
+
+def head_forward_all_rows(q, k, v, aq, ak, bvec, tau, m: MapDesc, causal, key_len_b, chunk=1024):
+    N = q.shape[0]
+    O = np.zeros_like(q)
+    L = np.zeros(N)
+    for r0 in range(0, N, chunk):
+        rows = np.arange(r0, min(N, r0 + chunk))
+        phi = phi_matrix(m, N, rows)
+        allowed = allowed_matrix(N, causal, key_len_b, rows)
+        o, lse, _ = head_forward(q[rows], k, v, aq, ak, bvec, tau, phi, allowed)
+        O[rows], L[rows] = o, lse
+    return O, L
+
+
+def head_grads_sampled(q, k, v, do, aq, ak, bvec, tau, m: MapDesc, causal, key_len_b, qrows, kcols, chunk=1024):
+    """dQ at query rows `qrows` and dK, dV at key columns `kcols` of one (b, h) slice,
+    plus O and LSE of every row.  Same formulas as head_backward."""
+    N = q.shape[0]
+    O, L = head_forward_all_rows(q, k, v, aq, ak, bvec, tau, m, causal, key_len_b, chunk)
+    D = np.sum(do * O, axis=1)
+    R = table_rows(m, N)
+    # query rows
+    qrows = np.asarray(qrows)
+    phi = phi_matrix(m, N, qrows)
+    allowed = allowed_matrix(N, causal, key_len_b, qrows)
+    S = head_scores(q[qrows], k, aq, ak, bvec, tau, phi, allowed)
+    Lr = L[qrows][:, None]
+    P = np.where(np.isfinite(Lr), np.exp(S - np.where(np.isfinite(Lr), Lr, 0.0)), 0.0)
+    dS = P * (do[qrows] @ v.T - D[qrows][:, None])
+    dq = tau * (dS @ k)
+    if aq is not None:
+        dzq = np.zeros((len(qrows), R))
+        for a in range(len(qrows)):
+            dzq[a] = tau * np.bincount(phi[a], weights=dS[a], minlength=R)
+        dq = dq + dzq @ aq
+    # key columns: scores of every query row against the chosen keys
+    kcols = np.asarray(kcols)
+    dk = np.zeros((len(kcols), q.shape[1]))
+    dv = np.zeros_like(dk)
+    dzk = np.zeros((len(kcols), R))
+    for r0 in range(0, N, chunk):
+        rows = np.arange(r0, min(N, r0 + chunk))
+        i = rows[:, None]
+        j = kcols[None, :]
+        phi_c = phi_of_delta(m, j - i, N)
+        ok = allowed_matrix(N, causal, key_len_b, rows)[:, kcols]
+        Sc = q[rows] @ k[kcols].T
+        if aq is not None:
+            ZQ = q[rows] @ aq.T
+            Sc = Sc + np.take_along_axis(ZQ, phi_c, axis=1)
+        if ak is not None:
+            ZK = k[kcols] @ ak.T
+            Sc = Sc + ZK[np.arange(len(kcols))[None, :], phi_c]
+        if bvec is not None:
+            Sc = Sc + bvec[phi_c]
+        Sc = np.where(ok, tau * Sc, -np.inf)
+        Lc = L[rows][:, None]
+        Pc = np.where(np.isfinite(Lc), np.exp(Sc - np.where(np.isfinite(Lc), Lc, 0.0)), 0.0)
+        dSc = Pc * (do[rows] @ v[kcols].T - D[rows][:, None])
+        dv += Pc.T @ do[rows]
+        dk += tau * (dSc.T @ q[rows])
+        for c in range(len(kcols)):
+            dzk[c] += tau * np.bincount(phi_c[:, c], weights=dSc[:, c], minlength=R)
+    if ak is not None:
+        dk = dk + dzk @ ak
+    return dict(o=O, lse=L, dq=dq, dk=dk, dv=dv)
+
+
+def head_block_step(q, k, v, do, aq, ak, bvec, tau, m: MapDesc, causal, key_len_b, rows):
+    """Forward and backward restricted to the query rows `rows` of one (b, h) slice.
+
+    Returns the block's outputs (o, lse, dq for those rows) and its additive
+    contributions to the sums over query rows (dv, dk, daq, dak, db).  Summed
+    over a partition of the rows these contributions give head_backward's
+    dV, dK and table gradients; this is the unit of work the CPU baseline
+    times."""
+    N = k.shape[0]
+    rows = np.asarray(rows)
+    R = table_rows(m, N)
+    phi = phi_matrix(m, N, rows)
+    allowed = allowed_matrix(N, causal, key_len_b, rows)
+    O, lse, P = head_forward(q[rows], k, v, aq, ak, bvec, tau, phi, allowed)
+    D = np.sum(do[rows] * O, axis=1, keepdims=True)
+    dS = P * (do[rows] @ v.T - D)
+    n = len(rows)
+    ri = np.repeat(np.arange(n), N)
+    cj = np.tile(np.arange(N), n)
+    fp = phi.reshape(-1)
+    dzq = tau * np.bincount(ri * R + fp, weights=dS.reshape(-1), minlength=n * R).reshape(n, R)
+    dzk = tau * np.bincount(cj * R + fp, weights=dS.reshape(-1), minlength=N * R).reshape(N, R)
+    out = dict(o=O, lse=lse, dv=P.T @ do[rows], dq=tau * (dS @ k), dk=tau * (dS.T @ q[rows]))
+    if aq is not None:
+        out["dq"] = out["dq"] + dzq @ aq
+        out["daq"] = dzq.T @ q[rows]
+    if ak is not None:
+        out["dak"] = dzk.T @ k
+        out["dk_rel"] = dzk @ ak
+    if bvec is not None:
+        out["db"] = tau * np.bincount(fp, weights=dS.reshape(-1), minlength=R)
+    return out

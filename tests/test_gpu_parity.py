@@ -1,0 +1,115 @@
+"""GPU parity: the CUDA library through its C ABI against the fp64 oracle.
+
+Small and ragged sizes (several 128-row tiles plus a tail), every map kind,
+every term subset, causal and key-padding masks, fp16 and bf16, empty and
+degenerate cases; bit-exact maps and tile plans; determinism.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from synth import small_workload
+from relpos_harness import (check_backward, check_forward, lmap, omap, run_library, run_oracle)
+import exact_relative_position_b200 as rp
+
+pytestmark = pytest.mark.gpu
+
+MAPS = {
+    "trunc16": dict(map_kind="truncated", clip=16),
+    "trunc200": dict(map_kind="truncated", clip=200),
+    "identity": dict(map_kind="identity"),
+    "t5": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=1),
+    "t5uni": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=0),
+    "log": dict(map_kind="log", num_buckets=32, max_distance=128),
+}
+
+
+@pytest.mark.parametrize("mname", list(MAPS))
+@pytest.mark.parametrize("N", [1, 2, 300, 1000])
+def test_device_phi_bit_exact(mname, N):
+    w = small_workload(N=N, **MAPS[mname])
+    got = rp.debug_phi_device(lmap(w), N).cpu().numpy()
+    want = orc.phi_of_delta(omap(w), np.arange(1 - N, N), N)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("mname", list(MAPS))
+@pytest.mark.parametrize("N,causal,key_len", [(300, False, None), (1000, True, None), (700, False, [700, 333, 1])])
+def test_device_tile_plan_bit_exact(mname, N, causal, key_len):
+    w = small_workload(N=N, **MAPS[mname])
+    B = 1 if key_len is None else len(key_len)
+    cls, seg = rp.debug_tile_plan_device(lmap(w), B, N, causal=causal, key_len=key_len)
+    ocls, oseg = orc.tile_plan_rule(omap(w), N, 128, causal, key_len, B)
+    assert np.array_equal(cls.cpu().numpy(), ocls)
+    assert np.array_equal(seg.cpu().numpy(), oseg)
+
+
+CASES = [
+    # map, N, terms, causal, key_len, dtype, per_head
+    ("trunc16", 1, ("aQ", "aK", "b"), False, None, torch.float16, False),
+    ("trunc16", 7, ("aQ",), False, None, torch.float16, False),
+    ("trunc16", 128, ("aQ", "aK"), False, None, torch.float16, False),
+    ("trunc16", 129, ("aQ", "aK", "b"), True, None, torch.float16, True),
+    ("trunc16", 300, ("aQ", "aK", "b"), False, [300, 211], torch.bfloat16, False),
+    ("trunc200", 255, ("aQ", "aK"), False, None, torch.float16, False),
+    ("identity", 127, ("aQ", "b"), True, None, torch.bfloat16, True),
+    ("identity", 300, ("aQ", "aK", "b"), False, None, torch.float16, True),
+    ("identity", 520, ("aQ", "b"), True, None, torch.float16, True),
+    ("t5", 300, ("b",), False, None, torch.float16, False),
+    ("t5", 513, ("b",), True, [513, 77], torch.float16, False),
+    ("t5", 400, ("aQ", "aK", "b"), False, [400, 399], torch.bfloat16, True),
+    ("t5uni", 300, ("b",), True, None, torch.float16, False),
+    ("log", 300, ("aQ", "aK"), False, [300, 290], torch.float16, True),
+    ("log", 777, ("aQ", "aK", "b"), False, None, torch.bfloat16, False),
+    ("trunc16", 200, (), False, None, torch.float16, False),
+    ("trunc16", 200, ("aK",), True, None, torch.float16, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}-N{c[1]}-{'+'.join(c[2]) or 'none'}-{'causal' if c[3] else ''}"
+                                             f"{'pad' if c[4] else ''}-{str(c[5])[6:]}" for c in CASES])
+def test_small_parity(case):
+    mname, N, terms, causal, key_len, dtype, per_head = case
+    B = 1 if key_len is None else len(key_len)
+    w = small_workload(N=N, B=B, H=2, terms=terms, causal=causal, key_len=key_len, dtype=dtype,
+                       per_head_tables=per_head, tau=0.125 if "b" not in terms else 0.5, **MAPS[mname])
+    got = run_library(w, out_f32=(dtype == torch.bfloat16))
+    want = run_oracle(w)
+    check_forward(got, want, str(case))
+    check_backward(got, want, str(case))
+
+
+def test_fully_masked_rows():
+    w = small_workload(N=200, B=2, H=2, terms=("aQ", "b"), key_len=[0, 200], **MAPS["trunc16"])
+    got = run_library(w)
+    want = run_oracle(w)
+    assert np.all(got["o"][0] == 0) and np.all(np.isneginf(got["lse"][0]))
+    check_forward(got, want)
+    check_backward(got, want)
+    assert np.all(got["dq"][0] == 0) and np.all(got["dk"][0] == 0) and np.all(got["dv"][0] == 0)
+
+
+def test_bucketed_equals_expanded_on_gpu():
+    """A T5 run equals a truncated-map run with the same expanded bias rows."""
+    N = 400
+    w = small_workload(N=N, terms=("b",), **MAPS["t5"])
+    elo, ehi = orc.expanded_bounds(omap(w), N)
+    rowmap = orc.phi_of_delta(omap(w), np.arange(elo, ehi + 1), N)
+    assert elo == -ehi
+    w2 = small_workload(N=N, terms=("b",), map_kind="truncated", clip=ehi)
+    w2.q, w2.k, w2.v, w2.do = w.q, w.k, w.v, w.do
+    w2.b = w.b[:, torch.as_tensor(rowmap)].contiguous()
+    a, b = run_library(w), run_library(w2)
+    np.testing.assert_array_equal(a["o"], b["o"])
+    folded = np.zeros_like(a["db"])
+    np.add.at(folded, (slice(None), rowmap), b["db"])
+    np.testing.assert_allclose(folded, a["db"], rtol=1e-5, atol=1e-7)
+
+
+def test_deterministic():
+    w = small_workload(N=600, B=2, H=3, terms=("aQ", "aK", "b"), key_len=[600, 451], **MAPS["log"])
+    r1, r2 = run_library(w), run_library(w)
+    for k in r1:
+        if r1[k] is not None:
+            assert np.array_equal(r1[k], r2[k]), k

@@ -411,3 +411,48 @@ def test_group_reach_overhead_matches_pages():
         reach.update(range(-i, N - i))
     assert len(reach) == N + G - 1
     assert abs((G - 1) / N - 0.016) < 0.001
+
+
+@pytest.mark.parametrize("kind,causal,kl", [("truncated", False, None), ("identity", True, None), ("log", False, 21)])
+def test_sampled_grads_equal_full_backward(kind, causal, kl):
+    """The sampled evaluation used at large N equals the full-matrix backward."""
+    N, d = 29, 4
+    m = {"truncated": orc.MapDesc("truncated", clip=3), "identity": orc.MapDesc("identity"),
+         "log": orc.MapDesc("log", num_buckets=8, max_distance=16)}[kind]
+    R = orc.table_rows(m, N)
+    q, k, v, do = (_rand((N, d), s) for s in range(4))
+    aq, ak, b = _rand((R, d), 5, 0.5), _rand((R, d), 6, 0.5), _rand((R,), 7)
+    phi = orc.phi_matrix(m, N)
+    allowed = orc.allowed_matrix(N, causal, kl)
+    full = orc.head_backward(q, k, v, do, aq, ak, b, 0.4, phi, allowed, R)
+    rows, cols = np.array([0, 5, 28]), np.array([1, 13, 28])
+    smp = orc.head_grads_sampled(q, k, v, do, aq, ak, b, 0.4, m, causal, kl, rows, cols, chunk=7)
+    np.testing.assert_allclose(smp["o"], full["o"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(smp["lse"], full["lse"], rtol=1e-12)
+    np.testing.assert_allclose(smp["dq"], full["dq"][rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(smp["dk"], full["dk"][cols], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(smp["dv"], full["dv"][cols], rtol=1e-10, atol=1e-12)
+
+
+def test_row_blocks_sum_to_full_backward():
+    """The CPU-baseline unit of work (a block of query rows) sums to the full backward."""
+    N, d = 31, 4
+    m = orc.MapDesc("truncated", clip=4)
+    R = orc.table_rows(m, N)
+    q, k, v, do = (_rand((N, d), s) for s in range(4))
+    aq, ak, b = _rand((R, d), 5, 0.5), _rand((R, d), 6, 0.5), _rand((R,), 7)
+    phi = orc.phi_matrix(m, N)
+    full = orc.head_backward(q, k, v, do, aq, ak, b, 0.3, phi, np.ones((N, N), bool), R)
+    acc = {n: 0.0 for n in ("dv", "dk", "daq", "dak", "db", "dk_rel")}
+    for r0 in range(0, N, 8):
+        rows = np.arange(r0, min(N, r0 + 8))
+        blk = orc.head_block_step(q, k, v, do, aq, ak, b, 0.3, m, False, None, rows)
+        np.testing.assert_allclose(blk["dq"], full["dq"][rows], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(blk["o"], full["o"][rows], rtol=1e-12, atol=1e-13)
+        for n in acc:
+            acc[n] = acc[n] + blk[n]
+    np.testing.assert_allclose(acc["dv"], full["dv"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(acc["dk"] + acc["dk_rel"], full["dk"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(acc["daq"], full["daq"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(acc["dak"], full["dak"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(acc["db"], full["db"], rtol=1e-10, atol=1e-12)
