@@ -216,6 +216,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ncu", action="store_true",
+                    help="one forward + backward only (for an ncu capture of each kernel's first launch)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -262,6 +264,12 @@ def main():
     def bwd():
         rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, workspace=ws, grads=grads, **kw)
 
+    if args.ncu:
+        fwd()
+        bwd()
+        torch.cuda.synchronize()
+        print(json.dumps({"ncu_case": args.workload, "launches": rp.kernel_launches()}))
+        return
     torch.cuda.reset_peak_memory_stats(dev)
     for _ in range(args.warmup):
         flush.zero_()
