@@ -52,7 +52,7 @@ class relpos_phase_stat(ctypes.Structure):
 EXPORTS = ["relpos_table_rows", "relpos_expanded_bounds", "relpos_workspace_size", "relpos_attn_fwd",
            "relpos_attn_bwd", "relpos_status_string", "relpos_last_cuda_error", "relpos_debug_phi",
            "relpos_debug_phi_device", "relpos_debug_tile_plan", "relpos_debug_tile_plan_device",
-           "relpos_profile_start", "relpos_profile_stop", "relpos_kernel_launches"]
+           "relpos_profile_start", "relpos_profile_stop", "relpos_kernel_launches", "relpos_attn_fwd_noalloc"]
 
 
 def load_library(path: str = LIBPATH) -> ctypes.CDLL:
@@ -78,6 +78,7 @@ def load_library(path: str = LIBPATH) -> ctypes.CDLL:
     sig["relpos_profile_start"] = []
     sig["relpos_profile_stop"] = [P(relpos_phase_stat), ctypes.c_int32, P(ctypes.c_int32)]
     sig["relpos_kernel_launches"] = []
+    sig["relpos_attn_fwd_noalloc"] = [P(relpos_fwd_args), ctypes.c_void_p]
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -286,3 +287,22 @@ def profile_stop():
 
 def kernel_launches() -> int:
     return int(lib().relpos_kernel_launches())
+
+
+NOALLOC_MAX_WORKSPACE = 32 << 20
+
+
+def relpos_attn_fwd_noalloc(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap, causal: bool = False,
+                            key_len=None, out_f32: bool = False, o=None, lse=None):
+    """Forward through relpos_attn_fwd_noalloc: the library's fixed 32 MiB scratch
+    array replaces the workspace, so the call needs no device allocation for it."""
+    B, H, N, d = q.shape
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=torch.float32 if out_f32 else q.dtype)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    if key_len is not None:
+        key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
+    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse)
+    _check(lib().relpos_attn_fwd_noalloc(ctypes.byref(a), _stream(q.device)), "relpos_attn_fwd_noalloc")
+    return o, lse

@@ -28,6 +28,12 @@ void note_launch(int n) { g_kernel_launches += n; }
 using namespace relpos;
 
 namespace {
+int cuda_fail(cudaError_t e);
+}
+
+int relpos::cuda_status(cudaError_t e) { return cuda_fail(e); }
+
+namespace {
 
 // ---- optional per-phase event timing (relpos_profile_start / _stop)
 enum Phase { PH_TABLES, PH_PROJ, PH_FWD, PH_PREP, PH_DQ, PH_DKDV, PH_FOLD, PH_RELGRAD, PH_COUNT };

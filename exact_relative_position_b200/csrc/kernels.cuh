@@ -35,6 +35,9 @@ struct Tensors {
   int is_bf16;
 };
 
+// Records e as this thread's last CUDA error and returns RELPOS_ERR_CUDA.
+int cuda_status(cudaError_t e);
+
 // Counts kernel launches (process-wide, reported by relpos_kernel_launches).
 void note_launch(int n);
 

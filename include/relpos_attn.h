@@ -157,6 +157,26 @@ const char* relpos_status_string(int status);
 /* The last cudaError_t seen by this thread inside the library (0 = none). */
 int relpos_last_cuda_error(void);
 
+/* Forward without a caller workspace (no counterpart in the paper; an
+ * addition for callers that cannot allocate device memory, e.g. code running
+ * while a memory pool or another runtime owns the whole device and forbids
+ * outside allocations, or an enqueue step that must not allocate).
+ *
+ * Same arguments, outputs and errors as relpos_attn_fwd, but the workspace is
+ * a fixed 32 MiB array inside the library's device image.  Every GPU that
+ * loads the library holds that array until the process exits.  The call
+ * itself calls no cudaMalloc / cudaFree or any allocating routine.
+ *  - Shapes whose forward workspace (relpos_workspace_size's fwd_bytes)
+ *    exceeds 32 MiB are rejected with RELPOS_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    outside any stream capture.
+ *  - All calls share the one array and it keeps the previous call's contents;
+ *    the forward reads nothing from it that the same call has not written.
+ *    Calls whose work overlaps on the GPU (different streams, or several
+ *    host threads) race on the array: serialise them. */
+int relpos_attn_fwd_noalloc(const relpos_fwd_args* a, relpos_stream_t stream);
+
 /* --- measurement ---------------------------------------------------------- */
 
 /* Per-phase device time collected between relpos_profile_start and
