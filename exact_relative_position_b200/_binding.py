@@ -52,7 +52,8 @@ class relpos_phase_stat(ctypes.Structure):
 EXPORTS = ["relpos_table_rows", "relpos_expanded_bounds", "relpos_workspace_size", "relpos_attn_fwd",
            "relpos_attn_bwd", "relpos_status_string", "relpos_last_cuda_error", "relpos_debug_phi",
            "relpos_debug_phi_device", "relpos_debug_tile_plan", "relpos_debug_tile_plan_device",
-           "relpos_profile_start", "relpos_profile_stop", "relpos_kernel_launches", "relpos_attn_fwd_noalloc"]
+           "relpos_profile_start", "relpos_profile_stop", "relpos_kernel_launches", "relpos_attn_fwd_noalloc",
+           "relpos_check_workspace"]
 
 
 def load_library(path: str = LIBPATH) -> ctypes.CDLL:
@@ -79,6 +80,7 @@ def load_library(path: str = LIBPATH) -> ctypes.CDLL:
     sig["relpos_profile_stop"] = [P(relpos_phase_stat), ctypes.c_int32, P(ctypes.c_int32)]
     sig["relpos_kernel_launches"] = []
     sig["relpos_attn_fwd_noalloc"] = [P(relpos_fwd_args), ctypes.c_void_p]
+    sig["relpos_check_workspace"] = [ctypes.c_void_p, ctypes.c_void_p, P(ctypes.c_int32)]
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -306,3 +308,12 @@ def relpos_attn_fwd_noalloc(q, k, v, aq=None, ak=None, b=None, *, tau: float, ma
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse)
     _check(lib().relpos_attn_fwd_noalloc(ctypes.byref(a), _stream(q.device)), "relpos_attn_fwd_noalloc")
     return o, lse
+
+
+def check_workspace(workspace) -> int:
+    """Synchronises the current stream and returns the device status word of the
+    last call that used `workspace` (0 = ok); raises RelPosError on a timeout."""
+    st = ctypes.c_int32()
+    _check(lib().relpos_check_workspace(workspace.data_ptr(), _stream(workspace.device), ctypes.byref(st)),
+           "relpos_check_workspace")
+    return st.value

@@ -8,6 +8,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -48,6 +49,26 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+# Kernels that split their registers between warpgroups with setmaxnreg: the
+# split adds up to (threads x registers at launch), so the launch register
+# count must be exactly this value or the split could wait forever.
+REGISTER_SPLIT_KERNELS = {"fwd_sm100_kernel": 168}
+
+
+def _check_register_split(ptxas_log: str):
+    current = None
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            current = line.split("'")[1] if "'" in line else line
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current:
+            for name, want in REGISTER_SPLIT_KERNELS.items():
+                if name in current and int(m.group(1)) != want:
+                    raise RuntimeError(f"{current}: {m.group(1)} registers at launch, the setmaxnreg split "
+                                       f"assumes {want}")
+            current = None
+
+
 def build_library(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
     """Compile every .cu under csrc/ into one shared library (sm_100a)."""
     if not force and not _stale():
@@ -61,7 +82,7 @@ def build_library(force: bool = False, verbose: bool = False, jobs: int = 0) -> 
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
-        cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+        cmd = [nvcc, *NVCC_FLAGS, "-Xptxas", "-v", "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -70,8 +91,8 @@ def build_library(force: bool = False, verbose: bool = False, jobs: int = 0) -> 
         out, _ = pr.communicate()
         if pr.returncode != 0:
             failed.append((src, out))
-        elif verbose and out.strip():
-            print(out, flush=True)
+        else:
+            _check_register_split(out)
     if failed:
         msg = "\n".join(f"--- {s}\n{o}" for s, o in failed)
         raise RuntimeError(f"nvcc failed:\n{msg}")

@@ -127,7 +127,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
+  size_t status, gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
   size_t dsum, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
   int R, Hq, expand, nsq, nsk, nsb;
 };
@@ -164,6 +164,7 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   const size_t BH = (size_t)a->B * a->H;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = up256(off + bytes); return o; };
+  L->status = take(sizeof(int));
   L->gq = take(sizeof(GroupInfo) * p->nT);
   L->gk = take(sizeof(GroupInfo) * p->nT);
   L->phi = take(sizeof(int) * p->Rexp);
@@ -221,6 +222,11 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
   t.is_bf16 = a->dtype == RELPOS_BF16;
   t.table_per_head = a->table_per_head;
   t.R = L.R;
+  t.status = reinterpret_cast<int*>(ws + L.status);
+  {
+    const cudaError_t e0 = cudaMemsetAsync(t.status, 0, sizeof(int), s);
+    if (e0 != cudaSuccess) return cuda_fail(e0);
+  }
   int* phi_exp = reinterpret_cast<int*>(ws + L.phi);
   t.phi_exp = phi_exp;
   t.fold_lo = reinterpret_cast<int*>(ws + L.fold_lo);
@@ -362,6 +368,17 @@ RELPOS_EXPORT const char* relpos_status_string(int status) {
 }
 
 RELPOS_EXPORT int relpos_last_cuda_error(void) { return g_last_cuda_error; }
+
+RELPOS_EXPORT int relpos_check_workspace(const void* workspace, relpos_stream_t stream, int32_t* device_status) {
+  if (!workspace) return RELPOS_ERR_INVALID_ARG;
+  int st = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (device_status) *device_status = st;
+  return st == 0 ? RELPOS_OK : RELPOS_ERR_TIMEOUT;
+}
 
 RELPOS_EXPORT int relpos_profile_start(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);

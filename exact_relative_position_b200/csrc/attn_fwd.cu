@@ -1,211 +1,442 @@
-// attn_fwd.cu -- fused forward of exact relative-position attention
+// attn_fwd.cu -- fused forward of exact relative-position attention on sm_100a
 // (digest of "Fast and Exact Relative-Position Attention via Structure-Aware
-// Kernels": Eq. (1)/(2) and the FlashAttention-style outer loop over query
-// tiles with an online softmax over key tiles).
+// Kernels": Eq. (1)/(2), the FlashAttention-style loop of the pipeline
+// section, and "constant tiles and the saturated region").
 //
-// One CTA owns 128 query rows of one (batch, head).  Q stays in registers as
-// tensor-core fragments; K/V tiles of 64 keys stream through a two-stage
-// cp.async ring.  Each score gets tau * (Z^Q[i,e] + Z^K[j,e] + b[e]) added in
-// registers, e = clamp(j - i, E_lo, E_hi) - E_lo being the expanded relation
-// row, before the base-2 online softmax.  No N x N tensor touches memory.
+// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and
+// walks the key tiles once for both, so each K/V tile that TMA brings into
+// shared memory feeds four tcgen05 GEMMs.  Warp roles:
+//   warp 0       TMA producer: Q0/Q1 once, then K/V tiles into a 3-stage ring
+//   warp 1       MMA issuer (one thread): S_g = Q_g K^T into tensor memory,
+//                O_g += P_g V with P_g read back from tensor memory
+//   warp 2       allocates / frees the 512 tensor-memory columns
+//   warps 4..7   softmax of Q0 (thread r owns row r = TMEM lane r)
+//   warps 8..11  softmax of Q1
+// Tensor memory: S0 cols [0,128), S1 [128,256) (P_g overwrites the first 64
+// columns of S_g as packed 16-bit pairs), O0 [256,320), O1 [320,384).
+//
+// Relation terms are added to the scores in registers.  A key tile whose
+// every offset saturates (CONST_LO / CONST_HI: two comparisons of the tile's
+// offset range with E_lo / E_hi) adds one per-row constant tau (Z^Q_i,sat +
+// b_sat) and one per-column vector tau Z^K_j,sat staged once in shared memory
+// and broadcast; a BAND tile gathers Z^Q[i, e], Z^K[j, e] and b[e] per score
+// with e = clamp(j - i, E_lo, E_hi) - E_lo.  The online softmax runs in base 2
+// and only rescales O when the running row maximum grows by more than 8
+// (a factor 256), which keeps every P <= 256 and the result exact.
+#include <cudaTypedefs.h>
+
 #include "kernels.cuh"
+#include "sm100.cuh"
 #include "warp_mma.cuh"
 
 namespace relpos {
 
 namespace {
 
-constexpr int kBM = 128;   // query rows per CTA (8 warps x 16)
-constexpr int kBN = 64;    // keys per inner step
-constexpr int kThreads = 256;
-constexpr int kSmem = kBM * 128 + 2 * 2 * kBN * 128;   // Q + 2 stages of (K, V)
+using namespace sm100;
 
-template <typename OutT> struct Store;
-template <> struct Store<float> {
-  static __device__ __forceinline__ void two(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+constexpr int kBQ = 128;          // rows per query tile (one softmax warpgroup)
+constexpr int kBK = 128;          // keys per key tile (the tile-plan edge)
+constexpr int kStages = 3;
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = 128 * 128;   // one [128 x 64] 16-bit tile
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = 2 * kTileBytes;
+constexpr uint32_t kOffColv = kOffKV + kStages * 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffColv + 2 * 2 * kBK * 4;
+constexpr uint32_t kOffAbort = kOffBar + 256;
+constexpr uint32_t kOffTmem = kOffAbort + 16;
+constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;   // + alignment slack
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;              // log2 of the largest P allowed before rescaling O
+
+// barrier slots (8 bytes each)
+constexpr int kBarQ = 0;
+constexpr int kBarKvFull = 1;
+constexpr int kBarKvEmpty = kBarKvFull + kStages;
+constexpr int kBarSFull = kBarKvEmpty + kStages;
+constexpr int kBarPReady = kBarSFull + 2;
+constexpr int kBarOFull = kBarPReady + 2;
+constexpr int kBarDrain = kBarOFull + 2;
+constexpr int kBarColv = kBarDrain + 1;   // 2: saturated-column vector staged (per softmax warpgroup)
+
+template <typename OutT> struct RowStore;
+template <> struct RowStore<float> {
+  static __device__ __forceinline__ void row(float* dst, const float* v) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+  }
 };
-template <> struct Store<__half> {
-  static __device__ __forceinline__ void two(__half* p, float a, float b) { *reinterpret_cast<__half2*>(p) = __floats2half2_rn(a, b); }
-};
-template <> struct Store<__nv_bfloat16> {
-  static __device__ __forceinline__ void two(__nv_bfloat16* p, float a, float b) {
-    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+template <typename T> struct RowStore {
+  static __device__ __forceinline__ void row(T* dst, const float* v) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) {
+      uint4 u;
+      u.x = DT<T>::pack(v[c], v[c + 1]);
+      u.y = DT<T>::pack(v[c + 2], v[c + 3]);
+      u.z = DT<T>::pack(v[c + 4], v[c + 5]);
+      u.w = DT<T>::pack(v[c + 6], v[c + 7]);
+      *reinterpret_cast<uint4*>(dst + c) = u;
+    }
   }
 };
 
 template <typename T, typename OutT, bool AQ, bool AK, bool BIAS>
-__global__ void __launch_bounds__(kThreads) fwd_kernel(const Plan p, const Tensors t) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
-  const int N = p.N, q0 = qt * kBM;
-  const size_t off = (size_t)bh * N * 64;
-  const T* Q = static_cast<const T*>(t.q) + off;
-  const T* K = static_cast<const T*>(t.k) + off;
-  const T* V = static_cast<const T*>(t.v) + off;
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sg = smem_raw + (sb - raw);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + kOffAbort);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sg + kOffTmem);
+  auto bar = [&](int slot) { return sb + kOffBar + 8u * (uint32_t)slot; };
 
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sKV = sQ + kBM * 128;
-
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
+  const int N = p.N, q0 = blockIdx.x * (2 * kBQ);
   const int nkv = p.padding ? p.key_len[b] : N;
   int kend = nkv;
-  if (p.causal) kend = imin(kend, imin(q0 + kBM, N));
-  const int ntiles = kend > 0 ? (kend + kBN - 1) / kBN : 0;
+  if (p.causal) kend = imin(kend, imin(q0 + 2 * kBQ, N));
+  const int nkt = kend > 0 ? (kend + kBK - 1) / kBK : 0;
 
-  load_tile_async<kBM, kThreads>(sQ, Q, q0, N, tid);
-  if (ntiles > 0) {
-    load_tile_async<kBN, kThreads>(sKV, K, 0, N, tid);
-    load_tile_async<kBN, kThreads>(sKV + kBN * 128, V, 0, N, tid);
-  }
-  cp_async_commit();
-
-  // Per-thread rows: hf = 0 -> row g, hf = 1 -> row g + 8 of the warp's 16.
-  const int g = lane >> 2, tq = lane & 3;
-  int irow[2];
-  const float* zq_row[2] = {nullptr, nullptr};
-  irow[0] = q0 + warp * 16 + g;
-  irow[1] = irow[0] + 8;
-  if (AQ) {
-    const GroupInfo gi = p.gq[qt];
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf)
-      zq_row[hf] = t.zq + (size_t)bh * p.zq_head + gi.base + (long long)(irow[hf] - q0) * gi.S - gi.e0;
-  }
-  const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
-  const float sc = p.tau * kLog2e;
-
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  float o[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  uint32_t qa[4][4];
-
-  for (int it = 0; it < ntiles; ++it) {
-    const int stage = it & 1;
-    if (it + 1 < ntiles) {
-      const uint32_t sb = sKV + (uint32_t)((it + 1) & 1) * (2 * kBN * 128);
-      load_tile_async<kBN, kThreads>(sb, K, (it + 1) * kBN, N, tid);
-      load_tile_async<kBN, kThreads>(sb + kBN * 128, V, (it + 1) * kBN, N, tid);
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQ), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarKvFull + s), 1);
+      mbar_init(bar(kBarKvEmpty + s), 1);
     }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    if (it == 0) load_a_frags(sQ, warp * 16, lane, qa);
-    const uint32_t sK = sKV + (uint32_t)stage * (2 * kBN * 128);
-    const uint32_t sV = sK + kBN * 128;
-    const int k0 = it * kBN;
-
-    float s[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-    mma_abt<T, 8>(s, qa, sK, 0, lane);
-
-    // Key-side projection rows of this key tile (64 keys lie in one 128-group).
-    const float* zk_tile = nullptr;
-    if (AK) {
-      const int kg = k0 / kTile;
-      const GroupInfo gi = p.gk[kg];
-      zk_tile = t.zk + (size_t)bh * p.zk_head + gi.base - gi.e0 + (long long)(k0 - kg * kTile) * gi.S;
-      // element for key k0 + c at expanded row e: zk_tile[c * S + e]
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(kBarSFull + g), 1);
+      mbar_init(bar(kBarPReady + g), 128);
+      mbar_init(bar(kBarOFull + g), 1);
     }
-    const int zk_S = AK ? p.gk[k0 / kTile].S : 0;
+    mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarColv + 0), 128);
+    mbar_init(bar(kBarColv + 1), 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
 
-    float mx[2] = {-INFINITY, -INFINITY};
+  // Register split: the launch gives every thread 168 registers (384 x 168 =
+  // 64512); warpgroup 0 (producer, MMA issuer, allocator) drops to 56 and the
+  // two softmax warpgroups take 224: 128 x 56 + 256 x 224 = 64512.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && nkt > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
+      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
+      tma_load_3d(sb + kOffQ + kTileBytes, &tmQ, bar(kBarQ), 0, q0 + kBQ, bh);
+      for (int it = 0; it < nkt; ++it) {
+        const int s = it % kStages;
+        if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+        const uint32_t dst = sb + kOffKV + (uint32_t)s * 2 * kTileBytes;
+        mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes);
+        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kBK, bh);
+        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kBK, bh);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nkt > 0) {
+      const bool bf = t.is_bf16 != 0;
+      const uint32_t id_qk = idesc_f16(bf, 128, 128, false, false);
+      const uint32_t id_pv = idesc_f16(bf, 128, 64, false, true);
+      auto issue_qk = [&](int g, int s) {
+        const uint32_t a = sb + kOffQ + (uint32_t)g * kTileBytes;
+        const uint32_t k = sb + kOffKV + (uint32_t)s * 2 * kTileBytes;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + (uint32_t)g * 128, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(k + kk * 32, 16, 1024),
+                 id_qk, kk > 0);
+      };
+      auto issue_pv = [&](int g, int s, bool acc) {
+        const uint32_t v = sb + kOffKV + (uint32_t)s * 2 * kTileBytes + kTileBytes;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int hf = r >> 1;
-        const int cj = nt * 8 + 2 * tq + (r & 1);
-        const int i = irow[hf], j = k0 + cj;
-        float x = -INFINITY;
-        const bool keep = (i < N) && (j < nkv) && !(p.causal && j > i);
-        if (keep) {
-          const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
-          float rel = 0.f;
-          if (AQ) rel += __ldg(zq_row[hf] + e);
-          if (AK) rel += __ldg(zk_tile + (long long)cj * zk_S + e);
-          if (BIAS) rel += __ldg(bexp + e);
-          x = (s[nt][r] + rel) * sc;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256 + (uint32_t)g * 64, tmem + (uint32_t)g * 128 + kk * 8,
+                 sdesc_sw128(v + kk * 2048, 8192, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(bar(kBarSFull + 0));
+        issue_qk(1, 0);
+        mma_commit(bar(kBarSFull + 1));
+        for (int it = 0; it < nkt && ok; ++it) {
+          const int s = it % kStages;
+          const int sn = (it + 1) % kStages;
+          for (int g = 0; g < 2; ++g) {
+            if (!mbar_wait(bar(kBarPReady + g), it & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(g, s, it > 0);
+            if (g == 1) mma_commit(bar(kBarKvEmpty + s));
+            if (it + 1 < nkt) {
+              if (g == 0) {
+                if (!mbar_wait(bar(kBarKvFull + sn), ((it + 1) / kStages) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+              }
+              issue_qk(g, sn);
+              mma_commit(bar(kBarSFull + g));
+            }
+          }
         }
-        s[nt][r] = x;
-        mx[hf] = fmaxf(mx[hf], x);
+      }
+      mma_commit(bar(kBarOFull + 0));
+      mma_commit(bar(kBarOFull + 1));
+      if (!ok) {
+        // drain: wait (bounded, ignoring the abort flag) until issued MMAs are done
+        mma_commit(bar(kBarDrain));
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+        }
       }
     }
-    float alpha[2];
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(0xffffffffu, mx[hf], 1));
-      mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(0xffffffffu, mx[hf], 2));
-      const float m_new = fmaxf(m_run[hf], mx[hf]);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      alpha[hf] = exp2f(m_run[hf] - m_use);
-      m_run[hf] = m_new;
-      mx[hf] = m_use;
-      l_run[hf] *= alpha[hf];
-    }
-#pragma unroll
-    for (int dt = 0; dt < 8; ++dt) {
-      o[dt][0] *= alpha[0]; o[dt][1] *= alpha[0];
-      o[dt][2] *= alpha[1]; o[dt][3] *= alpha[1];
-    }
-    uint32_t pa[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float pv = exp2f(s[nt][r] - mx[r >> 1]);
-        s[nt][r] = pv;
-        l_run[r >> 1] += pv;
-      }
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      pa[kk][0] = DT<T>::pack(s[2 * kk][0], s[2 * kk][1]);
-      pa[kk][1] = DT<T>::pack(s[2 * kk][2], s[2 * kk][3]);
-      pa[kk][2] = DT<T>::pack(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[kk][3] = DT<T>::pack(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-    }
-    mma_ab<T, 4>(o, pa, sV, 0, lane);
-    __syncthreads();
   }
-  cp_async_wait<0>();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+    // ------------------------------------------------------------ softmax
+    const int g = (warp - 4) >> 2;
+    const int wl = warp & 3;
+    const int r = wl * 32 + lane;
+    const int qtile = (q0 >> 7) + g;
+    const int i = q0 + g * kBQ + r;
+    const bool rok = i < N;
+    const uint32_t t_lane = (uint32_t)(wl * 32) << 16;
+    const uint32_t tS = tmem + t_lane + (uint32_t)g * 128;
+    const uint32_t tO = tmem + t_lane + 256 + (uint32_t)g * 64;
+    const float sc = p.tau * kLog2e;
+    const float* zq_row = nullptr;
+    float crow_lo = 0.f, crow_hi = 0.f;
+    if (rok) {
+      // saturated columns e = 0 / R_exp - 1 (present in the row's group whenever a
+      // CONST tile can occur for it)
+      const GroupInfo gi = p.gq[qtile];
+      if (AQ) {
+        zq_row = t.zq + (size_t)bh * p.zq_head + gi.base + (long long)(i - qtile * kBQ) * gi.S - gi.e0;
+        if (gi.e0 == 0) crow_lo += __ldg(zq_row);
+        if (gi.e0 + gi.W >= p.Rexp) crow_hi += __ldg(zq_row + p.Rexp - 1);
+      }
+      if (BIAS) {
+        crow_lo += __ldg(t.b_exp + (size_t)h * p.Rexp);
+        crow_hi += __ldg(t.b_exp + (size_t)h * p.Rexp + p.Rexp - 1);
+      }
+    }
+    crow_lo *= sc;
+    crow_hi *= sc;
+    const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
+    float* colv_base = reinterpret_cast<float*>(sg + kOffColv) + g * 2 * kBK;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    int colv_uses = 0;
+    for (int it = 0; it < nkt; ++it) {
+      const int j0 = it * kBK;
+      const int cls = tile_class(qtile, it, N, nkv, p.causal, p.E_lo, p.E_hi);
+      const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
+      float* cv = colv_base + (it & 1) * kBK;
+      if (AK && is_const) {
+        float z = 0.f;
+        if (j0 + r < N) {
+          const GroupInfo gk = p.gk[it];
+          const int e = cls == RELPOS_TILE_CONST_LO ? 0 : p.Rexp - 1;
+          z = __ldg(t.zk + (size_t)bh * p.zk_head + gk.base + (long long)r * gk.S + e - gk.e0) * sc;
+        }
+        cv[r] = z;
+        mbar_arrive(bar(kBarColv + g));
+        if (!mbar_wait(bar(kBarColv + g), colv_uses & 1, abort_flag)) { ok = false; break; }
+        ++colv_uses;
+      }
+      if (!mbar_wait(bar(kBarSFull + g), it & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tS + 0, sr + 0);
+      tmem_ld32(tS + 32, sr + 32);
+      tmem_ld32(tS + 64, sr + 64);
+      tmem_ld32(tS + 96, sr + 96);
+      tmem_wait_ld();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+      float rowc = 0.f;
+      if (is_const) {
+        rowc = cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi;
+        if (AK) {
+#pragma unroll
+          for (int c = 0; c < 128; c += 4) {
+            const float4 v4 = *reinterpret_cast<const float4*>(cv + c);
+            x[c] = fmaf(x[c], sc, v4.x);
+            x[c + 1] = fmaf(x[c + 1], sc, v4.y);
+            x[c + 2] = fmaf(x[c + 2], sc, v4.z);
+            x[c + 3] = fmaf(x[c + 3], sc, v4.w);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] *= sc;
+        }
+      } else {
+        const float* zk_tile = nullptr;
+        int zS = 0;
+        if (AK) {
+          const GroupInfo gk = p.gk[it];
+          zk_tile = t.zk + (size_t)bh * p.zk_head + gk.base - gk.e0;
+          zS = gk.S;
+        }
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          float rel = 0.f;
+          const int j = j0 + c;
+          // only kept cells: a masked cell's offset may lie outside the stored columns
+          if (rok && j < nkv && !(p.causal && j > i)) {
+            const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
+            if (AQ) rel += __ldg(zq_row + e);
+            if (AK) rel += __ldg(zk_tile + (long long)c * zS + e);
+            if (BIAS) rel += __ldg(bexp + e);
+          }
+          x[c] = (x[c] + rel) * sc;
+        }
+      }
+      const bool need_mask = (j0 + kBK > nkv) || (p.causal && j0 + kBK - 1 > q0 + g * kBQ);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int j = j0 + c;
+          if (j >= nkv || (p.causal && j > i)) x[c] = -INFINITY;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      mx += rowc;
+      const float m_new = fmaxf(m_run, mx);
+      if (m_new > m_run + kRescaleThreshold) {
+        const float alpha = exp2f(m_run - m_new);
+        if (it > 0) {
+          uint32_t ov[64];
+          tmem_ld32(tO + 0, ov);
+          tmem_ld32(tO + 32, ov + 32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 64; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st32(tO + 0, ov);
+          tmem_st32(tO + 32, ov + 32);
+        }
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        x[c] = exp2f(x[c] - msub);
+        lsum += x[c];
+      }
+      l_run += lsum;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) pk[c] = DT<T>::pack(x[2 * c], x[2 * c + 1]);
+      tmem_st32(tS + 0, pk);
+      tmem_st32(tS + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPReady + g));
+    }
+    // ------------------------------------------------------------ epilogue
+    float ov[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) ov[c] = 0.f;
+    if (nkt > 0 && ok && mbar_wait(bar(kBarOFull + g), 0, abort_flag)) {
+      tc_fence_after();
+      uint32_t u[64];
+      tmem_ld32(tO + 0, u);
+      tmem_ld32(tO + 32, u + 32);
+      tmem_wait_ld();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) ov[c] = __uint_as_float(u[c]) * inv;
+    }
+    if (rok) {
+      OutT* O = static_cast<OutT*>(t.o) + ((size_t)bh * N + i) * 64;
+      RowStore<OutT>::row(O, ov);
+      t.lse[(size_t)bh * N + i] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag && t.status) *t.status = kStatusTimeout;
+}
 
-  OutT* O = static_cast<OutT*>(t.o) + off;
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    float l = l_run[hf];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const int i = irow[hf];
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (i < N) {
-#pragma unroll
-      for (int dt = 0; dt < 8; ++dt)
-        Store<OutT>::two(O + (size_t)i * 64 + dt * 8 + 2 * tq, o[dt][2 * hf] * inv, o[dt][2 * hf + 1] * inv);
-      if (tq == 0) t.lse[(size_t)bh * N + i] = l > 0.f ? (m_run[hf] + log2f(l)) * kLn2 : -INFINITY;
-    }
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   }
+  return fn;
+}
+
+// [BH, N, 64] 16-bit tensor viewed as 3-D for TMA: 128-row boxes, 128-byte
+// swizzle, rows past N read as zero.
+bool make_rows_map(CUtensorMap* m, const void* base, int BH, int N, bool bf16) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 template <typename T, typename OutT>
 cudaError_t launch_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   const int mask = (t.aq_exp ? 1 : 0) | (t.ak_exp ? 2 : 0) | (t.b_exp ? 4 : 0);
-  void (*kern)(const Plan, const Tensors) = nullptr;
+  void (*kern)(const Plan, const Tensors, const CUtensorMap, const CUtensorMap, const CUtensorMap) = nullptr;
   switch (mask) {
-    case 0: kern = fwd_kernel<T, OutT, false, false, false>; break;
-    case 1: kern = fwd_kernel<T, OutT, true, false, false>; break;
-    case 2: kern = fwd_kernel<T, OutT, false, true, false>; break;
-    case 3: kern = fwd_kernel<T, OutT, true, true, false>; break;
-    case 4: kern = fwd_kernel<T, OutT, false, false, true>; break;
-    case 5: kern = fwd_kernel<T, OutT, true, false, true>; break;
-    case 6: kern = fwd_kernel<T, OutT, false, true, true>; break;
-    default: kern = fwd_kernel<T, OutT, true, true, true>; break;
+    case 0: kern = fwd_sm100_kernel<T, OutT, false, false, false>; break;
+    case 1: kern = fwd_sm100_kernel<T, OutT, true, false, false>; break;
+    case 2: kern = fwd_sm100_kernel<T, OutT, false, true, false>; break;
+    case 3: kern = fwd_sm100_kernel<T, OutT, true, true, false>; break;
+    case 4: kern = fwd_sm100_kernel<T, OutT, false, false, true>; break;
+    case 5: kern = fwd_sm100_kernel<T, OutT, true, false, true>; break;
+    case 6: kern = fwd_sm100_kernel<T, OutT, false, true, true>; break;
+    default: kern = fwd_sm100_kernel<T, OutT, true, true, true>; break;
   }
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  CUtensorMap mq, mk, mv;
+  const int BH = p.B * p.H;
+  const bool bf = t.is_bf16 != 0;
+  if (!make_rows_map(&mq, t.q, BH, p.N, bf) || !make_rows_map(&mk, t.k, BH, p.N, bf) ||
+      !make_rows_map(&mv, t.v, BH, p.N, bf))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.N + kBM - 1) / kBM, p.B * p.H);
-  { kern<<<grid, kThreads, kSmem, s>>>(p, t); note_launch(1); }
+  dim3 grid((p.N + 2 * kBQ - 1) / (2 * kBQ), BH);
+  { kern<<<grid, kThreads, kSmemBytes, s>>>(p, t, mq, mk, mv); note_launch(1); }
   return cudaGetLastError();
 }
 

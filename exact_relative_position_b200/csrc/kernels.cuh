@@ -33,6 +33,7 @@ struct Tensors {
   int R;
   float *daq, *dak, *db;         // final outputs
   int is_bf16;
+  int* status;                   // device status word (0 = ok; set when a kernel's bounded wait expires)
 };
 
 // Records e as this thread's last CUDA error and returns RELPOS_ERR_CUDA.

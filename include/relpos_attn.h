@@ -151,6 +151,14 @@ int relpos_attn_fwd(const relpos_fwd_args* a, void* workspace, size_t ws_bytes, 
  * batch, both in a fixed order.  workspace: device, >= bwd_bytes. */
 int relpos_attn_bwd(const relpos_bwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream);
 
+/* Device-side status of the last call that used `workspace` (synchronous:
+ * waits for `stream`).  The fused kernels bound every wait on an mbarrier;
+ * when one expires the kernel stops its pipeline, frees its tensor memory,
+ * returns, and leaves a non-zero status word at the start of the workspace
+ * (its outputs are then invalid).  Returns RELPOS_OK, RELPOS_ERR_TIMEOUT
+ * (*device_status = 1), or RELPOS_ERR_CUDA.  device_status: host, may be NULL. */
+int relpos_check_workspace(const void* workspace, relpos_stream_t stream, int32_t* device_status);
+
 /* Human-readable text of a relpos_status (static storage). */
 const char* relpos_status_string(int status);
 
