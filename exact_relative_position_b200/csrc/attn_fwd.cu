@@ -258,10 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cv[r] = z;
         mbar_arrive(bar(kBarColv + g));
-        if (!mbar_wait(bar(kBarColv + g), colv_uses & 1, abort_flag)) { ok = false; break; }
+        const bool got = mbar_wait(bar(kBarColv + g), colv_uses & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         ++colv_uses;
       }
-      if (!mbar_wait(bar(kBarSFull + g), it & 1, abort_flag)) { ok = false; break; }
+      // every decision before a tcgen05.ld/st (warp-collective) is warp-uniform
+      const bool got_s = mbar_wait(bar(kBarSFull + g), it & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32(tS + 0, sr + 0);
@@ -323,18 +326,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
       mx += rowc;
       const float m_new = fmaxf(m_run, mx);
-      if (m_new > m_run + kRescaleThreshold) {
-        const float alpha = exp2f(m_run - m_new);
-        if (it > 0) {
-          uint32_t ov[64];
-          tmem_ld32(tO + 0, ov);
-          tmem_ld32(tO + 32, ov + 32);
-          tmem_wait_ld();
+      // lazy rescale: only rows whose maximum grew by more than the threshold
+      // move their reference point; the O access is done by the whole warp
+      const bool grow = m_new > m_run + kRescaleThreshold;
+      const float alpha = grow ? exp2f(m_run - m_new) : 1.f;
+      if (it > 0 && __any_sync(0xffffffffu, grow)) {
+        uint32_t ov[64];
+        tmem_ld32(tO + 0, ov);
+        tmem_ld32(tO + 32, ov + 32);
+        tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 64; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-          tmem_st32(tO + 0, ov);
-          tmem_st32(tO + 32, ov + 32);
-        }
+        for (int c = 0; c < 64; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+        tmem_st32(tO + 0, ov);
+        tmem_st32(tO + 32, ov + 32);
+      }
+      if (grow) {
         l_run *= alpha;
         m_run = m_new;
       }
@@ -359,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float ov[64];
 #pragma unroll
     for (int c = 0; c < 64; ++c) ov[c] = 0.f;
-    if (nkt > 0 && ok && mbar_wait(bar(kBarOFull + g), 0, abort_flag)) {
+    const bool got_o = nkt > 0 && ok && mbar_wait(bar(kBarOFull + g), 0, abort_flag);
+    if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
       uint32_t u[64];
       tmem_ld32(tO + 0, u);

@@ -113,3 +113,14 @@ def test_deterministic():
     for k in r1:
         if r1[k] is not None:
             assert np.array_equal(r1[k], r2[k]), k
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_large_scores_exercise_lazy_rescale(dtype):
+    """Scores with a spread of many units in log2 make the running row maximum
+    grow past the rescale threshold on later key tiles for many rows."""
+    w = small_workload(N=1100, B=1, H=2, terms=("aQ", "aK", "b"), tau=1.5, dtype=dtype, **MAPS["trunc16"])
+    got = run_library(w, out_f32=True)
+    want = run_oracle(w)
+    check_forward(got, want)
+    check_backward(got, want)
