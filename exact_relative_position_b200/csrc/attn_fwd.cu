@@ -345,16 +345,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       }
       const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = exp2f(x[c] - msub);
+      // the row sum is taken over the rounded probabilities the PV product
+      // uses, so the normalisation matches the weights actually applied
+      uint32_t pk[64];
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = exp2f(x[c] - msub);
-        lsum += x[c];
+      for (int c = 0; c < 64; ++c) {
+        pk[c] = DT<T>::pack(x[2 * c], x[2 * c + 1]);
+        lsum += DT<T>::pair_sum(pk[c]);
       }
       l_run += lsum;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) pk[c] = DT<T>::pack(x[2 * c], x[2 * c + 1]);
       tmem_st32(tS + 0, pk);
       tmem_st32(tS + 32, pk + 32);
       tmem_wait_st();

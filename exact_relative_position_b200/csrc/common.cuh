@@ -181,6 +181,11 @@ template <> struct DT<__half> {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
   }
+  // sum of the two packed values, as fp32
+  static __device__ __forceinline__ float pair_sum(uint32_t u) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+    return f.x + f.y;
+  }
 };
 template <> struct DT<__nv_bfloat16> {
   static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -188,6 +193,9 @@ template <> struct DT<__nv_bfloat16> {
   static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float pair_sum(uint32_t u) {
+    return __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
   }
 };
 
