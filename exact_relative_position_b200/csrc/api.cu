@@ -127,7 +127,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t status, gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
+  size_t status, zksat, gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
   size_t dsum, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
   int R, Hq, expand, nsq, nsk, nsb;
 };
@@ -175,6 +175,7 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   L->ake = (ak && L->expand) ? take((size_t)2 * L->Hq * p->Rexp * 64) : 0;
   L->zq = aq ? take(sizeof(float) * BH * p->zq_head) : 0;
   L->zk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
+  L->zksat = ak ? take(sizeof(float) * BH * 2 * (size_t)p->nT * kTile) : 0;
   L->fwd_end = off;
   L->dsum = take(sizeof(float) * BH * N);
   L->dzq = (aq || bb) ? take(sizeof(float) * BH * p->zq_head) : 0;
@@ -246,6 +247,7 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
     if (L.expand) { t.ak_exp = ws + L.ake; t.ak_hs = (long long)p.Rexp * 64; }
     else { t.ak_exp = static_cast<const uint8_t*>(a->ak) + row0 * 64 * esz; t.ak_hs = (long long)L.R * 64; }
     t.zk = reinterpret_cast<float*>(ws + L.zk);
+    t.zk_sat = reinterpret_cast<float*>(ws + L.zksat);
   }
   cudaError_t e = run_phase(PH_TABLES, s, [&] {
     return launch_build_tables(p, a->map, gq, gk, phi_exp, L.R, a->aq, a->ak, a->table_per_head, ws + L.aqe,
@@ -253,7 +255,11 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
   });
   if (e != cudaSuccess) return cuda_fail(e);
   if (a->aq || a->ak) {
-    e = run_phase(PH_PROJ, s, [&] { return launch_projection(p, t, s); });
+    e = run_phase(PH_PROJ, s, [&] {
+      cudaError_t e1 = launch_projection(p, t, s);
+      if (e1 == cudaSuccess && a->ak) e1 = launch_saturated_columns(p, t, s);
+      return e1;
+    });
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return RELPOS_OK;

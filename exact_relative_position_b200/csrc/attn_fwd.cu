@@ -41,9 +41,12 @@ constexpr int kStages = 3;
 constexpr int kThreads = 384;
 constexpr uint32_t kTileBytes = 128 * 128;   // one [128 x 64] 16-bit tile
 constexpr uint32_t kOffQ = 0;
+// A K/V stage: K tile, V tile, then the key tile's two saturated relation
+// columns tau log2e Z^K[j, 0] and [j, R_exp - 1] (128 floats each).
+constexpr uint32_t kColvBytes = 2 * kBK * 4;
+constexpr uint32_t kStageBytes = 2 * kTileBytes + 1024;   // keeps every K/V tile 1024-byte aligned
 constexpr uint32_t kOffKV = 2 * kTileBytes;
-constexpr uint32_t kOffColv = kOffKV + kStages * 2 * kTileBytes;
-constexpr uint32_t kOffBar = kOffColv + 2 * 2 * kBK * 4;
+constexpr uint32_t kOffBar = kOffKV + kStages * kStageBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;   // + alignment slack
@@ -58,7 +61,6 @@ constexpr int kBarSFull = kBarKvEmpty + kStages;
 constexpr int kBarPReady = kBarSFull + 2;
 constexpr int kBarOFull = kBarPReady + 2;
 constexpr int kBarDrain = kBarOFull + 2;
-constexpr int kBarColv = kBarDrain + 1;   // 2: saturated-column vector staged (per softmax warpgroup)
 
 template <typename OutT> struct RowStore;
 template <> struct RowStore<float> {
@@ -113,8 +115,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarOFull + g), 1);
     }
     mbar_init(bar(kBarDrain), 1);
-    mbar_init(bar(kBarColv + 0), 128);
-    mbar_init(bar(kBarColv + 1), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -144,10 +144,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < nkt; ++it) {
         const int s = it % kStages;
         if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
-        const uint32_t dst = sb + kOffKV + (uint32_t)s * 2 * kTileBytes;
-        mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes);
+        const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
+        mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
         tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kBK, bh);
         tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kBK, bh);
+        if (AK) {
+          const float* src = t.zk_sat + (size_t)bh * 2 * p.nT * kBK + (size_t)it * kBK;
+          bulk_load(dst + 2 * kTileBytes, src, kBK * 4, bar(kBarKvFull + s));
+          bulk_load(dst + 2 * kTileBytes + kBK * 4, src + (size_t)p.nT * kBK, kBK * 4, bar(kBarKvFull + s));
+        }
       }
     }
   } else if (warp == 1) {
@@ -158,14 +163,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_pv = idesc_f16(bf, 128, 64, false, true);
       auto issue_qk = [&](int g, int s) {
         const uint32_t a = sb + kOffQ + (uint32_t)g * kTileBytes;
-        const uint32_t k = sb + kOffKV + (uint32_t)s * 2 * kTileBytes;
+        const uint32_t k = sb + kOffKV + (uint32_t)s * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem + (uint32_t)g * 128, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(k + kk * 32, 16, 1024),
                  id_qk, kk > 0);
       };
       auto issue_pv = [&](int g, int s, bool acc) {
-        const uint32_t v = sb + kOffKV + (uint32_t)s * 2 * kTileBytes + kTileBytes;
+        const uint32_t v = sb + kOffKV + (uint32_t)s * kStageBytes + kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + 256 + (uint32_t)g * 64, tmem + (uint32_t)g * 128 + kk * 8,
@@ -240,30 +245,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     crow_lo *= sc;
     crow_hi *= sc;
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
-    float* colv_base = reinterpret_cast<float*>(sg + kOffColv) + g * 2 * kBK;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int colv_uses = 0;
     for (int it = 0; it < nkt; ++it) {
       const int j0 = it * kBK;
       const int cls = tile_class(qtile, it, N, nkv, p.causal, p.E_lo, p.E_hi);
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
-      float* cv = colv_base + (it & 1) * kBK;
-      if (AK && is_const) {
-        float z = 0.f;
-        if (j0 + r < N) {
-          const GroupInfo gk = p.gk[it];
-          const int e = cls == RELPOS_TILE_CONST_LO ? 0 : p.Rexp - 1;
-          z = __ldg(t.zk + (size_t)bh * p.zk_head + gk.base + (long long)r * gk.S + e - gk.e0) * sc;
-        }
-        cv[r] = z;
-        mbar_arrive(bar(kBarColv + g));
-        const bool got = mbar_wait(bar(kBarColv + g), colv_uses & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        ++colv_uses;
-      }
+      const int stage = it % kStages;
+      const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
+                        (cls == RELPOS_TILE_CONST_LO ? 0 : kBK);
       // every decision before a tcgen05.ld/st (warp-collective) is warp-uniform
-      const bool got_s = mbar_wait(bar(kBarSFull + g), it & 1, abort_flag);
+      // S ready implies the stage's TMA data landed; waiting on the stage's own
+      // barrier as well makes its saturated columns visible to these threads
+      const bool got_s = mbar_wait(bar(kBarSFull + g), it & 1, abort_flag) &&
+                         (!AK || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
@@ -354,7 +349,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         pk[c] = DT<T>::pack(x[2 * c], x[2 * c + 1]);
-        lsum += DT<T>::pair_sum(pk[c]);
+        // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
+        // enough to sum the fp32 values and spare the conversions
+        lsum += DT<T>::kCoarse ? DT<T>::pair_sum(pk[c]) : x[2 * c] + x[2 * c + 1];
       }
       l_run += lsum;
       tmem_st32(tS + 0, pk);

@@ -175,6 +175,7 @@ RP_HD void tile_segments(int qi, int nT, int N, int nkv, int causal, int E_lo, i
 
 template <typename T> struct DT;
 template <> struct DT<__half> {
+  static constexpr bool kCoarse = false;
   static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
   static __device__ __forceinline__ __half from_f(float x) { return __float2half_rn(x); }
   static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
@@ -188,6 +189,7 @@ template <> struct DT<__half> {
   }
 };
 template <> struct DT<__nv_bfloat16> {
+  static constexpr bool kCoarse = true;
   static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
   static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
   static __device__ __forceinline__ uint32_t pack(float lo, float hi) {

@@ -14,6 +14,7 @@ struct Tensors {
   long long aq_hs, ak_hs;        // head stride (elements) of the expanded tables when per head
   const float* b_exp;            // [H][Rexp] or null
   float *zq, *zk;                // projections (grouped layout), or null
+  float* zk_sat;                 // [B*H][2][nT*128]: tau log2e Z^K[j, 0] and Z^K[j, R_exp-1], zero past N
   void* o;
   int o_f32;
   float* lse;
@@ -48,6 +49,7 @@ cudaError_t launch_build_tables(const Plan& p, const relpos_map_desc& map, Group
                                 int expand_tables, cudaStream_t s);
 cudaError_t launch_fold_ranges(const Plan& p, const int* phi_exp, int R, int* fold_lo, int* fold_hi, cudaStream_t s);
 cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_forward(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s);

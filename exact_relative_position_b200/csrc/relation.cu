@@ -108,6 +108,28 @@ __global__ void __launch_bounds__(256) projection_kernel(const Plan p, const int
   }
 }
 
+// ------------------------------------------------------------------ saturated key columns
+// out[bh][0][j] = tau log2e Z^K[j, 0], out[bh][1][j] = tau log2e Z^K[j, R_exp - 1]
+// (zero where the key's group does not store the column or j >= N), laid out
+// contiguously so the fused forward can bulk-copy one key tile's worth.
+__global__ void saturated_columns_kernel(const Plan p, const float* __restrict__ zk, float* __restrict__ out,
+                                         const float scale) {
+  const int npad = p.nT * kTile;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)p.B * p.H * npad) return;
+  const int j = (int)(idx % npad);
+  const long long bh = idx / npad;
+  float lo = 0.f, hi = 0.f;
+  if (j < p.N) {
+    const GroupInfo gi = p.gk[j / kTile];
+    const float* row = zk + bh * p.zk_head + gi.base + (long long)(j % kTile) * gi.S - gi.e0;
+    if (gi.e0 == 0) lo = row[0] * scale;
+    if (gi.e0 + gi.W >= p.Rexp) hi = row[p.Rexp - 1] * scale;
+  }
+  out[(bh * 2 + 0) * npad + j] = lo;
+  out[(bh * 2 + 1) * npad + j] = hi;
+}
+
 // ------------------------------------------------------------------ relgrad rows
 // out[rows of group g] = acc_in[rows] + dZ_g[rows, :W] A_exp[e0 .. e0 + W)   (tf32 tensor cores)
 constexpr int kRowPitchA = 36;   // floats, dZ chunk [128][32]
@@ -353,6 +375,12 @@ static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_
     { projection_kernel<T><<<grid, 256, kProjSmem, s>>>(p, 1, (const T*)t.k, (const T*)t.ak_exp,
                                                       t.table_per_head ? t.ak_hs : 0, t.zk, p.zk_head); note_launch(1); }
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream_t s) {
+  const long long n = (long long)p.B * p.H * p.nT * kTile;
+  { saturated_columns_kernel<<<nblk(n, 256), 256, 0, s>>>(p, t.zk, t.zk_sat, p.tau * kLog2e); note_launch(1); }
   return cudaGetLastError();
 }
 
