@@ -6,23 +6,26 @@
 // One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and
 // walks the key tiles once for both, so each K/V tile that TMA brings into
 // shared memory feeds four tcgen05 GEMMs.  Warp roles:
-//   warp 0       TMA producer: Q0/Q1 once, then K/V tiles into a 3-stage ring
+//   warp 0       TMA producer: Q0/Q1 once, then K/V tiles (and the key
+//                tile's saturated relation columns) into a 3-stage ring
 //   warp 1       MMA issuer (one thread): S_g = Q_g K^T into tensor memory,
-//                O_g += P_g V with P_g read back from tensor memory
-//   warp 2       allocates / frees the 512 tensor-memory columns
+//                O_g += P_g V with P_g from shared memory
+//   warp 2       allocates / frees the tensor-memory columns
 //   warps 4..7   softmax of Q0 (thread r owns row r = TMEM lane r)
 //   warps 8..11  softmax of Q1
-// Tensor memory: S0 cols [0,128), S1 [128,256) (P_g overwrites the first 64
-// columns of S_g as packed 16-bit pairs), O0 [256,320), O1 [320,384).
+// Tensor memory: S0 cols [0,128), S1 [128,256), O0 [256,320), O1 [320,384).
+// A softmax warpgroup releases S_g as soon as it has read it into registers,
+// so the GEMM of the next key tile runs while it computes; its 16-bit P_g
+// goes to a 128-byte-swizzled shared-memory tile that the PV GEMM reads.
 //
 // Relation terms are added to the scores in registers.  A key tile whose
 // every offset saturates (CONST_LO / CONST_HI: two comparisons of the tile's
 // offset range with E_lo / E_hi) adds one per-row constant tau (Z^Q_i,sat +
-// b_sat) and one per-column vector tau Z^K_j,sat staged once in shared memory
-// and broadcast; a BAND tile gathers Z^Q[i, e], Z^K[j, e] and b[e] per score
-// with e = clamp(j - i, E_lo, E_hi) - E_lo.  The online softmax runs in base 2
-// and only rescales O when the running row maximum grows by more than 8
-// (a factor 256), which keeps every P <= 256 and the result exact.
+// b_sat) and one per-column vector tau Z^K_j,sat staged with the K/V tile and
+// broadcast; a BAND tile gathers Z^Q[i, e], Z^K[j, e] and b[e] per score with
+// e = clamp(j - i, E_lo, E_hi) - E_lo.  The online softmax runs in base 2 and
+// only rescales O when the running row maximum grows by more than 8 (a
+// factor 256), which keeps every P <= 256 and the result exact.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -46,7 +49,10 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kColvBytes = 2 * kBK * 4;
 constexpr uint32_t kStageBytes = 2 * kTileBytes + 1024;   // keeps every K/V tile 1024-byte aligned
 constexpr uint32_t kOffKV = 2 * kTileBytes;
-constexpr uint32_t kOffBar = kOffKV + kStages * kStageBytes;
+// P_g: [128 rows x 128 keys] 16-bit, two 64-key swizzle atoms of 16 KB
+constexpr uint32_t kOffP = kOffKV + kStages * kStageBytes;
+constexpr uint32_t kPBytes = 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;   // + alignment slack
@@ -57,10 +63,24 @@ constexpr float kRescaleThreshold = 8.0f;              // log2 of the largest P 
 constexpr int kBarQ = 0;
 constexpr int kBarKvFull = 1;
 constexpr int kBarKvEmpty = kBarKvFull + kStages;
-constexpr int kBarSFull = kBarKvEmpty + kStages;
-constexpr int kBarPReady = kBarSFull + 2;
-constexpr int kBarOFull = kBarPReady + 2;
-constexpr int kBarDrain = kBarOFull + 2;
+constexpr int kBarSFull = kBarKvEmpty + kStages;   // 2: S_g written (MMA commit)
+constexpr int kBarSFree = kBarSFull + 2;           // 2: S_g read into registers (128 arrivals)
+constexpr int kBarPReady = kBarSFree + 2;          // 2: P_g written to shared memory (128 arrivals)
+constexpr int kBarPFree = kBarPReady + 2;          // 2: PV_g done: P_g buffer and O_g free (MMA commit)
+constexpr int kBarDrain = kBarPFree + 2;
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 template <typename OutT> struct RowStore;
 template <> struct RowStore<float> {
@@ -111,8 +131,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(kBarSFull + g), 1);
+      mbar_init(bar(kBarSFree + g), 128);
       mbar_init(bar(kBarPReady + g), 128);
-      mbar_init(bar(kBarOFull + g), 1);
+      mbar_init(bar(kBarPFree + g), 1);
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -132,9 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // two softmax warpgroups take 224: 128 x 56 + 256 x 224 = 64512.
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && nkt > 0) {
+    if (warp == 0 && lane == 0 && nkt > 0) {
+      // ---------------------------------------------------------- TMA producer
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
@@ -154,10 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(dst + 2 * kTileBytes + kBK * 4, src + (size_t)p.nT * kBK, kBK * 4, bar(kBarKvFull + s));
         }
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nkt > 0) {
+    } else if (warp == 1 && lane == 0 && nkt > 0) {
+      // ---------------------------------------------------------- MMA issuer
+      // order per key tile t: S_0(t+1), S_1(t+1) as soon as S_g(t) has been
+      // read, then PV_0(t), PV_1(t) as soon as P_g(t) is in shared memory
       const bool bf = t.is_bf16 != 0;
       const uint32_t id_qk = idesc_f16(bf, 128, 128, false, false);
       const uint32_t id_pv = idesc_f16(bf, 128, 64, false, true);
@@ -171,9 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int g, int s, bool acc) {
         const uint32_t v = sb + kOffKV + (uint32_t)s * kStageBytes + kTileBytes;
+        const uint32_t pp = sb + kOffP + (uint32_t)g * kPBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256 + (uint32_t)g * 64, tmem + (uint32_t)g * 128 + kk * 8,
+          mma_ss(tmem + 256 + (uint32_t)g * 64, sdesc_sw128(pp + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
                  sdesc_sw128(v + kk * 2048, 8192, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
@@ -185,25 +206,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar(kBarSFull + 1));
         for (int it = 0; it < nkt && ok; ++it) {
           const int s = it % kStages;
-          const int sn = (it + 1) % kStages;
-          for (int g = 0; g < 2; ++g) {
-            if (!mbar_wait(bar(kBarPReady + g), it & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(g, s, it > 0);
-            if (g == 1) mma_commit(bar(kBarKvEmpty + s));
-            if (it + 1 < nkt) {
-              if (g == 0) {
-                if (!mbar_wait(bar(kBarKvFull + sn), ((it + 1) / kStages) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-              }
+          if (it + 1 < nkt) {
+            const int sn = (it + 1) % kStages;
+            ok = mbar_wait(bar(kBarKvFull + sn), ((it + 1) / kStages) & 1, abort_flag);
+            for (int g = 0; g < 2 && ok; ++g) {
+              ok = mbar_wait(bar(kBarSFree + g), it & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
               issue_qk(g, sn);
               mma_commit(bar(kBarSFull + g));
             }
           }
+          for (int g = 0; g < 2 && ok; ++g) {
+            ok = mbar_wait(bar(kBarPReady + g), it & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(g, s, it > 0);
+            mma_commit(bar(kBarPFree + g));
+          }
+          if (ok) mma_commit(bar(kBarKvEmpty + s));
         }
       }
-      mma_commit(bar(kBarOFull + 0));
-      mma_commit(bar(kBarOFull + 1));
       if (!ok) {
         // drain: wait (bounded, ignoring the abort flag) until issued MMAs are done
         mma_commit(bar(kBarDrain));
@@ -212,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
     // ------------------------------------------------------------ softmax
@@ -225,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = (uint32_t)(wl * 32) << 16;
     const uint32_t tS = tmem + t_lane + (uint32_t)g * 128;
     const uint32_t tO = tmem + t_lane + 256 + (uint32_t)g * 64;
+    const uint32_t pbase = sb + kOffP + (uint32_t)g * kPBytes + (uint32_t)r * 128;
     const float sc = p.tau * kLog2e;
     const float* zq_row = nullptr;
     float crow_lo = 0.f, crow_hi = 0.f;
@@ -254,9 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int stage = it % kStages;
       const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
                         (cls == RELPOS_TILE_CONST_LO ? 0 : kBK);
-      // every decision before a tcgen05.ld/st (warp-collective) is warp-uniform
-      // S ready implies the stage's TMA data landed; waiting on the stage's own
-      // barrier as well makes its saturated columns visible to these threads
+      // every decision before a tcgen05.ld/st (warp-collective) is warp-uniform;
+      // S ready implies the stage's TMA data landed, and waiting on the stage's
+      // own barrier as well makes its saturated columns visible to these threads
       const bool got_s = mbar_wait(bar(kBarSFull + g), it & 1, abort_flag) &&
                          (!AK || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
@@ -267,10 +290,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 64, sr + 64);
       tmem_ld32(tS + 96, sr + 96);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + g));    // the next key tile's S_g may now be written
       float x[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
-      float rowc = 0.f;
+      // x holds the scaled score (without the row constant rowc) in base 2;
+      // for a saturated tile without key-side terms the scale is applied in
+      // the exponent instead (xs = sc) to save one pass
+      float rowc = 0.f, xs = 1.f;
       if (is_const) {
         rowc = cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi;
         if (AK) {
@@ -283,8 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             x[c + 3] = fmaf(x[c + 3], sc, v4.w);
           }
         } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] *= sc;
+          xs = sc;
         }
       } else {
         const float* zk_tile = nullptr;
@@ -316,16 +343,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j >= nkv || (p.causal && j > i)) x[c] = -INFINITY;
         }
       }
-      float mx = x[0];
+      // 8 independent partial maxima (three-input max) keep the chains short
+      float pm[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
-      mx += rowc;
+      for (int u = 0; u < 8; ++u) pm[u] = max3(x[u], x[u + 8], x[u + 16]);
+#pragma unroll
+      for (int c = 24; c < 128; c += 16) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pm[u] = max3(pm[u], x[c + u], c + 8 + u < 128 ? x[c + 8 + u] : pm[u]);
+      }
+      float mx = max3(max3(pm[0], pm[1], pm[2]), max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+      mx = mx * xs + rowc;
       const float m_new = fmaxf(m_run, mx);
       // lazy rescale: only rows whose maximum grew by more than the threshold
-      // move their reference point; the O access is done by the whole warp
+      // move their reference point; O is touched by the whole warp once
+      // PV of the previous key tile is done
       const bool grow = m_new > m_run + kRescaleThreshold;
-      const float alpha = grow ? exp2f(m_run - m_new) : 1.f;
+      const float alpha = grow ? fast_exp2(m_run - m_new) : 1.f;
+      bool pfree_seen = it == 0;
       if (it > 0 && __any_sync(0xffffffffu, grow)) {
+        const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        pfree_seen = true;
+        tc_fence_after();
         uint32_t ov[64];
         tmem_ld32(tO + 0, ov);
         tmem_ld32(tO + 32, ov + 32);
@@ -334,37 +374,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 64; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
         tmem_st32(tO + 0, ov);
         tmem_st32(tO + 32, ov + 32);
+        tmem_wait_st();
       }
       if (grow) {
         l_run *= alpha;
         m_run = m_new;
       }
+      // p = 2^(x * xs + rowc - m_run)
       const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = exp2f(x[c] - msub);
-      // the row sum is taken over the rounded probabilities the PV product
-      // uses, so the normalisation matches the weights actually applied
+      for (int c = 0; c < 128; ++c) x[c] = fast_exp2(fmaf(x[c], xs, -msub));
       uint32_t pk[64];
-      float lsum = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         pk[c] = DT<T>::pack(x[2 * c], x[2 * c + 1]);
         // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
         // enough to sum the fp32 values and spare the conversions
-        lsum += DT<T>::kCoarse ? DT<T>::pair_sum(pk[c]) : x[2 * c] + x[2 * c + 1];
+        ps[c & 7] += DT<T>::kCoarse ? DT<T>::pair_sum(pk[c]) : x[2 * c] + x[2 * c + 1];
       }
-      l_run += lsum;
-      tmem_st32(tS + 0, pk);
-      tmem_st32(tS + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before();
+      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      // P_g of the previous key tile must have been consumed by its PV GEMM
+      if (!pfree_seen) {
+        const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+      // row r of P: 16 chunks of 16 bytes in two 64-key swizzle atoms
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t addr = pbase + (uint32_t)(c >> 3) * kTileBytes + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+        st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
       mbar_arrive(bar(kBarPReady + g));
     }
     // ------------------------------------------------------------ epilogue
     float ov[64];
 #pragma unroll
     for (int c = 0; c < 64; ++c) ov[c] = 0.f;
-    const bool got_o = nkt > 0 && ok && mbar_wait(bar(kBarOFull + g), 0, abort_flag);
+    const bool got_o = nkt > 0 && ok && mbar_wait(bar(kBarPFree + g), (nkt - 1) & 1, abort_flag);
     if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
       uint32_t u[64];
