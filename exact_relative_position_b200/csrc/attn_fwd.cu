@@ -181,21 +181,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool bf = t.is_bf16 != 0;
       const uint32_t id_qk = idesc_f16(bf, 128, 128, false, false);
       const uint32_t id_pv = idesc_f16(bf, 128, 64, false, true);
+      // descriptors are built once; a K step inside a 128-byte swizzle atom
+      // advances the start address by 32 bytes (+2 in the descriptor), a V
+      // step by 16 keys = 2048 bytes (+128), a P step across atoms by 16 KB
+      const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sb + kOffKV, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 8192, 1024);
+      const uint64_t dp0 = sdesc_sw128(sb + kOffP, 16, 1024);
+      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4, kP16 = kPBytes >> 4;
       auto issue_qk = [&](int g, int s) {
-        const uint32_t a = sb + kOffQ + (uint32_t)g * kTileBytes;
-        const uint32_t k = sb + kOffKV + (uint32_t)s * kStageBytes;
+        const uint64_t a = dq0 + (uint64_t)g * kTile16;
+        const uint64_t k = dk0 + (uint64_t)s * kStage16;
+        const uint32_t d = tmem + (uint32_t)g * 128;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + (uint32_t)g * 128, sdesc_sw128(a + kk * 32, 16, 1024), sdesc_sw128(k + kk * 32, 16, 1024),
-                 id_qk, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) mma_ss(d, a + 2 * kk, k + 2 * kk, id_qk, kk > 0);
       };
       auto issue_pv = [&](int g, int s, bool acc) {
-        const uint32_t v = sb + kOffKV + (uint32_t)s * kStageBytes + kTileBytes;
-        const uint32_t pp = sb + kOffP + (uint32_t)g * kPBytes;
+        const uint64_t v = dv0 + (uint64_t)s * kStage16;
+        const uint64_t pp = dp0 + (uint64_t)g * kP16;
+        const uint32_t d = tmem + 256 + (uint32_t)g * 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + 256 + (uint32_t)g * 64, sdesc_sw128(pp + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(v + kk * 2048, 8192, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
+          mma_ss(d, pp + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), v + 128 * kk, id_pv, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
       if (ok) {
