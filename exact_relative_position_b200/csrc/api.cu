@@ -128,7 +128,7 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
   size_t status, zksat, gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
-  size_t dsum, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
+  size_t dsum, lse2, zqsat, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
   int R, Hq, expand, nsq, nsk, nsb;
 };
 
@@ -177,7 +177,10 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   L->zk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
   L->zksat = ak ? take(sizeof(float) * BH * 2 * (size_t)p->nT * kTile) : 0;
   L->fwd_end = off;
-  L->dsum = take(sizeof(float) * BH * N);
+  const size_t npad = (size_t)p->nT * kTile;
+  L->dsum = take(sizeof(float) * BH * npad);
+  L->lse2 = take(sizeof(float) * BH * npad);
+  L->zqsat = (aq || bb) ? take(sizeof(float) * BH * 2 * npad) : 0;
   L->dzq = (aq || bb) ? take(sizeof(float) * BH * p->zq_head) : 0;
   L->dzk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
   L->dqacc = aq ? take(sizeof(float) * BH * N * 64) : 0;
@@ -332,10 +335,15 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   if (st) return st;
   t.dout = g->dout;
   t.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  t.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   t.dq = g->dq; t.dk = g->dk; t.dv = g->dv;
   t.daq = g->daq; t.dak = g->dak; t.db = g->db;
   const size_t BH = (size_t)a->B * a->H;
   cudaError_t e;
+  if (a->aq || a->b) {
+    t.zq_sat = reinterpret_cast<float*>(ws + L.zqsat);
+    if ((e = run_phase(PH_PROJ, s, [&] { return launch_saturated_rows(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  }
   if (a->aq || a->b) {
     t.dzq = reinterpret_cast<float*>(ws + L.dzq);
     e = cudaMemsetAsync(t.dzq, 0, sizeof(float) * BH * p.zq_head, s);

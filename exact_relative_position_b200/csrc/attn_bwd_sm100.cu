@@ -1,0 +1,1011 @@
+// attn_bwd_sm100.cu -- two-pass backward of exact relative-position attention
+// on sm_100a (digest of "Fast and Exact Relative-Position Attention via
+// Structure-Aware Kernels": backward section, Eq. (4), "constant tiles and
+// the saturated region").
+//
+//   prep         D_i = sum_c dO_ic O_ic and LSE_i log2 e, padded to whole tiles
+//   Q-parallel   one CTA per 128 query rows: S = Q K^T and dP = dO V^T on
+//                tcgen05 into tensor memory, P = 2^(S' - LSE'), dS = P (dP - D)
+//                in registers, dQ += dS K on tcgen05; the query-side relation
+//                gradient is written by offset (one key per interior offset,
+//                so a plain store by the row's owner) and the two saturated
+//                offsets are summed on chip and stored once per row.
+//   K-parallel   one CTA per 128 keys: S^T = K Q^T, dP^T = V dO^T,
+//                dV += P^T dO, dK += dS^T Q, and the key-side relation
+//                gradient by offset in the same single-writer way.
+// No gradient entry has two writers: no atomics, fixed summation order.
+//
+// Pipelining (both passes): the score GEMM of tile t+2 and the dP GEMM of
+// tile t+1 are issued while the compute warps work on tile t, with two score
+// buffers and one dP buffer in tensor memory.  Compute threads own one row of
+// the tile (its tensor-memory lane) and write the 16-bit P / dS operands of
+// the next GEMMs into 128-byte-swizzled shared-memory tiles.  Every mbarrier
+// wait is bounded (see sm100.cuh).
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+#include "warp_mma.cuh"
+
+namespace relpos {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kT = 128;                       // rows / keys per tile
+constexpr uint32_t kTileBytes = 128 * 128;    // one [128 x 64] 16-bit tile
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-bit [128 rows x 128 cols] K-major tile as two 64-column swizzle atoms:
+// address of the 16-byte chunk c (0..15) of row r.
+__device__ __forceinline__ uint32_t op_chunk(uint32_t base, int r, int c) {
+  return base + (uint32_t)(c >> 3) * kTileBytes + (uint32_t)r * 128 + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+}
+
+// ------------------------------------------------------------------ prep
+// dsum[bh][i] = sum_c dO_ic O_ic and lse2[bh][i] = LSE_i log2 e for i < N;
+// rows past N (up to a whole tile) get D = 0 and LSE = +inf (so P = 0).  A
+// row whose keys were all masked (LSE = -inf) also gets +inf.
+template <typename OT, typename T>
+__global__ void __launch_bounds__(256) prep_sm100_kernel(const OT* __restrict__ o, const T* __restrict__ dout,
+                                                         const float* __restrict__ lse, float* __restrict__ dsum,
+                                                         float* __restrict__ lse2, int N, int npad, long long BH) {
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = gt >> 3;
+  const int part = (int)(gt & 7);
+  const long long bh = row / npad;
+  const int i = (int)(row - bh * npad);
+  float acc = 0.f;
+  const bool ok = bh < BH && i < N;
+  if (ok) {
+    const size_t off = ((size_t)bh * N + i) * 64 + part * 8;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc += (float)o[off + c] * (float)dout[off + c];
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  if (bh < BH && part == 0) {
+    dsum[row] = acc;
+    float l2 = INFINITY;
+    if (ok) {
+      const float l = lse[(size_t)bh * N + i];
+      if (l != -INFINITY) l2 = l * kLog2e;
+    }
+    lse2[row] = l2;
+  }
+}
+
+// ------------------------------------------------------------------ Q-parallel
+namespace qp {
+constexpr int kThreads = 256;                 // warps 0..3: TMA, MMA, TMEM alloc, idle; 4..7 compute
+constexpr int kStages = 4;
+constexpr uint32_t kColvBytes = 2 * kT * 4;
+constexpr uint32_t kStageBytes = 2 * kTileBytes + 1024;   // K, V, saturated key columns
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffDO = kTileBytes;
+constexpr uint32_t kOffKV = 2 * kTileBytes;
+constexpr uint32_t kOffDS = kOffKV + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
+constexpr uint32_t kOffAbort = kOffBar + 256;
+constexpr uint32_t kOffTmem = kOffAbort + 16;
+constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;
+// tensor memory: S buffers [0,128) and [128,256), dP [256,384), dQ [384,448)
+constexpr uint32_t kTmDP = 256, kTmDQ = 384;
+// barriers
+constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kStages, kBarSFull = kBarKvEmpty + kStages,
+              kBarSFree = kBarSFull + 2, kBarDpFull = kBarSFree + 2, kBarDpFree = kBarDpFull + 1,
+              kBarDsReady = kBarDpFree + 1, kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
+}  // namespace qp
+
+// Relation terms (scaled by tau log2 e) of one row of a BAND tile, added in
+// place to the 128 raw scores x[] (kept cells only: a masked cell's offset may
+// lie outside the stored projection columns).  In chunks of 32 columns so the
+// compiler cannot hoist all gathers at once and keeps registers bounded.
+template <bool AQ, bool AK, bool BIAS>
+__device__ __forceinline__ void band_terms(float (&x)[128], const Plan& p, int i, int j0, int nkv, bool rok,
+                                           const float* zq_row, const float* zk_tile, int zS, const float* bexp,
+                                           float sc) {
+#pragma unroll
+  for (int c0 = 0; c0 < 128; c0 += 32) {
+#pragma unroll
+    for (int c = c0; c < c0 + 32; ++c) {
+      float rel = 0.f;
+      const int j = j0 + c;
+      if (rok && j < nkv && !(p.causal && j > i)) {
+        const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
+        if (AQ) rel += __ldg(zq_row + e);
+        if (AK) rel += __ldg(zk_tile + (long long)c * zS + e);
+        if (BIAS) rel += __ldg(bexp + e);
+      }
+      x[c] = (x[c] + rel) * sc;
+    }
+    asm volatile("" ::: "memory");
+  }
+}
+
+template <typename T, bool AQ, bool AK, bool BIAS, bool DZQ, bool DQ32>
+__global__ void __launch_bounds__(qp::kThreads, 1)
+    dq_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmDO) {
+  using namespace qp;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sg = smem_raw + (sb - raw);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + kOffAbort);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sg + kOffTmem);
+  auto bar = [&](int slot) { return sb + kOffBar + 8u * (uint32_t)slot; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
+  const int N = p.N, q0 = qt * kT;
+  const int npad = p.nT * kT;
+  const int nkv = p.padding ? p.key_len[b] : N;
+  int kend = nkv;
+  if (p.causal) kend = imin(kend, imin(q0 + kT, N));
+  const int nkt = kend > 0 ? (kend + kT - 1) / kT : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQ), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarKvFull + s), 1);
+      mbar_init(bar(kBarKvEmpty + s), 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(kBarSFull + u), 1);
+      mbar_init(bar(kBarSFree + u), 128);
+    }
+    mbar_init(bar(kBarDpFull), 1);
+    mbar_init(bar(kBarDpFree), 128);
+    mbar_init(bar(kBarDsReady), 128);
+    mbar_init(bar(kBarDsFree), 1);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0 && nkt > 0) {
+      // ------------------------------------------------------------ TMA producer
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmDO);
+      mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
+      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
+      tma_load_3d(sb + kOffDO, &tmDO, bar(kBarQ), 0, q0, bh);
+#pragma unroll 1
+      for (int it = 0; it < nkt; ++it) {
+        const int s = it % kStages;
+        if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+        const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
+        mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
+        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kT, bh);
+        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kT, bh);
+        if (AK) {
+          const float* src = t.zk_sat + (size_t)bh * 2 * npad + (size_t)it * kT;
+          bulk_load(dst + 2 * kTileBytes, src, kT * 4, bar(kBarKvFull + s));
+          bulk_load(dst + 2 * kTileBytes + kT * 4, src + npad, kT * 4, bar(kBarKvFull + s));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nkt > 0) {
+      // ------------------------------------------------------------ MMA issuer
+      // per tile t: dP(t+1) once dP(t) has been read, dQ += dS(t) K(t) once
+      // dS(t) is in shared memory, S(t+2) once S(t) has been read
+      const bool bf = t.is_bf16 != 0;
+      const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
+      const uint32_t id_dq = idesc_f16(bf, 128, 64, false, true);
+      const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t ddo0 = sdesc_sw128(sb + kOffDO, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sb + kOffKV, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 16, 1024);
+      const uint64_t dkmn0 = sdesc_sw128(sb + kOffKV, 8192, 1024);
+      const uint64_t dds0 = sdesc_sw128(sb + kOffDS, 16, 1024);
+      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
+      auto issue_s = [&](int buf, int s) {
+        const uint64_t kd = dk0 + (uint64_t)s * kStage16;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dq0 + 2 * kk, kd + 2 * kk, id_s, kk > 0);
+      };
+      auto issue_dp = [&](int s) {
+        const uint64_t vd = dv0 + (uint64_t)s * kStage16;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, ddo0 + 2 * kk, vd + 2 * kk, id_s, kk > 0);
+      };
+      auto issue_dq = [&](int s, bool acc) {
+        const uint64_t kd = dkmn0 + (uint64_t)s * kStage16;
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + kTmDQ, dds0 + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), kd + 128 * kk, id_dq,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(bar(kBarSFull + 0));
+        issue_dp(0);
+        mma_commit(bar(kBarDpFull));
+        if (nkt > 1) {
+          ok = mbar_wait(bar(kBarKvFull + 1), 0, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            issue_s(1, 1);
+            mma_commit(bar(kBarSFull + 1));
+          }
+        }
+      }
+#pragma unroll 1
+      for (int it = 0; it < nkt && ok; ++it) {
+        const int s = it % kStages;
+        if (it + 1 < nkt) {
+          ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp((it + 1) % kStages);
+          mma_commit(bar(kBarDpFull));
+        }
+        ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dq(s, it > 0);
+        mma_commit(bar(kBarDsFree));
+        mma_commit(bar(kBarKvEmpty + s));
+        if (it + 2 < nkt) {
+          const int s2 = (it + 2) % kStages;
+          ok = mbar_wait(bar(kBarKvFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
+               mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it & 1, s2);
+          mma_commit(bar(kBarSFull + (it & 1)));
+        }
+      }
+      if (!ok) {
+        mma_commit(bar(kBarDrain));
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- compute
+    const int r = (warp - 4) * 32 + lane;        // row of the tile = tensor-memory lane
+    const int i = q0 + r;
+    const bool rok = i < N;
+    const uint32_t t_lane = (uint32_t)((warp & 3) * 32) << 16;
+    const float sc = p.tau * kLog2e;
+    const size_t prow = (size_t)bh * npad + q0 + r;
+    const float lse2 = t.lse2[prow];
+    const float dval = t.dsum[prow];
+    // saturated-offset row constants tau log2e (Z^Q[i, sat] + b_sat), zero past N
+    const float crow_lo = (AQ || BIAS) ? t.zq_sat[(size_t)bh * 2 * npad + q0 + r] : 0.f;
+    const float crow_hi = (AQ || BIAS) ? t.zq_sat[(size_t)bh * 2 * npad + npad + q0 + r] : 0.f;
+    const float* zq_row = nullptr;
+    float* dzq_row = nullptr;
+    GroupInfo gi{};
+    if (rok) {
+      gi = p.gq[qt];
+      const long long ro = gi.base + (long long)(i - q0) * gi.S - gi.e0;
+      if (AQ) zq_row = t.zq + (size_t)bh * p.zq_head + ro;
+      if (DZQ) dzq_row = t.dzq + (size_t)bh * p.zq_head + ro;
+    }
+    const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
+    const uint32_t dsb = sb + kOffDS;
+    float sat_lo = 0.f, sat_hi = 0.f;
+    bool ok = true;
+#pragma unroll 1
+    for (int it = 0; it < nkt; ++it) {
+      const int j0 = it * kT;
+      const int cls = tile_class(qt, it, N, nkv, p.causal, p.E_lo, p.E_hi);
+      const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
+      const int stage = it % kStages, buf = it & 1;
+      const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
+                        (cls == RELPOS_TILE_CONST_LO ? 0 : kT);
+      const bool got_s = mbar_wait(bar(kBarSFull + buf), (it >> 1) & 1, abort_flag) &&
+                         (!(AK && is_const) || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
+      if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
+      tc_fence_after();
+      float x[128];
+      {
+        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128;
+        tmem_ld32(ts + 0, reinterpret_cast<uint32_t*>(x) + 0);
+        tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
+        tmem_ld32(ts + 64, reinterpret_cast<uint32_t*>(x) + 64);
+        tmem_ld32(ts + 96, reinterpret_cast<uint32_t*>(x) + 96);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + buf));   // S(t + 2) may now be written here
+      // P = 2^(S tau log2e + relation terms - LSE log2e)
+      if (is_const) {
+        const float off = (cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi) - lse2;
+        if (AK) {
+#pragma unroll
+          for (int c = 0; c < 128; c += 4) {
+            const float4 v4 = *reinterpret_cast<const float4*>(cv + c);
+            x[c] = fast_exp2(fmaf(x[c], sc, v4.x) + off);
+            x[c + 1] = fast_exp2(fmaf(x[c + 1], sc, v4.y) + off);
+            x[c + 2] = fast_exp2(fmaf(x[c + 2], sc, v4.z) + off);
+            x[c + 3] = fast_exp2(fmaf(x[c + 3], sc, v4.w) + off);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = fast_exp2(fmaf(x[c], sc, off));
+        }
+      } else {
+        const float* zk_tile = nullptr;
+        int zS = 0;
+        if (AK) {
+          const GroupInfo gk = p.gk[it];
+          zk_tile = t.zk + (size_t)bh * p.zk_head + gk.base - gk.e0;
+          zS = gk.S;
+        }
+        band_terms<AQ, AK, BIAS>(x, p, i, j0, nkv, rok, zq_row, zk_tile, zS, bexp, sc);
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] = fast_exp2(x[c] - lse2);
+      }
+      const bool need_mask = (j0 + kT > nkv) || (p.causal && j0 + kT - 1 > q0);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int j = j0 + c;
+          if (j >= nkv || (p.causal && j > i)) x[c] = 0.f;
+        }
+      }
+      // dS = P (dP - D) in two halves of 64 keys; written as the 16-bit A
+      // operand of dQ += dS K
+      const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
+      tc_fence_after();
+      float ssum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[64];
+        const uint32_t td = tmem + t_lane + kTmDP + 64 * half;
+        tmem_ld32(td, dp);
+        tmem_ld32(td + 32, dp + 32);
+        tmem_wait_ld();
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(kBarDpFree));     // dP(t + 1) may now be written
+        }
+        if (half == 0 && it > 0) {
+          const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int cc = 64 * half + c;
+          const float ds = x[cc] * (__uint_as_float(dp[c]) - dval);
+          x[cc] = ds;
+          if (DZQ) {
+            if (is_const) {
+              ssum[c & 1] += ds;
+            } else {
+              const int j = j0 + cc;
+              if (rok && j < nkv && !(p.causal && j > i)) {
+                const int delta = j - i;
+                if (delta <= p.E_lo) sat_lo += ds;
+                else if (delta >= p.E_hi) sat_hi += ds;
+                else dzq_row[delta - p.E_lo] = p.tau * ds;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const int cc = 64 * half + 8 * ch;
+          st_shared_v4(op_chunk(dsb, r, 8 * half + ch), DT<T>::pack(x[cc], x[cc + 1]), DT<T>::pack(x[cc + 2], x[cc + 3]),
+                       DT<T>::pack(x[cc + 4], x[cc + 5]), DT<T>::pack(x[cc + 6], x[cc + 7]));
+        }
+      }
+      if (!ok) break;
+      if (DZQ && is_const) {
+        if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
+        else sat_hi += ssum[0] + ssum[1];
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarDsReady));
+    }
+    // -------------------------------------------------------------- epilogue
+    if (DZQ && rok) {
+      // the two saturated offsets of the row, written once
+      if (p.Rexp == 1) {
+        dzq_row[0] = p.tau * (sat_lo + sat_hi);
+      } else {
+        if (gi.e0 == 0) dzq_row[0] = p.tau * sat_lo;
+        if (p.Rexp - 1 < gi.e0 + gi.W) dzq_row[p.Rexp - 1] = p.tau * sat_hi;
+      }
+    }
+    float dq[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) dq[c] = 0.f;
+    const bool got_q = nkt > 0 && ok && mbar_wait(bar(kBarDsFree), (nkt - 1) & 1, abort_flag);
+    if (__all_sync(0xffffffffu, got_q)) {
+      tc_fence_after();
+      uint32_t u[64];
+      tmem_ld32(tmem + t_lane + kTmDQ, u);
+      tmem_ld32(tmem + t_lane + kTmDQ + 32, u + 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; ++c) dq[c] = __uint_as_float(u[c]) * p.tau;
+    }
+    if (rok) {
+      const size_t o = ((size_t)bh * N + i) * 64;
+      if (DQ32) {
+        float* dst = t.dq_acc + o;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dq[c], dq[c + 1], dq[c + 2], dq[c + 3]);
+      } else {
+        T* dst = static_cast<T*>(t.dq) + o;
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          uint4 w;
+          w.x = DT<T>::pack(dq[c], dq[c + 1]);
+          w.y = DT<T>::pack(dq[c + 2], dq[c + 3]);
+          w.z = DT<T>::pack(dq[c + 4], dq[c + 5]);
+          w.w = DT<T>::pack(dq[c + 6], dq[c + 7]);
+          *reinterpret_cast<uint4*>(dst + c) = w;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag && t.status) *t.status = kStatusTimeout;
+}
+
+// ------------------------------------------------------------------ K-parallel
+namespace kp {
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+// a stage: Q tile, dO tile, then LSE log2e, D and the two saturated query
+// columns (tau log2e (Z^Q[i, sat] + b_sat)) of the query tile, 128 floats each
+constexpr uint32_t kVecBytes = 4 * kT * 4;
+constexpr uint32_t kStageBytes = 2 * kTileBytes + 2048;
+constexpr uint32_t kOffK = 0;
+constexpr uint32_t kOffV = kTileBytes;
+constexpr uint32_t kOffQD = 2 * kTileBytes;
+constexpr uint32_t kOffP = kOffQD + kStages * kStageBytes;
+constexpr uint32_t kOffDS = kOffP + 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
+constexpr uint32_t kOffAbort = kOffBar + 256;
+constexpr uint32_t kOffTmem = kOffAbort + 16;
+constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;
+// tensor memory: S^T buffers [0,128), [128,256), dP^T [256,384), dV [384,448), dK [448,512)
+constexpr uint32_t kTmDP = 256, kTmDV = 384, kTmDK = 448;
+constexpr int kBarKV = 0, kBarQsFull = 1, kBarQsEmpty = kBarQsFull + kStages, kBarSFull = kBarQsEmpty + kStages,
+              kBarSFree = kBarSFull + 2, kBarDpFull = kBarSFree + 2, kBarDpFree = kBarDpFull + 1,
+              kBarPReady = kBarDpFree + 1, kBarPFree = kBarPReady + 1, kBarDsReady = kBarPFree + 1,
+              kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
+}  // namespace kp
+
+template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32>
+__global__ void __launch_bounds__(kp::kThreads, 1)
+    dkdv_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmDO) {
+  using namespace kp;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sg = smem_raw + (sb - raw);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + kOffAbort);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sg + kOffTmem);
+  auto bar = [&](int slot) { return sb + kOffBar + 8u * (uint32_t)slot; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
+  const int N = p.N, k0 = kt * kT;
+  const int npad = p.nT * kT;
+  const int nkv = p.padding ? p.key_len[b] : N;
+  const int qt0 = p.causal ? kt : 0;            // queries i >= j only under the causal mask
+  const int nq = k0 < nkv ? p.nT - qt0 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarKV), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarQsFull + s), 1);
+      mbar_init(bar(kBarQsEmpty + s), 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(kBarSFull + u), 1);
+      mbar_init(bar(kBarSFree + u), 128);
+    }
+    mbar_init(bar(kBarDpFull), 1);
+    mbar_init(bar(kBarDpFree), 128);
+    mbar_init(bar(kBarPReady), 128);
+    mbar_init(bar(kBarPFree), 1);
+    mbar_init(bar(kBarDsReady), 128);
+    mbar_init(bar(kBarDsFree), 1);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0 && nq > 0) {
+      // ------------------------------------------------------------ TMA producer
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmDO);
+      mbar_expect_tx(bar(kBarKV), 2 * kTileBytes);
+      tma_load_3d(sb + kOffK, &tmK, bar(kBarKV), 0, k0, bh);
+      tma_load_3d(sb + kOffV, &tmV, bar(kBarKV), 0, k0, bh);
+#pragma unroll 1
+      for (int it = 0; it < nq; ++it) {
+        const int s = it % kStages;
+        if (it >= kStages && !mbar_wait(bar(kBarQsEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+        const int qb = (qt0 + it) * kT;
+        const uint32_t dst = sb + kOffQD + (uint32_t)s * kStageBytes;
+        const uint32_t fb = bar(kBarQsFull + s);
+        mbar_expect_tx(fb, 2 * kTileBytes + ((AQ || BIAS) ? kVecBytes : kVecBytes / 2));
+        tma_load_3d(dst, &tmQ, fb, 0, qb, bh);
+        tma_load_3d(dst + kTileBytes, &tmDO, fb, 0, qb, bh);
+        const size_t vo = (size_t)bh * npad + qb;
+        bulk_load(dst + 2 * kTileBytes, t.lse2 + vo, kT * 4, fb);
+        bulk_load(dst + 2 * kTileBytes + kT * 4, t.dsum + vo, kT * 4, fb);
+        if (AQ || BIAS) {
+          const float* src = t.zq_sat + (size_t)bh * 2 * npad + qb;
+          bulk_load(dst + 2 * kTileBytes + 2 * kT * 4, src, kT * 4, fb);
+          bulk_load(dst + 2 * kTileBytes + 3 * kT * 4, src + npad, kT * 4, fb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nq > 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const bool bf = t.is_bf16 != 0;
+      const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
+      const uint32_t id_g = idesc_f16(bf, 128, 64, false, true);
+      const uint64_t dk = sdesc_sw128(sb + kOffK, 16, 1024);
+      const uint64_t dv = sdesc_sw128(sb + kOffV, 16, 1024);
+      const uint64_t dq0 = sdesc_sw128(sb + kOffQD, 16, 1024);
+      const uint64_t ddo0 = sdesc_sw128(sb + kOffQD + kTileBytes, 16, 1024);
+      const uint64_t dqmn0 = sdesc_sw128(sb + kOffQD, 8192, 1024);
+      const uint64_t ddomn0 = sdesc_sw128(sb + kOffQD + kTileBytes, 8192, 1024);
+      const uint64_t dp_ = sdesc_sw128(sb + kOffP, 16, 1024);
+      const uint64_t dds = sdesc_sw128(sb + kOffDS, 16, 1024);
+      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
+      auto issue_s = [&](int buf, int s) {
+        const uint64_t qd = dq0 + (uint64_t)s * kStage16;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dk + 2 * kk, qd + 2 * kk, id_s, kk > 0);
+      };
+      auto issue_dp = [&](int s) {
+        const uint64_t od = ddo0 + (uint64_t)s * kStage16;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, dv + 2 * kk, od + 2 * kk, id_s, kk > 0);
+      };
+      // D[keys x 64] (+)= A[keys x queries] (shared) * B[queries x 64] (MN-major)
+      auto issue_g = [&](uint32_t d, uint64_t a, uint64_t bmn, bool acc) {
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(d, a + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(kBarKV), 0, abort_flag) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(bar(kBarSFull + 0));
+        issue_dp(0);
+        mma_commit(bar(kBarDpFull));
+        if (nq > 1) {
+          ok = mbar_wait(bar(kBarQsFull + 1), 0, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            issue_s(1, 1);
+            mma_commit(bar(kBarSFull + 1));
+          }
+        }
+      }
+#pragma unroll 1
+      for (int it = 0; it < nq && ok; ++it) {
+        const int s = it % kStages;
+        if (it + 1 < nq) {
+          ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp((it + 1) % kStages);
+          mma_commit(bar(kBarDpFull));
+        }
+        ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_g(tmem + kTmDV, dp_, ddomn0 + (uint64_t)s * kStage16, it > 0);
+        mma_commit(bar(kBarPFree));
+        ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_g(tmem + kTmDK, dds, dqmn0 + (uint64_t)s * kStage16, it > 0);
+        mma_commit(bar(kBarDsFree));
+        mma_commit(bar(kBarQsEmpty + s));
+        if (it + 2 < nq) {
+          const int s2 = (it + 2) % kStages;
+          ok = mbar_wait(bar(kBarQsFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
+               mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it & 1, s2);
+          mma_commit(bar(kBarSFull + (it & 1)));
+        }
+      }
+      if (!ok) {
+        mma_commit(bar(kBarDrain));
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- compute
+    const int r = (warp - 4) * 32 + lane;        // key of the tile = tensor-memory lane
+    const int j = k0 + r;
+    const bool jok = j < N;
+    const bool jkeep = j < nkv;                  // keys past key_len are masked for every query
+    const uint32_t t_lane = (uint32_t)((warp & 3) * 32) << 16;
+    const float sc = p.tau * kLog2e;
+    // saturated-offset row constants tau log2e Z^K[j, sat] (zero past N)
+    const float rowk_lo = AK ? t.zk_sat[(size_t)bh * 2 * npad + k0 + r] : 0.f;
+    const float rowk_hi = AK ? t.zk_sat[(size_t)bh * 2 * npad + npad + k0 + r] : 0.f;
+    const float* zk_row = nullptr;
+    float* dzk_row = nullptr;
+    GroupInfo gk{};
+    if (jok) {
+      gk = p.gk[kt];
+      const long long ro = gk.base + (long long)r * gk.S - gk.e0;
+      if (AK) zk_row = t.zk + (size_t)bh * p.zk_head + ro;
+      if (DZK) dzk_row = t.dzk + (size_t)bh * p.zk_head + ro;
+    }
+    const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
+    const uint32_t pb = sb + kOffP, dsb = sb + kOffDS;
+    float sat_lo = 0.f, sat_hi = 0.f;
+    bool ok = true;
+#pragma unroll 1
+    for (int it = 0; it < nq; ++it) {
+      const int qi = qt0 + it, qb = qi * kT;
+      const int cls = tile_class(qi, kt, N, nkv, p.causal, p.E_lo, p.E_hi);
+      const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
+      const int stage = it % kStages, buf = it & 1;
+      const float* vec = reinterpret_cast<const float*>(sg + kOffQD + (uint32_t)stage * kStageBytes + 2 * kTileBytes);
+      const float* lse2v = vec;
+      const float* dvec = vec + kT;
+      const float* cvq = vec + (cls == RELPOS_TILE_CONST_LO ? 2 * kT : 3 * kT);
+      // the stage's own barrier makes its TMA-written vectors visible to these threads
+      const bool got_s = mbar_wait(bar(kBarSFull + buf), (it >> 1) & 1, abort_flag) &&
+                         mbar_wait(bar(kBarQsFull + stage), (it / kStages) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
+      tc_fence_after();
+      float x[128];
+      {
+        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128;
+        tmem_ld32(ts + 0, reinterpret_cast<uint32_t*>(x) + 0);
+        tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
+        tmem_ld32(ts + 64, reinterpret_cast<uint32_t*>(x) + 64);
+        tmem_ld32(ts + 96, reinterpret_cast<uint32_t*>(x) + 96);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + buf));
+      // P^T = 2^(S^T tau log2e + relation terms - LSE_i log2e), column c = query qb + c
+      if (is_const) {
+        const float rowk = cls == RELPOS_TILE_CONST_LO ? rowk_lo : rowk_hi;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
+          float4 w4 = make_float4(-l4.x, -l4.y, -l4.z, -l4.w);
+          if (AQ || BIAS) {
+            const float4 c4 = *reinterpret_cast<const float4*>(cvq + c);
+            w4.x += c4.x; w4.y += c4.y; w4.z += c4.z; w4.w += c4.w;
+          }
+          x[c] = fast_exp2(fmaf(x[c], sc, w4.x) + rowk);
+          x[c + 1] = fast_exp2(fmaf(x[c + 1], sc, w4.y) + rowk);
+          x[c + 2] = fast_exp2(fmaf(x[c + 2], sc, w4.z) + rowk);
+          x[c + 3] = fast_exp2(fmaf(x[c + 3], sc, w4.w) + rowk);
+        }
+      } else {
+        const float* zq_tile = nullptr;
+        int zS = 0;
+        if (AQ) {
+          const GroupInfo gq = p.gq[qi];
+          zq_tile = t.zq + (size_t)bh * p.zq_head + gq.base - gq.e0;
+          zS = gq.S;
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+#pragma unroll
+          for (int c = c0; c < c0 + 32; ++c) {
+            float rel = 0.f;
+            const int i = qb + c;
+            if (jkeep && i < N && !(p.causal && j > i)) {
+              const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
+              if (AQ) rel += __ldg(zq_tile + (long long)c * zS + e);
+              if (AK) rel += __ldg(zk_row + e);
+              if (BIAS) rel += __ldg(bexp + e);
+            }
+            x[c] = (x[c] + rel) * sc;
+          }
+          asm volatile("" ::: "memory");
+        }
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
+          x[c] = fast_exp2(x[c] - l4.x);
+          x[c + 1] = fast_exp2(x[c + 1] - l4.y);
+          x[c + 2] = fast_exp2(x[c + 2] - l4.z);
+          x[c + 3] = fast_exp2(x[c + 3] - l4.w);
+        }
+      }
+      const bool need_mask = !jkeep || (p.causal && k0 + kT - 1 > qb);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          if (!jkeep || (p.causal && j > qb + c)) x[c] = 0.f;
+        }
+      }
+      // P^T to shared memory: the A operand of dV += P^T dO
+      if (it > 0) {
+        const bool got = mbar_wait(bar(kBarPFree), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const int cc = 8 * ch;
+        st_shared_v4(op_chunk(pb, r, ch), DT<T>::pack(x[cc], x[cc + 1]), DT<T>::pack(x[cc + 2], x[cc + 3]),
+                     DT<T>::pack(x[cc + 4], x[cc + 5]), DT<T>::pack(x[cc + 6], x[cc + 7]));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarPReady));
+      // dS^T = P^T (dP^T - D_i) in two halves of 64 queries: the A operand of
+      // dK += dS^T Q, and the key-side relation gradient of this key row
+      const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
+      tc_fence_after();
+      float ssum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[64];
+        const uint32_t td = tmem + t_lane + kTmDP + 64 * half;
+        tmem_ld32(td, dp);
+        tmem_ld32(td + 32, dp + 32);
+        tmem_wait_ld();
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(kBarDpFree));
+        }
+        if (half == 0 && it > 0) {
+          const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const int cc0 = 64 * half + c;
+          const float4 d4 = *reinterpret_cast<const float4*>(dvec + cc0);
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int cc = cc0 + u;
+            const float ds = x[cc] * (__uint_as_float(dp[c + u]) - dd[u]);
+            x[cc] = ds;
+            if (DZK) {
+              if (is_const) {
+                ssum[u & 1] += ds;
+              } else {
+                const int i = qb + cc;
+                if (jkeep && i < N && !(p.causal && j > i)) {
+                  const int delta = j - i;
+                  if (delta <= p.E_lo) sat_lo += ds;
+                  else if (delta >= p.E_hi) sat_hi += ds;
+                  else dzk_row[delta - p.E_lo] = p.tau * ds;
+                }
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const int cc = 64 * half + 8 * ch;
+          st_shared_v4(op_chunk(dsb, r, 8 * half + ch), DT<T>::pack(x[cc], x[cc + 1]), DT<T>::pack(x[cc + 2], x[cc + 3]),
+                       DT<T>::pack(x[cc + 4], x[cc + 5]), DT<T>::pack(x[cc + 6], x[cc + 7]));
+        }
+      }
+      if (!ok) break;
+      if (DZK && is_const) {
+        if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
+        else sat_hi += ssum[0] + ssum[1];
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarDsReady));
+    }
+    // -------------------------------------------------------------- epilogue
+    if (DZK && jok) {
+      if (p.Rexp == 1) {
+        dzk_row[0] = p.tau * (sat_lo + sat_hi);
+      } else {
+        if (gk.e0 == 0) dzk_row[0] = p.tau * sat_lo;
+        if (p.Rexp - 1 < gk.e0 + gk.W) dzk_row[p.Rexp - 1] = p.tau * sat_hi;
+      }
+    }
+    float dv[64], dk[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) dv[c] = dk[c] = 0.f;
+    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDsFree), (nq - 1) & 1, abort_flag);
+    if (__all_sync(0xffffffffu, got_o)) {
+      tc_fence_after();
+      uint32_t u[64];
+      tmem_ld32(tmem + t_lane + kTmDV, u);
+      tmem_ld32(tmem + t_lane + kTmDV + 32, u + 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; ++c) dv[c] = __uint_as_float(u[c]);
+      tmem_ld32(tmem + t_lane + kTmDK, u);
+      tmem_ld32(tmem + t_lane + kTmDK + 32, u + 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; ++c) dk[c] = __uint_as_float(u[c]) * p.tau;
+    }
+    if (jok) {
+      const size_t o = ((size_t)bh * N + j) * 64;
+      T* vdst = static_cast<T*>(t.dv) + o;
+#pragma unroll
+      for (int c = 0; c < 64; c += 8) {
+        uint4 w;
+        w.x = DT<T>::pack(dv[c], dv[c + 1]);
+        w.y = DT<T>::pack(dv[c + 2], dv[c + 3]);
+        w.z = DT<T>::pack(dv[c + 4], dv[c + 5]);
+        w.w = DT<T>::pack(dv[c + 6], dv[c + 7]);
+        *reinterpret_cast<uint4*>(vdst + c) = w;
+      }
+      if (DK32) {
+        float* dst = t.dk_acc + o;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dk[c], dk[c + 1], dk[c + 2], dk[c + 3]);
+      } else {
+        T* dst = static_cast<T*>(t.dk) + o;
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          uint4 w;
+          w.x = DT<T>::pack(dk[c], dk[c + 1]);
+          w.y = DT<T>::pack(dk[c + 2], dk[c + 3]);
+          w.z = DT<T>::pack(dk[c + 4], dk[c + 5]);
+          w.w = DT<T>::pack(dk[c + 6], dk[c + 7]);
+          *reinterpret_cast<uint4*>(dst + c) = w;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag && t.status) *t.status = kStatusTimeout;
+}
+
+// ---------------------------------------------------------------- host side
+template <typename K>
+cudaError_t launch4(K kern, dim3 grid, int threads, uint32_t smem, const Plan& p, const Tensors& t,
+                    const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, const CUtensorMap& d,
+                    cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  { kern<<<grid, threads, smem, s>>>(p, t, a, b, c, d); note_launch(1); }
+  return cudaGetLastError();
+}
+
+struct Maps {
+  CUtensorMap q, k, v, dout;
+};
+
+bool make_maps(const Plan& p, const Tensors& t, Maps& m) {
+  const int BH = p.B * p.H;
+  const bool bf = t.is_bf16 != 0;
+  return make_rows_map(&m.q, t.q, BH, p.N, bf) && make_rows_map(&m.k, t.k, BH, p.N, bf) &&
+         make_rows_map(&m.v, t.v, BH, p.N, bf) && make_rows_map(&m.dout, t.dout, BH, p.N, bf);
+}
+
+template <typename T>
+cudaError_t dq_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
+  Maps m;
+  if (!make_maps(p, t, m)) return cudaErrorInvalidValue;
+  const bool aq = t.aq_exp, ak = t.ak_exp, bb = t.b_exp;
+  const dim3 grid(p.nT, p.B * p.H);
+#define RP_DQ(A, K_, B_)                                                                                       \
+  if (aq == A && ak == K_ && bb == B_)                                                                         \
+    return launch4(dq_sm100_kernel<T, A, K_, B_, (A || B_), A>, grid, qp::kThreads, qp::kSmemBytes, p, t, m.q, \
+                   m.k, m.v, m.dout, s);
+  RP_DQ(false, false, false) RP_DQ(true, false, false) RP_DQ(false, true, false) RP_DQ(true, true, false)
+  RP_DQ(false, false, true) RP_DQ(true, false, true) RP_DQ(false, true, true) RP_DQ(true, true, true)
+#undef RP_DQ
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t dk_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
+  Maps m;
+  if (!make_maps(p, t, m)) return cudaErrorInvalidValue;
+  const bool aq = t.aq_exp, ak = t.ak_exp, bb = t.b_exp;
+  const dim3 grid(p.nT, p.B * p.H);
+#define RP_DK(A, K_, B_)                                                                                         \
+  if (aq == A && ak == K_ && bb == B_)                                                                           \
+    return launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_>, grid, kp::kThreads, kp::kSmemBytes, p, t, m.q, m.k, \
+                   m.v, m.dout, s);
+  RP_DK(false, false, false) RP_DK(true, false, false) RP_DK(false, true, false) RP_DK(true, true, false)
+  RP_DK(false, false, true) RP_DK(true, false, true) RP_DK(false, true, true) RP_DK(true, true, true)
+#undef RP_DK
+  return cudaErrorInvalidValue;
+}
+
+inline unsigned nblocks(long long n, int t) { return (unsigned)((n + t - 1) / t); }
+
+}  // namespace
+
+cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s) {
+  const long long BH = (long long)p.B * p.H;
+  const int npad = p.nT * kT;
+  const unsigned blocks = nblocks(BH * npad * 8, 256);
+  if (t.is_bf16) {
+    if (t.o_f32) {
+      prep_sm100_kernel<float, __nv_bfloat16><<<blocks, 256, 0, s>>>((const float*)t.o, (const __nv_bfloat16*)t.dout,
+                                                                      t.lse, t.dsum, t.lse2, p.N, npad, BH);
+    } else {
+      prep_sm100_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(
+          (const __nv_bfloat16*)t.o, (const __nv_bfloat16*)t.dout, t.lse, t.dsum, t.lse2, p.N, npad, BH);
+    }
+  } else {
+    if (t.o_f32) {
+      prep_sm100_kernel<float, __half><<<blocks, 256, 0, s>>>((const float*)t.o, (const __half*)t.dout, t.lse,
+                                                               t.dsum, t.lse2, p.N, npad, BH);
+    } else {
+      prep_sm100_kernel<__half, __half><<<blocks, 256, 0, s>>>((const __half*)t.o, (const __half*)t.dout, t.lse,
+                                                                t.dsum, t.lse2, p.N, npad, BH);
+    }
+  }
+  note_launch(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s) {
+  return t.is_bf16 ? dq_typed<__nv_bfloat16>(p, t, s) : dq_typed<__half>(p, t, s);
+}
+
+cudaError_t launch_bwd_dkdv(const Plan& p, const Tensors& t, cudaStream_t s) {
+  return t.is_bf16 ? dk_typed<__nv_bfloat16>(p, t, s) : dk_typed<__half>(p, t, s);
+}
+
+}  // namespace relpos

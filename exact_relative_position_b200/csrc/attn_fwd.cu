@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
       tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
       tma_load_3d(sb + kOffQ + kTileBytes, &tmQ, bar(kBarQ), 0, q0 + kBQ, bh);
+#pragma unroll 1
       for (int it = 0; it < nkt; ++it) {
         const int s = it % kStages;
         if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
@@ -193,14 +194,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t a = dq0 + (uint64_t)g * kTile16;
         const uint64_t k = dk0 + (uint64_t)s * kStage16;
         const uint32_t d = tmem + (uint32_t)g * 128;
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < 4; ++kk) mma_ss(d, a + 2 * kk, k + 2 * kk, id_qk, kk > 0);
       };
       auto issue_pv = [&](int g, int s, bool acc) {
         const uint64_t v = dv0 + (uint64_t)s * kStage16;
         const uint64_t pp = dp0 + (uint64_t)g * kP16;
         const uint32_t d = tmem + 256 + (uint32_t)g * 64;
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(d, pp + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), v + 128 * kk, id_pv, (acc || kk > 0) ? 1u : 0u);
       };
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar(kBarSFull + 0));
         issue_qk(1, 0);
         mma_commit(bar(kBarSFull + 1));
+#pragma unroll 1
         for (int it = 0; it < nkt && ok; ++it) {
           const int s = it % kStages;
           if (it + 1 < nkt) {
@@ -291,17 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                          (!AK || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(tS + 0, sr + 0);
-      tmem_ld32(tS + 32, sr + 32);
-      tmem_ld32(tS + 64, sr + 64);
-      tmem_ld32(tS + 96, sr + 96);
+      float x[128];
+      tmem_ld32(tS + 0, reinterpret_cast<uint32_t*>(x) + 0);
+      tmem_ld32(tS + 32, reinterpret_cast<uint32_t*>(x) + 32);
+      tmem_ld32(tS + 64, reinterpret_cast<uint32_t*>(x) + 64);
+      tmem_ld32(tS + 96, reinterpret_cast<uint32_t*>(x) + 96);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(kBarSFree + g));    // the next key tile's S_g may now be written
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
       // x holds the scaled score (without the row constant rowc) in base 2;
       // for a saturated tile without key-side terms the scale is applied in
       // the exponent instead (xs = sc) to save one pass
@@ -328,18 +327,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           zk_tile = t.zk + (size_t)bh * p.zk_head + gk.base - gk.e0;
           zS = gk.S;
         }
+        // in chunks of 32 columns: the compiler may not hoist the gathers of
+        // later chunks, which keeps the live registers bounded
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float rel = 0.f;
-          const int j = j0 + c;
-          // only kept cells: a masked cell's offset may lie outside the stored columns
-          if (rok && j < nkv && !(p.causal && j > i)) {
-            const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
-            if (AQ) rel += __ldg(zq_row + e);
-            if (AK) rel += __ldg(zk_tile + (long long)c * zS + e);
-            if (BIAS) rel += __ldg(bexp + e);
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+#pragma unroll
+          for (int c = c0; c < c0 + 32; ++c) {
+            float rel = 0.f;
+            const int j = j0 + c;
+            // only kept cells: a masked cell's offset may lie outside the stored columns
+            if (rok && j < nkv && !(p.causal && j > i)) {
+              const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
+              if (AQ) rel += __ldg(zq_row + e);
+              if (AK) rel += __ldg(zk_tile + (long long)c * zS + e);
+              if (BIAS) rel += __ldg(bexp + e);
+            }
+            x[c] = (x[c] + rel) * sc;
           }
-          x[c] = (x[c] + rel) * sc;
+          asm volatile("" ::: "memory");
         }
       }
       const bool need_mask = (j0 + kBK > nkv) || (p.causal && j0 + kBK - 1 > q0 + g * kBQ);
@@ -387,31 +392,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run *= alpha;
         m_run = m_new;
       }
-      // p = 2^(x * xs + rowc - m_run)
-      const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = fast_exp2(fmaf(x[c], xs, -msub));
-      uint32_t pk[64];
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        pk[c] = DT<T>::pack(x[2 * c], x[2 * c + 1]);
-        // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
-        // enough to sum the fp32 values and spare the conversions
-        ps[c & 7] += DT<T>::kCoarse ? DT<T>::pair_sum(pk[c]) : x[2 * c] + x[2 * c + 1];
-      }
-      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       // P_g of the previous key tile must have been consumed by its PV GEMM
       if (!pfree_seen) {
         const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
-      // row r of P: 16 chunks of 16 bytes in two 64-key swizzle atoms
+      // p = 2^(x * xs + rowc - m_run), streamed 8 keys at a time into row r of
+      // P (16-byte chunks of two 64-key swizzle atoms)
+      const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
+        float e8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) e8[u] = fast_exp2(fmaf(x[8 * c + u], xs, -msub));
+        uint32_t pk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          pk[u] = DT<T>::pack(e8[2 * u], e8[2 * u + 1]);
+          // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
+          // enough to sum the fp32 values and spare the conversions
+          ps[u] += DT<T>::kCoarse ? DT<T>::pair_sum(pk[u]) : e8[2 * u] + e8[2 * u + 1];
+        }
         const uint32_t addr = pbase + (uint32_t)(c >> 3) * kTileBytes + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-        st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        st_shared_v4(addr, pk[0], pk[1], pk[2], pk[3]);
       }
+      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarPReady + g));
     }
@@ -445,6 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag && t.status) *t.status = kStatusTimeout;
 }
 
+}  // namespace
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -473,6 +481,8 @@ bool make_rows_map(CUtensorMap* m, const void* base, int BH, int N, bool bf16) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <typename T, typename OutT>
 cudaError_t launch_typed(const Plan& p, const Tensors& t, cudaStream_t s) {

@@ -2,6 +2,8 @@
 // unit per kernel family) and the parameter blocks they take.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace relpos {
@@ -20,7 +22,9 @@ struct Tensors {
   float* lse;
   // backward
   const void* dout;
-  float* dsum;                   // D_i = sum_c dO_ic O_ic, [B,H,N]
+  float* dsum;                   // D_i = sum_c dO_ic O_ic, [B*H][nT*128] (0 past N)
+  float* lse2;                   // LSE_i log2 e, [B*H][nT*128] (+inf past N and for rows with every key masked)
+  float* zq_sat;                 // [B*H][2][nT*128]: tau log2e (Z^Q[i, sat] + b_sat) for sat = 0, R_exp-1
   float *dzq, *dzk;              // offset-sharded relation gradients (same layout as zq/zk)
   void *dq, *dk, *dv;
   float *dq_acc, *dk_acc;        // fp32 [B,H,N,64] before the relation-GEMM epilogue (or null)
@@ -50,6 +54,11 @@ cudaError_t launch_build_tables(const Plan& p, const relpos_map_desc& map, Group
 cudaError_t launch_fold_ranges(const Plan& p, const int* phi_exp, int R, int* fold_lo, int* fold_hi, cudaStream_t s);
 cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t s);
+
+// [BH, N, 64] 16-bit tensor viewed as 3-D for TMA: 128-row boxes, 128-byte
+// swizzle, rows past N read as zero.
+bool make_rows_map(CUtensorMap* m, const void* base, int BH, int N, bool bf16);
 cudaError_t launch_forward(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s);

@@ -130,6 +130,34 @@ __global__ void saturated_columns_kernel(const Plan p, const float* __restrict__
   out[(bh * 2 + 1) * npad + j] = hi;
 }
 
+// out[bh][0][i] = tau log2e (Z^Q[i, 0] + b_exp[0]), out[bh][1][i] = the same at
+// R_exp - 1 (each term only when present; zero for i >= N): the row constants
+// of saturated tiles for the backward passes.
+__global__ void saturated_rows_kernel(const Plan p, const float* __restrict__ zq, const float* __restrict__ b_exp,
+                                      float* __restrict__ out, const float scale) {
+  const int npad = p.nT * kTile;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)p.B * p.H * npad) return;
+  const int i = (int)(idx % npad);
+  const long long bh = idx / npad;
+  const int h = (int)(bh % p.H);
+  float lo = 0.f, hi = 0.f;
+  if (i < p.N) {
+    if (zq) {
+      const GroupInfo gi = p.gq[i / kTile];
+      const float* row = zq + bh * p.zq_head + gi.base + (long long)(i % kTile) * gi.S - gi.e0;
+      if (gi.e0 == 0) lo += row[0];
+      if (gi.e0 + gi.W >= p.Rexp) hi += row[p.Rexp - 1];
+    }
+    if (b_exp) {
+      lo += b_exp[(size_t)h * p.Rexp];
+      hi += b_exp[(size_t)h * p.Rexp + p.Rexp - 1];
+    }
+  }
+  out[(bh * 2 + 0) * npad + i] = lo * scale;
+  out[(bh * 2 + 1) * npad + i] = hi * scale;
+}
+
 // ------------------------------------------------------------------ relgrad rows
 // out[rows of group g] = acc_in[rows] + dZ_g[rows, :W] A_exp[e0 .. e0 + W)   (tf32 tensor cores)
 constexpr int kRowPitchA = 36;   // floats, dZ chunk [128][32]
@@ -381,6 +409,16 @@ static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_
 cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream_t s) {
   const long long n = (long long)p.B * p.H * p.nT * kTile;
   { saturated_columns_kernel<<<nblk(n, 256), 256, 0, s>>>(p, t.zk, t.zk_sat, p.tau * kLog2e); note_launch(1); }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t s) {
+  const long long n = (long long)p.B * p.H * p.nT * kTile;
+  {
+    saturated_rows_kernel<<<nblk(n, 256), 256, 0, s>>>(p, t.aq_exp ? t.zq : nullptr, t.b_exp, t.zq_sat,
+                                                       p.tau * kLog2e);
+    note_launch(1);
+  }
   return cudaGetLastError();
 }
 
