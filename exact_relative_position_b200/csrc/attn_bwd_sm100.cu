@@ -23,6 +23,7 @@
 // wait is bounded (see sm100.cuh).
 #include <cudaTypedefs.h>
 
+#include "band.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 #include "warp_mma.cuh"
@@ -105,32 +106,6 @@ constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kStages, kBa
               kBarSFree = kBarSFull + 2, kBarDpFull = kBarSFree + 2, kBarDpFree = kBarDpFull + 1,
               kBarDsReady = kBarDpFree + 1, kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
 }  // namespace qp
-
-// Relation terms (scaled by tau log2 e) of one row of a BAND tile, added in
-// place to the 128 raw scores x[] (kept cells only: a masked cell's offset may
-// lie outside the stored projection columns).  In chunks of 32 columns so the
-// compiler cannot hoist all gathers at once and keeps registers bounded.
-template <bool AQ, bool AK, bool BIAS>
-__device__ __forceinline__ void band_terms(float (&x)[128], const Plan& p, int i, int j0, int nkv, bool rok,
-                                           const float* zq_row, const float* zk_tile, int zS, const float* bexp,
-                                           float sc) {
-#pragma unroll
-  for (int c0 = 0; c0 < 128; c0 += 32) {
-#pragma unroll
-    for (int c = c0; c < c0 + 32; ++c) {
-      float rel = 0.f;
-      const int j = j0 + c;
-      if (rok && j < nkv && !(p.causal && j > i)) {
-        const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
-        if (AQ) rel += __ldg(zq_row + e);
-        if (AK) rel += __ldg(zk_tile + (long long)c * zS + e);
-        if (BIAS) rel += __ldg(bexp + e);
-      }
-      x[c] = (x[c] + rel) * sc;
-    }
-    asm volatile("" ::: "memory");
-  }
-}
 
 template <typename T, bool AQ, bool AK, bool BIAS, bool DZQ, bool DQ32>
 __global__ void __launch_bounds__(qp::kThreads, 1)
@@ -301,15 +276,13 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     // saturated-offset row constants tau log2e (Z^Q[i, sat] + b_sat), zero past N
     const float crow_lo = (AQ || BIAS) ? t.zq_sat[(size_t)bh * 2 * npad + q0 + r] : 0.f;
     const float crow_hi = (AQ || BIAS) ? t.zq_sat[(size_t)bh * 2 * npad + npad + q0 + r] : 0.f;
-    const float* zq_row = nullptr;
-    float* dzq_row = nullptr;
-    GroupInfo gi{};
-    if (rok) {
-      gi = p.gq[qt];
-      const long long ro = gi.base + (long long)(i - q0) * gi.S - gi.e0;
-      if (AQ) zq_row = t.zq + (size_t)bh * p.zq_head + ro;
-      if (DZQ) dzq_row = t.dzq + (size_t)bh * p.zq_head + ro;
-    }
+    // projection group of this query tile; rows past N use row 0 (in bounds)
+    const GroupInfo gi = p.gq[qt];
+    const int rrow = rok ? r : 0;
+    const float* zq_row = AQ ? t.zq + (size_t)bh * p.zq_head + gi.base + (long long)rrow * gi.S - gi.e0 : nullptr;
+    float* dzq_base = DZQ ? t.dzq + (size_t)bh * p.zq_head + gi.base : nullptr;
+    float* dzq_row = DZQ ? dzq_base + (long long)rrow * gi.S - gi.e0 : nullptr;
+    const int nrows_q = imin(kT, N - q0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
     const uint32_t dsb = sb + kOffDS;
     float sat_lo = 0.f, sat_hi = 0.f;
@@ -355,13 +328,16 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         }
       } else {
         const float* zk_tile = nullptr;
-        int zS = 0;
+        int zS = 0, ek0 = 0, ek1 = 0;
         if (AK) {
           const GroupInfo gk = p.gk[it];
           zk_tile = t.zk + (size_t)bh * p.zk_head + gk.base - gk.e0;
           zS = gk.S;
+          ek0 = gk.e0;
+          ek1 = gk.e0 + gk.W - 1;
         }
-        band_terms<AQ, AK, BIAS>(x, p, i, j0, nkv, rok, zq_row, zk_tile, zS, bexp, sc);
+        band_terms_q<AQ, AK, BIAS>(x, p.E_lo, p.E_hi, i, j0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
+                                   imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
 #pragma unroll
         for (int c = 0; c < 128; ++c) x[c] = fast_exp2(x[c] - lse2);
       }
@@ -395,22 +371,28 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int cc = 64 * half + c;
-          const float ds = x[cc] * (__uint_as_float(dp[c]) - dval);
-          x[cc] = ds;
-          if (DZQ) {
-            if (is_const) {
-              ssum[c & 1] += ds;
-            } else {
-              const int j = j0 + cc;
-              if (rok && j < nkv && !(p.causal && j > i)) {
-                const int delta = j - i;
-                if (delta <= p.E_lo) sat_lo += ds;
-                else if (delta >= p.E_hi) sat_hi += ds;
-                else dzq_row[delta - p.E_lo] = p.tau * ds;
-              }
-            }
+        if (!DZQ || is_const) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int cc = 64 * half + c;
+            const float ds = x[cc] * (__uint_as_float(dp[c]) - dval);
+            x[cc] = ds;
+            if (DZQ) ssum[c & 1] += ds;
+          }
+        } else {
+          // saturated cells summed here; the interior ones are stored below.
+          // Kept columns are c <= ckeep; low-saturated c <= clo, high c >= chi.
+          int ckeep = rok ? imin(nkv - 1 - j0, 127) : -1;
+          if (p.causal) ckeep = imin(ckeep, i - j0);
+          const int clo = imin(p.E_lo + i - j0, ckeep);
+          const int chi = imax(p.E_hi + i - j0, p.E_lo + i - j0 + 1);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int cc = 64 * half + c;
+            const float ds = x[cc] * (__uint_as_float(dp[c]) - dval);
+            x[cc] = ds;
+            sat_lo += cc <= clo ? ds : 0.f;
+            sat_hi += (cc >= chi && cc <= ckeep) ? ds : 0.f;
           }
         }
 #pragma unroll
@@ -424,6 +406,11 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       if (DZQ && is_const) {
         if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
         else sat_hi += ssum[0] + ssum[1];
+      }
+      if (DZQ && !is_const) {
+        __syncwarp();
+        dz_band_store<T>(dsb, (warp - 4) * 32, lane, false, q0, j0, nrows_q, nkv, N, p.causal, p.E_lo, p.E_hi,
+                         dzq_base, gi.S, gi.e0, p.tau);
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarDsReady));
@@ -682,15 +669,13 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     // saturated-offset row constants tau log2e Z^K[j, sat] (zero past N)
     const float rowk_lo = AK ? t.zk_sat[(size_t)bh * 2 * npad + k0 + r] : 0.f;
     const float rowk_hi = AK ? t.zk_sat[(size_t)bh * 2 * npad + npad + k0 + r] : 0.f;
-    const float* zk_row = nullptr;
-    float* dzk_row = nullptr;
-    GroupInfo gk{};
-    if (jok) {
-      gk = p.gk[kt];
-      const long long ro = gk.base + (long long)r * gk.S - gk.e0;
-      if (AK) zk_row = t.zk + (size_t)bh * p.zk_head + ro;
-      if (DZK) dzk_row = t.dzk + (size_t)bh * p.zk_head + ro;
-    }
+    // projection group of this key tile; keys past N use row 0 (in bounds)
+    const GroupInfo gk = p.gk[kt];
+    const int krow = jok ? r : 0;
+    const float* zk_row = AK ? t.zk + (size_t)bh * p.zk_head + gk.base + (long long)krow * gk.S - gk.e0 : nullptr;
+    float* dzk_base = DZK ? t.dzk + (size_t)bh * p.zk_head + gk.base : nullptr;
+    float* dzk_row = DZK ? dzk_base + (long long)krow * gk.S - gk.e0 : nullptr;
+    const int nrows_k = imin(kT, N - k0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
     const uint32_t pb = sb + kOffP, dsb = sb + kOffDS;
     float sat_lo = 0.f, sat_hi = 0.f;
@@ -739,28 +724,16 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         }
       } else {
         const float* zq_tile = nullptr;
-        int zS = 0;
+        int zS = 0, eq0 = 0, eq1 = 0;
         if (AQ) {
           const GroupInfo gq = p.gq[qi];
           zq_tile = t.zq + (size_t)bh * p.zq_head + gq.base - gq.e0;
           zS = gq.S;
+          eq0 = gq.e0;
+          eq1 = gq.e0 + gq.W - 1;
         }
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-#pragma unroll
-          for (int c = c0; c < c0 + 32; ++c) {
-            float rel = 0.f;
-            const int i = qb + c;
-            if (jkeep && i < N && !(p.causal && j > i)) {
-              const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
-              if (AQ) rel += __ldg(zq_tile + (long long)c * zS + e);
-              if (AK) rel += __ldg(zk_row + e);
-              if (BIAS) rel += __ldg(bexp + e);
-            }
-            x[c] = (x[c] + rel) * sc;
-          }
-          asm volatile("" ::: "memory");
-        }
+        band_terms_k<AQ, AK, BIAS>(x, p.E_lo, p.E_hi, j, qb, zk_row, gk.e0, gk.e0 + gk.W - 1, zq_tile, zS,
+                                   imin(kT, N - qb) - 1, eq0, eq1, bexp, sc);
 #pragma unroll
         for (int c = 0; c < 128; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
@@ -796,6 +769,13 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
       tc_fence_after();
       float ssum[2] = {0.f, 0.f};
+      // column ranges of this key row (column cc = query qb + cc): kept for
+      // ckeep_lo <= cc <= ckeep_hi; low-saturated (j - i <= E_lo) for cc >= clo;
+      // high-saturated (j - i >= E_hi, not low) for cc <= chi
+      const int ckeep_lo = p.causal ? imax(j - qb, 0) : 0;
+      const int ckeep_hi = jkeep ? imin(N - 1 - qb, 127) : -1;
+      const int clo = j - qb - p.E_lo;
+      const int chi = imin(j - qb - p.E_hi, clo - 1);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t dp[64];
@@ -811,28 +791,36 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
+        if (!DZK || is_const) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const int cc0 = 64 * half + c;
-          const float4 d4 = *reinterpret_cast<const float4*>(dvec + cc0);
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+          for (int c = 0; c < 64; c += 4) {
+            const int cc0 = 64 * half + c;
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + cc0);
+            const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int cc = cc0 + u;
-            const float ds = x[cc] * (__uint_as_float(dp[c + u]) - dd[u]);
-            x[cc] = ds;
-            if (DZK) {
-              if (is_const) {
-                ssum[u & 1] += ds;
-              } else {
-                const int i = qb + cc;
-                if (jkeep && i < N && !(p.causal && j > i)) {
-                  const int delta = j - i;
-                  if (delta <= p.E_lo) sat_lo += ds;
-                  else if (delta >= p.E_hi) sat_hi += ds;
-                  else dzk_row[delta - p.E_lo] = p.tau * ds;
-                }
-              }
+            for (int u = 0; u < 4; ++u) {
+              const int cc = cc0 + u;
+              const float ds = x[cc] * (__uint_as_float(dp[c + u]) - dd[u]);
+              x[cc] = ds;
+              if (DZK) ssum[u & 1] += ds;
+            }
+          }
+        } else {
+          // kept columns are ckeep_lo <= cc <= ckeep_hi; delta = j - qb - cc is
+          // low-saturated for cc >= clo and high-saturated for cc <= chi
+          const int lo_beg = imax(clo, ckeep_lo), hi_end = imin(chi, ckeep_hi);
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const int cc0 = 64 * half + c;
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + cc0);
+            const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int cc = cc0 + u;
+              const float ds = x[cc] * (__uint_as_float(dp[c + u]) - dd[u]);
+              x[cc] = ds;
+              sat_lo += (cc >= lo_beg && cc <= ckeep_hi) ? ds : 0.f;
+              sat_hi += (cc <= hi_end && cc >= ckeep_lo) ? ds : 0.f;
             }
           }
         }
@@ -847,6 +835,11 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       if (DZK && is_const) {
         if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
         else sat_hi += ssum[0] + ssum[1];
+      }
+      if (DZK && !is_const) {
+        __syncwarp();
+        dz_band_store<T>(dsb, (warp - 4) * 32, lane, true, k0, qb, nrows_k, nkv, N, p.causal, p.E_lo, p.E_hi,
+                         dzk_base, gk.S, gk.e0, p.tau);
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarDsReady));

@@ -28,6 +28,7 @@
 // factor 256), which keeps every P <= 256 and the result exact.
 #include <cudaTypedefs.h>
 
+#include "band.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 #include "warp_mma.cuh"
@@ -258,14 +259,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + t_lane + 256 + (uint32_t)g * 64;
     const uint32_t pbase = sb + kOffP + (uint32_t)g * kPBytes + (uint32_t)r * 128;
     const float sc = p.tau * kLog2e;
-    const float* zq_row = nullptr;
+    // projection group of this query tile (the last one for a tile past N,
+    // whose rows are all discarded); rows past N read row 0 (in bounds)
+    const GroupInfo gi = p.gq[imin(qtile, p.nT - 1)];
+    const int rrow = rok ? i - qtile * kBQ : 0;
+    const float* zq_row = AQ ? t.zq + (size_t)bh * p.zq_head + gi.base + (long long)rrow * gi.S - gi.e0 : nullptr;
     float crow_lo = 0.f, crow_hi = 0.f;
     if (rok) {
       // saturated columns e = 0 / R_exp - 1 (present in the row's group whenever a
       // CONST tile can occur for it)
-      const GroupInfo gi = p.gq[qtile];
       if (AQ) {
-        zq_row = t.zq + (size_t)bh * p.zq_head + gi.base + (long long)(i - qtile * kBQ) * gi.S - gi.e0;
         if (gi.e0 == 0) crow_lo += __ldg(zq_row);
         if (gi.e0 + gi.W >= p.Rexp) crow_hi += __ldg(zq_row + p.Rexp - 1);
       }
@@ -321,31 +324,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const float* zk_tile = nullptr;
-        int zS = 0;
+        int zS = 0, ek0 = 0, ek1 = 0;
         if (AK) {
           const GroupInfo gk = p.gk[it];
           zk_tile = t.zk + (size_t)bh * p.zk_head + gk.base - gk.e0;
           zS = gk.S;
+          ek0 = gk.e0;
+          ek1 = gk.e0 + gk.W - 1;
         }
-        // in chunks of 32 columns: the compiler may not hoist the gathers of
-        // later chunks, which keeps the live registers bounded
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-#pragma unroll
-          for (int c = c0; c < c0 + 32; ++c) {
-            float rel = 0.f;
-            const int j = j0 + c;
-            // only kept cells: a masked cell's offset may lie outside the stored columns
-            if (rok && j < nkv && !(p.causal && j > i)) {
-              const int e = iclamp(j - i, p.E_lo, p.E_hi) - p.E_lo;
-              if (AQ) rel += __ldg(zq_row + e);
-              if (AK) rel += __ldg(zk_tile + (long long)c * zS + e);
-              if (BIAS) rel += __ldg(bexp + e);
-            }
-            x[c] = (x[c] + rel) * sc;
-          }
-          asm volatile("" ::: "memory");
-        }
+        band_terms_q<AQ, AK, BIAS>(x, p.E_lo, p.E_hi, i, j0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
+                                   imin(kBK, N - j0) - 1, ek0, ek1, bexp, sc);
       }
       const bool need_mask = (j0 + kBK > nkv) || (p.causal && j0 + kBK - 1 > q0 + g * kBQ);
       if (need_mask) {
