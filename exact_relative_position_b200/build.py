@@ -52,7 +52,7 @@ def _stale() -> bool:
 # Kernels that split their registers between warpgroups with setmaxnreg: the
 # split adds up to (threads x registers at launch), so the launch register
 # count must be exactly this value or the split could wait forever.
-REGISTER_SPLIT_KERNELS = {"fwd_sm100_kernel": 168}
+REGISTER_SPLIT_KERNELS = {"fwd_sm100_kernel": 168, "dq_sm100_kernel": 168, "dkdv_sm100_kernel": 168}
 
 
 def _check_register_split(ptxas_log: str):

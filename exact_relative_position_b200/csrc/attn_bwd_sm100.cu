@@ -87,7 +87,9 @@ __global__ void __launch_bounds__(256) prep_sm100_kernel(const OT* __restrict__ 
 
 // ------------------------------------------------------------------ Q-parallel
 namespace qp {
-constexpr int kThreads = 256;                 // warps 0..3: TMA, MMA, TMEM alloc, idle; 4..7 compute
+constexpr int kThreads = 384;                 // warps 0..3: TMA, MMA, TMEM alloc, idle; 4..11 compute
+constexpr int kRegLaunch = 168, kRegLow = 72, kRegHigh = 208;
+static_assert(128 * kRegLow + 256 * kRegHigh <= kThreads * kRegLaunch, "register split exceeds the launch");
 constexpr int kStages = 4;
 constexpr uint32_t kColvBytes = 2 * kT * 4;
 constexpr uint32_t kStageBytes = 2 * kTileBytes + 1024;   // K, V, saturated key columns
@@ -98,7 +100,8 @@ constexpr uint32_t kOffDS = kOffKV + kStages * kStageBytes;
 constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
-constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;
+constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 rows][2] saturated sums of column half 1
+constexpr uint32_t kSmemBytes = kOffSat + 1024 + 1024;
 // tensor memory: S buffers [0,128) and [128,256), dP [256,384), dQ [384,448)
 constexpr uint32_t kTmDP = 256, kTmDQ = 384;
 // barriers
@@ -138,11 +141,11 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(kBarSFull + u), 1);
-      mbar_init(bar(kBarSFree + u), 128);
+      mbar_init(bar(kBarSFree + u), 256);
     }
     mbar_init(bar(kBarDpFull), 1);
-    mbar_init(bar(kBarDpFree), 128);
-    mbar_init(bar(kBarDsReady), 128);
+    mbar_init(bar(kBarDpFree), 256);
+    mbar_init(bar(kBarDsReady), 256);
     mbar_init(bar(kBarDsFree), 1);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -157,115 +160,126 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    if (lane == 0 && nkt > 0) {
-      // ------------------------------------------------------------ TMA producer
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      prefetch_tmap(&tmDO);
-      mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
-      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
-      tma_load_3d(sb + kOffDO, &tmDO, bar(kBarQ), 0, q0, bh);
-#pragma unroll 1
-      for (int it = 0; it < nkt; ++it) {
-        const int s = it % kStages;
-        if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
-        const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
-        mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
-        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kT, bh);
-        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kT, bh);
-        if (AK) {
-          const float* src = t.zk_sat + (size_t)bh * 2 * npad + (size_t)it * kT;
-          bulk_load(dst + 2 * kTileBytes, src, kT * 4, bar(kBarKvFull + s));
-          bulk_load(dst + 2 * kTileBytes + kT * 4, src + npad, kT * 4, bar(kBarKvFull + s));
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && nkt > 0) {
-      // ------------------------------------------------------------ MMA issuer
-      // per tile t: dP(t+1) once dP(t) has been read, dQ += dS(t) K(t) once
-      // dS(t) is in shared memory, S(t+2) once S(t) has been read
-      const bool bf = t.is_bf16 != 0;
-      const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
-      const uint32_t id_dq = idesc_f16(bf, 128, 64, false, true);
-      const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
-      const uint64_t ddo0 = sdesc_sw128(sb + kOffDO, 16, 1024);
-      const uint64_t dk0 = sdesc_sw128(sb + kOffKV, 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 16, 1024);
-      const uint64_t dkmn0 = sdesc_sw128(sb + kOffKV, 8192, 1024);
-      const uint64_t dds0 = sdesc_sw128(sb + kOffDS, 16, 1024);
-      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
-      auto issue_s = [&](int buf, int s) {
-        const uint64_t kd = dk0 + (uint64_t)s * kStage16;
-#pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dq0 + 2 * kk, kd + 2 * kk, id_s, kk > 0);
-      };
-      auto issue_dp = [&](int s) {
-        const uint64_t vd = dv0 + (uint64_t)s * kStage16;
-#pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, ddo0 + 2 * kk, vd + 2 * kk, id_s, kk > 0);
-      };
-      auto issue_dq = [&](int s, bool acc) {
-        const uint64_t kd = dkmn0 + (uint64_t)s * kStage16;
-#pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kTmDQ, dds0 + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), kd + 128 * kk, id_dq,
-                 (acc || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        mma_commit(bar(kBarSFull + 0));
-        issue_dp(0);
-        mma_commit(bar(kBarDpFull));
-        if (nkt > 1) {
-          ok = mbar_wait(bar(kBarKvFull + 1), 0, abort_flag);
-          if (ok) {
-            tc_fence_after();
-            issue_s(1, 1);
-            mma_commit(bar(kBarSFull + 1));
+  // Register split: the launch gives every thread 168 registers (384 x 168 =
+  // 64512); warpgroup 0 (producer, MMA issuer, allocator) drops to kRegLow
+  // and the two compute warpgroups take kRegHigh (the sum fits: static_assert).
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow) : "memory");
+    if (warp == 0) {
+      if (lane == 0 && nkt > 0) {
+        // ------------------------------------------------------------ TMA producer
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmDO);
+        mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
+        tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
+        tma_load_3d(sb + kOffDO, &tmDO, bar(kBarQ), 0, q0, bh);
+  #pragma unroll 1
+        for (int it = 0; it < nkt; ++it) {
+          const int s = it % kStages;
+          if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+          const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
+          mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
+          tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kT, bh);
+          tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kT, bh);
+          if (AK) {
+            const float* src = t.zk_sat + (size_t)bh * 2 * npad + (size_t)it * kT;
+            bulk_load(dst + 2 * kTileBytes, src, kT * 4, bar(kBarKvFull + s));
+            bulk_load(dst + 2 * kTileBytes + kT * 4, src + npad, kT * 4, bar(kBarKvFull + s));
           }
         }
       }
-#pragma unroll 1
-      for (int it = 0; it < nkt && ok; ++it) {
-        const int s = it % kStages;
-        if (it + 1 < nkt) {
-          ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
-          if (!ok) break;
+    } else if (warp == 1) {
+      if (lane == 0 && nkt > 0) {
+        // ------------------------------------------------------------ MMA issuer
+        // per tile t: dP(t+1) once dP(t) has been read, dQ += dS(t) K(t) once
+        // dS(t) is in shared memory, S(t+2) once S(t) has been read
+        const bool bf = t.is_bf16 != 0;
+        const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
+        const uint32_t id_dq = idesc_f16(bf, 128, 64, false, true);
+        const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
+        const uint64_t ddo0 = sdesc_sw128(sb + kOffDO, 16, 1024);
+        const uint64_t dk0 = sdesc_sw128(sb + kOffKV, 16, 1024);
+        const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 16, 1024);
+        const uint64_t dkmn0 = sdesc_sw128(sb + kOffKV, 8192, 1024);
+        const uint64_t dds0 = sdesc_sw128(sb + kOffDS, 16, 1024);
+        constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
+        auto issue_s = [&](int buf, int s) {
+          const uint64_t kd = dk0 + (uint64_t)s * kStage16;
+  #pragma unroll 1
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dq0 + 2 * kk, kd + 2 * kk, id_s, kk > 0);
+        };
+        auto issue_dp = [&](int s) {
+          const uint64_t vd = dv0 + (uint64_t)s * kStage16;
+  #pragma unroll 1
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, ddo0 + 2 * kk, vd + 2 * kk, id_s, kk > 0);
+        };
+        auto issue_dq = [&](int s, bool acc) {
+          const uint64_t kd = dkmn0 + (uint64_t)s * kStage16;
+  #pragma unroll 1
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + kTmDQ, dds0 + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), kd + 128 * kk, id_dq,
+                   (acc || kk > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
+        if (ok) {
           tc_fence_after();
-          issue_dp((it + 1) % kStages);
+          issue_s(0, 0);
+          mma_commit(bar(kBarSFull + 0));
+          issue_dp(0);
           mma_commit(bar(kBarDpFull));
+          if (nkt > 1) {
+            ok = mbar_wait(bar(kBarKvFull + 1), 0, abort_flag);
+            if (ok) {
+              tc_fence_after();
+              issue_s(1, 1);
+              mma_commit(bar(kBarSFull + 1));
+            }
+          }
         }
-        ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_dq(s, it > 0);
-        mma_commit(bar(kBarDsFree));
-        mma_commit(bar(kBarKvEmpty + s));
-        if (it + 2 < nkt) {
-          const int s2 = (it + 2) % kStages;
-          ok = mbar_wait(bar(kBarKvFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
-               mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+  #pragma unroll 1
+        for (int it = 0; it < nkt && ok; ++it) {
+          const int s = it % kStages;
+          if (it + 1 < nkt) {
+            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp((it + 1) % kStages);
+            mma_commit(bar(kBarDpFull));
+          }
+          ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_s(it & 1, s2);
-          mma_commit(bar(kBarSFull + (it & 1)));
+          issue_dq(s, it > 0);
+          mma_commit(bar(kBarDsFree));
+          mma_commit(bar(kBarKvEmpty + s));
+          if (it + 2 < nkt) {
+            const int s2 = (it + 2) % kStages;
+            ok = mbar_wait(bar(kBarKvFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
+                 mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(it & 1, s2);
+            mma_commit(bar(kBarSFull + (it & 1)));
+          }
         }
-      }
-      if (!ok) {
-        mma_commit(bar(kBarDrain));
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+        if (!ok) {
+          mma_commit(bar(kBarDrain));
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+          }
         }
       }
     }
-  } else if (warp >= 4) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh) : "memory");
     // -------------------------------------------------------------- compute
-    const int r = (warp - 4) * 32 + lane;        // row of the tile = tensor-memory lane
+    // warps 4..7 take key columns 0..63 of the tile, warps 8..11 columns
+    // 64..127, both for rows r = (warp & 3) * 32 + lane (the tensor-memory lane)
+    const int hc = (warp - 4) >> 2;
+    const int cb = 64 * hc;
+    const int r = (warp & 3) * 32 + lane;
     const int i = q0 + r;
     const bool rok = i < N;
     const uint32_t t_lane = (uint32_t)((warp & 3) * 32) << 16;
@@ -294,18 +308,16 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
       const int stage = it % kStages, buf = it & 1;
       const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
-                        (cls == RELPOS_TILE_CONST_LO ? 0 : kT);
+                        (cls == RELPOS_TILE_CONST_LO ? 0 : kT) + cb;
       const bool got_s = mbar_wait(bar(kBarSFull + buf), (it >> 1) & 1, abort_flag) &&
                          (!(AK && is_const) || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
+      float x[64];
       {
-        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128;
+        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128 + cb;
         tmem_ld32(ts + 0, reinterpret_cast<uint32_t*>(x) + 0);
         tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
-        tmem_ld32(ts + 64, reinterpret_cast<uint32_t*>(x) + 64);
-        tmem_ld32(ts + 96, reinterpret_cast<uint32_t*>(x) + 96);
         tmem_wait_ld();
       }
       tc_fence_before();
@@ -315,7 +327,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         const float off = (cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi) - lse2;
         if (AK) {
 #pragma unroll
-          for (int c = 0; c < 128; c += 4) {
+          for (int c = 0; c < 64; c += 4) {
             const float4 v4 = *reinterpret_cast<const float4*>(cv + c);
             x[c] = fast_exp2(fmaf(x[c], sc, v4.x) + off);
             x[c + 1] = fast_exp2(fmaf(x[c + 1], sc, v4.y) + off);
@@ -324,7 +336,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] = fast_exp2(fmaf(x[c], sc, off));
+          for (int c = 0; c < 64; ++c) x[c] = fast_exp2(fmaf(x[c], sc, off));
         }
       } else {
         const float* zk_tile = nullptr;
@@ -336,118 +348,122 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           ek0 = gk.e0;
           ek1 = gk.e0 + gk.W - 1;
         }
-        band_terms_q<AQ, AK, BIAS>(x, p.E_lo, p.E_hi, i, j0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
-                                   imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
+        band_terms_q<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, i, j0, cb, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
+                                       imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = fast_exp2(x[c] - lse2);
+        for (int c = 0; c < 64; ++c) x[c] = fast_exp2(x[c] - lse2);
       }
       const bool need_mask = (j0 + kT > nkv) || (p.causal && j0 + kT - 1 > q0);
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int j = j0 + c;
+        for (int c = 0; c < 64; ++c) {
+          const int j = j0 + cb + c;
           if (j >= nkv || (p.causal && j > i)) x[c] = 0.f;
         }
       }
-      // dS = P (dP - D) in two halves of 64 keys; written as the 16-bit A
+      // dS = P (dP - D) for this thread's 64 keys; written as the 16-bit A
       // operand of dQ += dS K
       const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
       tc_fence_after();
-      float ssum[2] = {0.f, 0.f};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t dp[64];
-        const uint32_t td = tmem + t_lane + kTmDP + 64 * half;
+        const uint32_t td = tmem + t_lane + kTmDP + cb;
         tmem_ld32(td, dp);
         tmem_ld32(td + 32, dp + 32);
         tmem_wait_ld();
-        if (half == 1) {
-          tc_fence_before();
-          mbar_arrive(bar(kBarDpFree));     // dP(t + 1) may now be written
-        }
-        if (half == 0 && it > 0) {
-          const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        }
-#pragma unroll
+        tc_fence_before();
+        mbar_arrive(bar(kBarDpFree));     // dP(t + 1) may now be written
         if (!DZQ || is_const) {
+          float ssum[2] = {0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            const int cc = 64 * half + c;
-            const float ds = x[cc] * (__uint_as_float(dp[c]) - dval);
-            x[cc] = ds;
+            const float ds = x[c] * (__uint_as_float(dp[c]) - dval);
+            x[c] = ds;
             if (DZQ) ssum[c & 1] += ds;
+          }
+          if (DZQ) {
+            if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
+            else sat_hi += ssum[0] + ssum[1];
           }
         } else {
           // saturated cells summed here; the interior ones are stored below.
-          // Kept columns are c <= ckeep; low-saturated c <= clo, high c >= chi.
+          // Kept keys are cc <= ckeep (cc = key - j0); low-saturated cc <= clo, high cc >= chi.
           int ckeep = rok ? imin(nkv - 1 - j0, 127) : -1;
           if (p.causal) ckeep = imin(ckeep, i - j0);
           const int clo = imin(p.E_lo + i - j0, ckeep);
           const int chi = imax(p.E_hi + i - j0, p.E_lo + i - j0 + 1);
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            const int cc = 64 * half + c;
-            const float ds = x[cc] * (__uint_as_float(dp[c]) - dval);
-            x[cc] = ds;
+            const int cc = cb + c;
+            const float ds = x[c] * (__uint_as_float(dp[c]) - dval);
+            x[c] = ds;
             sat_lo += cc <= clo ? ds : 0.f;
             sat_hi += (cc >= chi && cc <= ckeep) ? ds : 0.f;
           }
         }
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int cc = 64 * half + 8 * ch;
-          st_shared_v4(op_chunk(dsb, r, 8 * half + ch), DT<T>::pack(x[cc], x[cc + 1]), DT<T>::pack(x[cc + 2], x[cc + 3]),
-                       DT<T>::pack(x[cc + 4], x[cc + 5]), DT<T>::pack(x[cc + 6], x[cc + 7]));
-        }
       }
-      if (!ok) break;
-      if (DZQ && is_const) {
-        if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
-        else sat_hi += ssum[0] + ssum[1];
+      if (it > 0) {
+        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const int c = 8 * ch;
+        st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), DT<T>::pack(x[c], x[c + 1]), DT<T>::pack(x[c + 2], x[c + 3]),
+                     DT<T>::pack(x[c + 4], x[c + 5]), DT<T>::pack(x[c + 6], x[c + 7]));
       }
       if (DZQ && !is_const) {
         __syncwarp();
-        dz_band_store<T>(dsb, (warp - 4) * 32, lane, false, q0, j0, nrows_q, nkv, N, p.causal, p.E_lo, p.E_hi,
-                         dzq_base, gi.S, gi.e0, p.tau);
+        dz_band_store<T, 64>(dsb, (warp & 3) * 32, lane, false, q0, j0, cb, nrows_q, nkv, N, p.causal, p.E_lo,
+                             p.E_hi, dzq_base, gi.S, gi.e0, p.tau);
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarDsReady));
     }
     // -------------------------------------------------------------- epilogue
-    if (DZQ && rok) {
-      // the two saturated offsets of the row, written once
-      if (p.Rexp == 1) {
-        dzq_row[0] = p.tau * (sat_lo + sat_hi);
-      } else {
-        if (gi.e0 == 0) dzq_row[0] = p.tau * sat_lo;
-        if (p.Rexp - 1 < gi.e0 + gi.W) dzq_row[p.Rexp - 1] = p.tau * sat_hi;
+    if (DZQ) {
+      // combine the two column halves' saturated sums; half 0 writes them
+      float* sat = reinterpret_cast<float*>(sg + kOffSat);
+      if (hc == 1) {
+        sat[2 * r] = sat_lo;
+        sat[2 * r + 1] = sat_hi;
+      }
+      named_bar_sync(1, 256);
+      if (hc == 0 && rok) {
+        sat_lo += sat[2 * r];
+        sat_hi += sat[2 * r + 1];
+        if (p.Rexp == 1) {
+          dzq_row[0] = p.tau * (sat_lo + sat_hi);
+        } else {
+          if (gi.e0 == 0) dzq_row[0] = p.tau * sat_lo;
+          if (p.Rexp - 1 < gi.e0 + gi.W) dzq_row[p.Rexp - 1] = p.tau * sat_hi;
+        }
       }
     }
-    float dq[64];
+    // dQ: half hc stores head-dim columns [32 hc, 32 hc + 32) of its row
+    float dq[32];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) dq[c] = 0.f;
+    for (int c = 0; c < 32; ++c) dq[c] = 0.f;
     const bool got_q = nkt > 0 && ok && mbar_wait(bar(kBarDsFree), (nkt - 1) & 1, abort_flag);
     if (__all_sync(0xffffffffu, got_q)) {
       tc_fence_after();
-      uint32_t u[64];
-      tmem_ld32(tmem + t_lane + kTmDQ, u);
-      tmem_ld32(tmem + t_lane + kTmDQ + 32, u + 32);
+      uint32_t u[32];
+      tmem_ld32(tmem + t_lane + kTmDQ + 32 * hc, u);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 64; ++c) dq[c] = __uint_as_float(u[c]) * p.tau;
+      for (int c = 0; c < 32; ++c) dq[c] = __uint_as_float(u[c]) * p.tau;
     }
     if (rok) {
-      const size_t o = ((size_t)bh * N + i) * 64;
+      const size_t o = ((size_t)bh * N + i) * 64 + 32 * hc;
       if (DQ32) {
         float* dst = t.dq_acc + o;
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dq[c], dq[c + 1], dq[c + 2], dq[c + 3]);
+        for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dq[c], dq[c + 1], dq[c + 2], dq[c + 3]);
       } else {
         T* dst = static_cast<T*>(t.dq) + o;
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
+        for (int c = 0; c < 32; c += 8) {
           uint4 w;
           w.x = DT<T>::pack(dq[c], dq[c + 1]);
           w.y = DT<T>::pack(dq[c + 2], dq[c + 3]);
@@ -469,7 +485,9 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
 
 // ------------------------------------------------------------------ K-parallel
 namespace kp {
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;                 // warps 0..3: TMA, MMA, TMEM alloc, idle; 4..11 compute
+constexpr int kRegLaunch = 168, kRegLow = 88, kRegHigh = 208;
+static_assert(128 * kRegLow + 256 * kRegHigh <= kThreads * kRegLaunch, "register split exceeds the launch");
 constexpr int kStages = 3;
 // a stage: Q tile, dO tile, then LSE log2e, D and the two saturated query
 // columns (tau log2e (Z^Q[i, sat] + b_sat)) of the query tile, 128 floats each
@@ -483,7 +501,8 @@ constexpr uint32_t kOffDS = kOffP + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
-constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;
+constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 keys][2] saturated sums of column half 1
+constexpr uint32_t kSmemBytes = kOffSat + 1024 + 1024;
 // tensor memory: S^T buffers [0,128), [128,256), dP^T [256,384), dV [384,448), dK [448,512)
 constexpr uint32_t kTmDP = 256, kTmDV = 384, kTmDK = 448;
 constexpr int kBarKV = 0, kBarQsFull = 1, kBarQsEmpty = kBarQsFull + kStages, kBarSFull = kBarQsEmpty + kStages,
@@ -522,13 +541,13 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(kBarSFull + u), 1);
-      mbar_init(bar(kBarSFree + u), 128);
+      mbar_init(bar(kBarSFree + u), 256);
     }
     mbar_init(bar(kBarDpFull), 1);
-    mbar_init(bar(kBarDpFree), 128);
-    mbar_init(bar(kBarPReady), 128);
+    mbar_init(bar(kBarDpFree), 256);
+    mbar_init(bar(kBarPReady), 256);
     mbar_init(bar(kBarPFree), 1);
-    mbar_init(bar(kBarDsReady), 128);
+    mbar_init(bar(kBarDsReady), 256);
     mbar_init(bar(kBarDsFree), 1);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
@@ -543,124 +562,135 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    if (lane == 0 && nq > 0) {
-      // ------------------------------------------------------------ TMA producer
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      prefetch_tmap(&tmDO);
-      mbar_expect_tx(bar(kBarKV), 2 * kTileBytes);
-      tma_load_3d(sb + kOffK, &tmK, bar(kBarKV), 0, k0, bh);
-      tma_load_3d(sb + kOffV, &tmV, bar(kBarKV), 0, k0, bh);
-#pragma unroll 1
-      for (int it = 0; it < nq; ++it) {
-        const int s = it % kStages;
-        if (it >= kStages && !mbar_wait(bar(kBarQsEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
-        const int qb = (qt0 + it) * kT;
-        const uint32_t dst = sb + kOffQD + (uint32_t)s * kStageBytes;
-        const uint32_t fb = bar(kBarQsFull + s);
-        mbar_expect_tx(fb, 2 * kTileBytes + ((AQ || BIAS) ? kVecBytes : kVecBytes / 2));
-        tma_load_3d(dst, &tmQ, fb, 0, qb, bh);
-        tma_load_3d(dst + kTileBytes, &tmDO, fb, 0, qb, bh);
-        const size_t vo = (size_t)bh * npad + qb;
-        bulk_load(dst + 2 * kTileBytes, t.lse2 + vo, kT * 4, fb);
-        bulk_load(dst + 2 * kTileBytes + kT * 4, t.dsum + vo, kT * 4, fb);
-        if (AQ || BIAS) {
-          const float* src = t.zq_sat + (size_t)bh * 2 * npad + qb;
-          bulk_load(dst + 2 * kTileBytes + 2 * kT * 4, src, kT * 4, fb);
-          bulk_load(dst + 2 * kTileBytes + 3 * kT * 4, src + npad, kT * 4, fb);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && nq > 0) {
-      // ------------------------------------------------------------ MMA issuer
-      const bool bf = t.is_bf16 != 0;
-      const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
-      const uint32_t id_g = idesc_f16(bf, 128, 64, false, true);
-      const uint64_t dk = sdesc_sw128(sb + kOffK, 16, 1024);
-      const uint64_t dv = sdesc_sw128(sb + kOffV, 16, 1024);
-      const uint64_t dq0 = sdesc_sw128(sb + kOffQD, 16, 1024);
-      const uint64_t ddo0 = sdesc_sw128(sb + kOffQD + kTileBytes, 16, 1024);
-      const uint64_t dqmn0 = sdesc_sw128(sb + kOffQD, 8192, 1024);
-      const uint64_t ddomn0 = sdesc_sw128(sb + kOffQD + kTileBytes, 8192, 1024);
-      const uint64_t dp_ = sdesc_sw128(sb + kOffP, 16, 1024);
-      const uint64_t dds = sdesc_sw128(sb + kOffDS, 16, 1024);
-      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
-      auto issue_s = [&](int buf, int s) {
-        const uint64_t qd = dq0 + (uint64_t)s * kStage16;
-#pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dk + 2 * kk, qd + 2 * kk, id_s, kk > 0);
-      };
-      auto issue_dp = [&](int s) {
-        const uint64_t od = ddo0 + (uint64_t)s * kStage16;
-#pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, dv + 2 * kk, od + 2 * kk, id_s, kk > 0);
-      };
-      // D[keys x 64] (+)= A[keys x queries] (shared) * B[queries x 64] (MN-major)
-      auto issue_g = [&](uint32_t d, uint64_t a, uint64_t bmn, bool acc) {
-#pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(d, a + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(bar(kBarKV), 0, abort_flag) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        mma_commit(bar(kBarSFull + 0));
-        issue_dp(0);
-        mma_commit(bar(kBarDpFull));
-        if (nq > 1) {
-          ok = mbar_wait(bar(kBarQsFull + 1), 0, abort_flag);
-          if (ok) {
-            tc_fence_after();
-            issue_s(1, 1);
-            mma_commit(bar(kBarSFull + 1));
+  // Register split: the launch gives every thread 168 registers (384 x 168 =
+  // 64512); warpgroup 0 (producer, MMA issuer, allocator) drops to kRegLow
+  // and the two compute warpgroups take kRegHigh (the sum fits: static_assert).
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow) : "memory");
+    if (warp == 0) {
+      if (lane == 0 && nq > 0) {
+        // ------------------------------------------------------------ TMA producer
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmDO);
+        mbar_expect_tx(bar(kBarKV), 2 * kTileBytes);
+        tma_load_3d(sb + kOffK, &tmK, bar(kBarKV), 0, k0, bh);
+        tma_load_3d(sb + kOffV, &tmV, bar(kBarKV), 0, k0, bh);
+  #pragma unroll 1
+        for (int it = 0; it < nq; ++it) {
+          const int s = it % kStages;
+          if (it >= kStages && !mbar_wait(bar(kBarQsEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+          const int qb = (qt0 + it) * kT;
+          const uint32_t dst = sb + kOffQD + (uint32_t)s * kStageBytes;
+          const uint32_t fb = bar(kBarQsFull + s);
+          mbar_expect_tx(fb, 2 * kTileBytes + ((AQ || BIAS) ? kVecBytes : kVecBytes / 2));
+          tma_load_3d(dst, &tmQ, fb, 0, qb, bh);
+          tma_load_3d(dst + kTileBytes, &tmDO, fb, 0, qb, bh);
+          const size_t vo = (size_t)bh * npad + qb;
+          bulk_load(dst + 2 * kTileBytes, t.lse2 + vo, kT * 4, fb);
+          bulk_load(dst + 2 * kTileBytes + kT * 4, t.dsum + vo, kT * 4, fb);
+          if (AQ || BIAS) {
+            const float* src = t.zq_sat + (size_t)bh * 2 * npad + qb;
+            bulk_load(dst + 2 * kTileBytes + 2 * kT * 4, src, kT * 4, fb);
+            bulk_load(dst + 2 * kTileBytes + 3 * kT * 4, src + npad, kT * 4, fb);
           }
         }
       }
-#pragma unroll 1
-      for (int it = 0; it < nq && ok; ++it) {
-        const int s = it % kStages;
-        if (it + 1 < nq) {
-          ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
-          if (!ok) break;
+    } else if (warp == 1) {
+      if (lane == 0 && nq > 0) {
+        // ------------------------------------------------------------ MMA issuer
+        const bool bf = t.is_bf16 != 0;
+        const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
+        const uint32_t id_g = idesc_f16(bf, 128, 64, false, true);
+        const uint64_t dk = sdesc_sw128(sb + kOffK, 16, 1024);
+        const uint64_t dv = sdesc_sw128(sb + kOffV, 16, 1024);
+        const uint64_t dq0 = sdesc_sw128(sb + kOffQD, 16, 1024);
+        const uint64_t ddo0 = sdesc_sw128(sb + kOffQD + kTileBytes, 16, 1024);
+        const uint64_t dqmn0 = sdesc_sw128(sb + kOffQD, 8192, 1024);
+        const uint64_t ddomn0 = sdesc_sw128(sb + kOffQD + kTileBytes, 8192, 1024);
+        const uint64_t dp_ = sdesc_sw128(sb + kOffP, 16, 1024);
+        const uint64_t dds = sdesc_sw128(sb + kOffDS, 16, 1024);
+        constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
+        auto issue_s = [&](int buf, int s) {
+          const uint64_t qd = dq0 + (uint64_t)s * kStage16;
+  #pragma unroll 1
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dk + 2 * kk, qd + 2 * kk, id_s, kk > 0);
+        };
+        auto issue_dp = [&](int s) {
+          const uint64_t od = ddo0 + (uint64_t)s * kStage16;
+  #pragma unroll 1
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, dv + 2 * kk, od + 2 * kk, id_s, kk > 0);
+        };
+        // D[keys x 64] (+)= A[keys x queries] (shared) * B[queries x 64] (MN-major)
+        auto issue_g = [&](uint32_t d, uint64_t a, uint64_t bmn, bool acc) {
+  #pragma unroll 1
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(d, a + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait(bar(kBarKV), 0, abort_flag) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag);
+        if (ok) {
           tc_fence_after();
-          issue_dp((it + 1) % kStages);
+          issue_s(0, 0);
+          mma_commit(bar(kBarSFull + 0));
+          issue_dp(0);
           mma_commit(bar(kBarDpFull));
+          if (nq > 1) {
+            ok = mbar_wait(bar(kBarQsFull + 1), 0, abort_flag);
+            if (ok) {
+              tc_fence_after();
+              issue_s(1, 1);
+              mma_commit(bar(kBarSFull + 1));
+            }
+          }
         }
-        ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_g(tmem + kTmDV, dp_, ddomn0 + (uint64_t)s * kStage16, it > 0);
-        mma_commit(bar(kBarPFree));
-        ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_g(tmem + kTmDK, dds, dqmn0 + (uint64_t)s * kStage16, it > 0);
-        mma_commit(bar(kBarDsFree));
-        mma_commit(bar(kBarQsEmpty + s));
-        if (it + 2 < nq) {
-          const int s2 = (it + 2) % kStages;
-          ok = mbar_wait(bar(kBarQsFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
-               mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+  #pragma unroll 1
+        for (int it = 0; it < nq && ok; ++it) {
+          const int s = it % kStages;
+          if (it + 1 < nq) {
+            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp((it + 1) % kStages);
+            mma_commit(bar(kBarDpFull));
+          }
+          ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_s(it & 1, s2);
-          mma_commit(bar(kBarSFull + (it & 1)));
+          issue_g(tmem + kTmDV, dp_, ddomn0 + (uint64_t)s * kStage16, it > 0);
+          mma_commit(bar(kBarPFree));
+          ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_g(tmem + kTmDK, dds, dqmn0 + (uint64_t)s * kStage16, it > 0);
+          mma_commit(bar(kBarDsFree));
+          mma_commit(bar(kBarQsEmpty + s));
+          if (it + 2 < nq) {
+            const int s2 = (it + 2) % kStages;
+            ok = mbar_wait(bar(kBarQsFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
+                 mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(it & 1, s2);
+            mma_commit(bar(kBarSFull + (it & 1)));
+          }
         }
-      }
-      if (!ok) {
-        mma_commit(bar(kBarDrain));
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+        if (!ok) {
+          mma_commit(bar(kBarDrain));
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
+          }
         }
       }
     }
-  } else if (warp >= 4) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh) : "memory");
     // -------------------------------------------------------------- compute
-    const int r = (warp - 4) * 32 + lane;        // key of the tile = tensor-memory lane
+    // warps 4..7 take query columns 0..63 of the tile, warps 8..11 columns
+    // 64..127, both for keys r = (warp & 3) * 32 + lane (the tensor-memory lane)
+    const int hc = (warp - 4) >> 2;
+    const int cb = 64 * hc;
+    const int r = (warp & 3) * 32 + lane;
     const int j = k0 + r;
     const bool jok = j < N;
     const bool jkeep = j < nkv;                  // keys past key_len are masked for every query
@@ -687,30 +717,28 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
       const int stage = it % kStages, buf = it & 1;
       const float* vec = reinterpret_cast<const float*>(sg + kOffQD + (uint32_t)stage * kStageBytes + 2 * kTileBytes);
-      const float* lse2v = vec;
-      const float* dvec = vec + kT;
-      const float* cvq = vec + (cls == RELPOS_TILE_CONST_LO ? 2 * kT : 3 * kT);
+      const float* lse2v = vec + cb;
+      const float* dvec = vec + kT + cb;
+      const float* cvq = vec + (cls == RELPOS_TILE_CONST_LO ? 2 * kT : 3 * kT) + cb;
       // the stage's own barrier makes its TMA-written vectors visible to these threads
       const bool got_s = mbar_wait(bar(kBarSFull + buf), (it >> 1) & 1, abort_flag) &&
                          mbar_wait(bar(kBarQsFull + stage), (it / kStages) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
+      float x[64];
       {
-        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128;
+        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128 + cb;
         tmem_ld32(ts + 0, reinterpret_cast<uint32_t*>(x) + 0);
         tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
-        tmem_ld32(ts + 64, reinterpret_cast<uint32_t*>(x) + 64);
-        tmem_ld32(ts + 96, reinterpret_cast<uint32_t*>(x) + 96);
         tmem_wait_ld();
       }
       tc_fence_before();
       mbar_arrive(bar(kBarSFree + buf));
-      // P^T = 2^(S^T tau log2e + relation terms - LSE_i log2e), column c = query qb + c
+      // P^T = 2^(S^T tau log2e + relation terms - LSE_i log2e), column c = query qb + cb + c
       if (is_const) {
         const float rowk = cls == RELPOS_TILE_CONST_LO ? rowk_lo : rowk_hi;
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
           float4 w4 = make_float4(-l4.x, -l4.y, -l4.z, -l4.w);
           if (AQ || BIAS) {
@@ -732,10 +760,10 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           eq0 = gq.e0;
           eq1 = gq.e0 + gq.W - 1;
         }
-        band_terms_k<AQ, AK, BIAS>(x, p.E_lo, p.E_hi, j, qb, zk_row, gk.e0, gk.e0 + gk.W - 1, zq_tile, zS,
-                                   imin(kT, N - qb) - 1, eq0, eq1, bexp, sc);
+        band_terms_k<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, j, qb, cb, zk_row, gk.e0, gk.e0 + gk.W - 1, zq_tile, zS,
+                                       imin(kT, N - qb) - 1, eq0, eq1, bexp, sc);
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
           x[c] = fast_exp2(x[c] - l4.x);
           x[c + 1] = fast_exp2(x[c + 1] - l4.y);
@@ -746,8 +774,8 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       const bool need_mask = !jkeep || (p.causal && k0 + kT - 1 > qb);
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          if (!jkeep || (p.causal && j > qb + c)) x[c] = 0.f;
+        for (int c = 0; c < 64; ++c) {
+          if (!jkeep || (p.causal && j > qb + cb + c)) x[c] = 0.f;
         }
       }
       // P^T to shared memory: the A operand of dV += P^T dO
@@ -756,126 +784,127 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int cc = 8 * ch;
-        st_shared_v4(op_chunk(pb, r, ch), DT<T>::pack(x[cc], x[cc + 1]), DT<T>::pack(x[cc + 2], x[cc + 3]),
-                     DT<T>::pack(x[cc + 4], x[cc + 5]), DT<T>::pack(x[cc + 6], x[cc + 7]));
+      for (int ch = 0; ch < 8; ++ch) {
+        const int c = 8 * ch;
+        st_shared_v4(op_chunk(pb, r, 8 * hc + ch), DT<T>::pack(x[c], x[c + 1]), DT<T>::pack(x[c + 2], x[c + 3]),
+                     DT<T>::pack(x[c + 4], x[c + 5]), DT<T>::pack(x[c + 6], x[c + 7]));
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarPReady));
-      // dS^T = P^T (dP^T - D_i) in two halves of 64 queries: the A operand of
-      // dK += dS^T Q, and the key-side relation gradient of this key row
+      // dS^T = P^T (dP^T - D_i): the A operand of dK += dS^T Q, and the
+      // key-side relation gradient of this key row
       const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
       tc_fence_after();
-      float ssum[2] = {0.f, 0.f};
-      // column ranges of this key row (column cc = query qb + cc): kept for
-      // ckeep_lo <= cc <= ckeep_hi; low-saturated (j - i <= E_lo) for cc >= clo;
-      // high-saturated (j - i >= E_hi, not low) for cc <= chi
-      const int ckeep_lo = p.causal ? imax(j - qb, 0) : 0;
-      const int ckeep_hi = jkeep ? imin(N - 1 - qb, 127) : -1;
-      const int clo = j - qb - p.E_lo;
-      const int chi = imin(j - qb - p.E_hi, clo - 1);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t dp[64];
-        const uint32_t td = tmem + t_lane + kTmDP + 64 * half;
+        const uint32_t td = tmem + t_lane + kTmDP + cb;
         tmem_ld32(td, dp);
         tmem_ld32(td + 32, dp + 32);
         tmem_wait_ld();
-        if (half == 1) {
-          tc_fence_before();
-          mbar_arrive(bar(kBarDpFree));
-        }
-        if (half == 0 && it > 0) {
-          const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        }
+        tc_fence_before();
+        mbar_arrive(bar(kBarDpFree));
         if (!DZK || is_const) {
+          float ssum[2] = {0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
-            const int cc0 = 64 * half + c;
-            const float4 d4 = *reinterpret_cast<const float4*>(dvec + cc0);
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + c);
             const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const int cc = cc0 + u;
-              const float ds = x[cc] * (__uint_as_float(dp[c + u]) - dd[u]);
-              x[cc] = ds;
+              const float ds = x[c + u] * (__uint_as_float(dp[c + u]) - dd[u]);
+              x[c + u] = ds;
               if (DZK) ssum[u & 1] += ds;
             }
           }
+          if (DZK) {
+            if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
+            else sat_hi += ssum[0] + ssum[1];
+          }
         } else {
-          // kept columns are ckeep_lo <= cc <= ckeep_hi; delta = j - qb - cc is
-          // low-saturated for cc >= clo and high-saturated for cc <= chi
+          // column cc = query qb + cc of this key row: kept for
+          // ckeep_lo <= cc <= ckeep_hi; delta = j - qb - cc is low-saturated
+          // for cc >= clo and high-saturated (and not low) for cc <= chi
+          const int ckeep_lo = p.causal ? imax(j - qb, 0) : 0;
+          const int ckeep_hi = jkeep ? imin(N - 1 - qb, 127) : -1;
+          const int clo = j - qb - p.E_lo;
+          const int chi = imin(j - qb - p.E_hi, clo - 1);
           const int lo_beg = imax(clo, ckeep_lo), hi_end = imin(chi, ckeep_hi);
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
-            const int cc0 = 64 * half + c;
-            const float4 d4 = *reinterpret_cast<const float4*>(dvec + cc0);
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + c);
             const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const int cc = cc0 + u;
-              const float ds = x[cc] * (__uint_as_float(dp[c + u]) - dd[u]);
-              x[cc] = ds;
+              const int cc = cb + c + u;
+              const float ds = x[c + u] * (__uint_as_float(dp[c + u]) - dd[u]);
+              x[c + u] = ds;
               sat_lo += (cc >= lo_beg && cc <= ckeep_hi) ? ds : 0.f;
               sat_hi += (cc <= hi_end && cc >= ckeep_lo) ? ds : 0.f;
             }
           }
         }
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int cc = 64 * half + 8 * ch;
-          st_shared_v4(op_chunk(dsb, r, 8 * half + ch), DT<T>::pack(x[cc], x[cc + 1]), DT<T>::pack(x[cc + 2], x[cc + 3]),
-                       DT<T>::pack(x[cc + 4], x[cc + 5]), DT<T>::pack(x[cc + 6], x[cc + 7]));
-        }
       }
-      if (!ok) break;
-      if (DZK && is_const) {
-        if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
-        else sat_hi += ssum[0] + ssum[1];
+      if (it > 0) {
+        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const int c = 8 * ch;
+        st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), DT<T>::pack(x[c], x[c + 1]), DT<T>::pack(x[c + 2], x[c + 3]),
+                     DT<T>::pack(x[c + 4], x[c + 5]), DT<T>::pack(x[c + 6], x[c + 7]));
       }
       if (DZK && !is_const) {
         __syncwarp();
-        dz_band_store<T>(dsb, (warp - 4) * 32, lane, true, k0, qb, nrows_k, nkv, N, p.causal, p.E_lo, p.E_hi,
-                         dzk_base, gk.S, gk.e0, p.tau);
+        dz_band_store<T, 64>(dsb, (warp & 3) * 32, lane, true, k0, qb, cb, nrows_k, nkv, N, p.causal, p.E_lo,
+                             p.E_hi, dzk_base, gk.S, gk.e0, p.tau);
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarDsReady));
     }
     // -------------------------------------------------------------- epilogue
-    if (DZK && jok) {
-      if (p.Rexp == 1) {
-        dzk_row[0] = p.tau * (sat_lo + sat_hi);
-      } else {
-        if (gk.e0 == 0) dzk_row[0] = p.tau * sat_lo;
-        if (p.Rexp - 1 < gk.e0 + gk.W) dzk_row[p.Rexp - 1] = p.tau * sat_hi;
+    if (DZK) {
+      // combine the two column halves' saturated sums; half 0 writes them
+      float* sat = reinterpret_cast<float*>(sg + kOffSat);
+      if (hc == 1) {
+        sat[2 * r] = sat_lo;
+        sat[2 * r + 1] = sat_hi;
+      }
+      named_bar_sync(1, 256);
+      if (hc == 0 && jok) {
+        sat_lo += sat[2 * r];
+        sat_hi += sat[2 * r + 1];
+        if (p.Rexp == 1) {
+          dzk_row[0] = p.tau * (sat_lo + sat_hi);
+        } else {
+          if (gk.e0 == 0) dzk_row[0] = p.tau * sat_lo;
+          if (p.Rexp - 1 < gk.e0 + gk.W) dzk_row[p.Rexp - 1] = p.tau * sat_hi;
+        }
       }
     }
-    float dv[64], dk[64];
+    // dV and dK: half hc stores head-dim columns [32 hc, 32 hc + 32) of its key
+    float dv[32], dk[32];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) dv[c] = dk[c] = 0.f;
+    for (int c = 0; c < 32; ++c) dv[c] = dk[c] = 0.f;
     const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDsFree), (nq - 1) & 1, abort_flag);
     if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
-      uint32_t u[64];
-      tmem_ld32(tmem + t_lane + kTmDV, u);
-      tmem_ld32(tmem + t_lane + kTmDV + 32, u + 32);
+      uint32_t u[32];
+      tmem_ld32(tmem + t_lane + kTmDV + 32 * hc, u);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 64; ++c) dv[c] = __uint_as_float(u[c]);
-      tmem_ld32(tmem + t_lane + kTmDK, u);
-      tmem_ld32(tmem + t_lane + kTmDK + 32, u + 32);
+      for (int c = 0; c < 32; ++c) dv[c] = __uint_as_float(u[c]);
+      tmem_ld32(tmem + t_lane + kTmDK + 32 * hc, u);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 64; ++c) dk[c] = __uint_as_float(u[c]) * p.tau;
+      for (int c = 0; c < 32; ++c) dk[c] = __uint_as_float(u[c]) * p.tau;
     }
     if (jok) {
-      const size_t o = ((size_t)bh * N + j) * 64;
+      const size_t o = ((size_t)bh * N + j) * 64 + 32 * hc;
       T* vdst = static_cast<T*>(t.dv) + o;
 #pragma unroll
-      for (int c = 0; c < 64; c += 8) {
+      for (int c = 0; c < 32; c += 8) {
         uint4 w;
         w.x = DT<T>::pack(dv[c], dv[c + 1]);
         w.y = DT<T>::pack(dv[c + 2], dv[c + 3]);
@@ -886,11 +915,11 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       if (DK32) {
         float* dst = t.dk_acc + o;
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dk[c], dk[c + 1], dk[c + 2], dk[c + 3]);
+        for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dk[c], dk[c + 1], dk[c + 2], dk[c + 3]);
       } else {
         T* dst = static_cast<T*>(t.dk) + o;
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
+        for (int c = 0; c < 32; c += 8) {
           uint4 w;
           w.x = DT<T>::pack(dk[c], dk[c + 1]);
           w.y = DT<T>::pack(dk[c + 2], dk[c + 3]);

@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ek0 = gk.e0;
           ek1 = gk.e0 + gk.W - 1;
         }
-        band_terms_q<AQ, AK, BIAS>(x, p.E_lo, p.E_hi, i, j0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
-                                   imin(kBK, N - j0) - 1, ek0, ek1, bexp, sc);
+        band_terms_q<AQ, AK, BIAS, 128>(x, p.E_lo, p.E_hi, i, j0, 0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
+                                        imin(kBK, N - j0) - 1, ek0, ek1, bexp, sc);
       }
       const bool need_mask = (j0 + kBK > nkv) || (p.causal && j0 + kBK - 1 > q0 + g * kBQ);
       if (need_mask) {

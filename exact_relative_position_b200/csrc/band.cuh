@@ -15,22 +15,22 @@
 
 namespace relpos {
 
-// Row = query i (forward, Q-parallel backward).  x[c] holds the raw score of
-// key j0 + c and becomes (score + relation terms) * sc.
+// Row = query i (forward, Q-parallel backward).  x[c] (c < NC) holds the raw
+// score of key j0 + coff + c and becomes (score + relation terms) * sc.
 //   zq_row: Z^Q row of i, indexable by expanded column in [eq0, eq1]
-//   zk_tile: Z^K of key j0 + c at zk_tile[c * zS + e], e in [ek0, ek1], c <= kmax
-template <bool AQ, bool AK, bool BIAS>
-__device__ __forceinline__ void band_terms_q(float (&x)[128], int E_lo, int E_hi, int i, int j0, const float* zq_row,
-                                             int eq0, int eq1, const float* zk_tile, int zS, int kmax, int ek0,
-                                             int ek1, const float* bexp, float sc) {
+//   zk_tile: Z^K of the key tile's key t at zk_tile[t * zS + e], e in [ek0, ek1], t <= kmax
+template <bool AQ, bool AK, bool BIAS, int NC>
+__device__ __forceinline__ void band_terms_q(float (&x)[NC], int E_lo, int E_hi, int i, int j0, int coff,
+                                             const float* zq_row, int eq0, int eq1, const float* zk_tile, int zS,
+                                             int kmax, int ek0, int ek1, const float* bexp, float sc) {
 #pragma unroll
-  for (int c0 = 0; c0 < 128; c0 += 32) {
+  for (int c0 = 0; c0 < NC; c0 += 32) {
 #pragma unroll
     for (int c = c0; c < c0 + 32; ++c) {
-      const int e = iclamp(j0 + c - i, E_lo, E_hi) - E_lo;
+      const int e = iclamp(j0 + coff + c - i, E_lo, E_hi) - E_lo;
       float rel = 0.f;
       if (AQ) rel += __ldg(zq_row + iclamp(e, eq0, eq1));
-      if (AK) rel += __ldg(zk_tile + (long long)imin(c, kmax) * zS + iclamp(e, ek0, ek1));
+      if (AK) rel += __ldg(zk_tile + (long long)imin(coff + c, kmax) * zS + iclamp(e, ek0, ek1));
       if (BIAS) rel += __ldg(bexp + e);
       x[c] = (x[c] + rel) * sc;
     }
@@ -38,18 +38,18 @@ __device__ __forceinline__ void band_terms_q(float (&x)[128], int E_lo, int E_hi
   }
 }
 
-// Row = key j (K-parallel backward).  x[c] holds the raw score of query qb + c.
-template <bool AQ, bool AK, bool BIAS>
-__device__ __forceinline__ void band_terms_k(float (&x)[128], int E_lo, int E_hi, int j, int qb, const float* zk_row,
-                                             int ek0, int ek1, const float* zq_tile, int zS, int qmax, int eq0,
-                                             int eq1, const float* bexp, float sc) {
+// Row = key j (K-parallel backward).  x[c] holds the raw score of query qb + coff + c.
+template <bool AQ, bool AK, bool BIAS, int NC>
+__device__ __forceinline__ void band_terms_k(float (&x)[NC], int E_lo, int E_hi, int j, int qb, int coff,
+                                             const float* zk_row, int ek0, int ek1, const float* zq_tile, int zS,
+                                             int qmax, int eq0, int eq1, const float* bexp, float sc) {
 #pragma unroll
-  for (int c0 = 0; c0 < 128; c0 += 32) {
+  for (int c0 = 0; c0 < NC; c0 += 32) {
 #pragma unroll
     for (int c = c0; c < c0 + 32; ++c) {
-      const int e = iclamp(j - qb - c, E_lo, E_hi) - E_lo;
+      const int e = iclamp(j - qb - coff - c, E_lo, E_hi) - E_lo;
       float rel = 0.f;
-      if (AQ) rel += __ldg(zq_tile + (long long)imin(c, qmax) * zS + iclamp(e, eq0, eq1));
+      if (AQ) rel += __ldg(zq_tile + (long long)imin(coff + c, qmax) * zS + iclamp(e, eq0, eq1));
       if (AK) rel += __ldg(zk_row + iclamp(e, ek0, ek1));
       if (BIAS) rel += __ldg(bexp + e);
       x[c] = (x[c] + rel) * sc;
@@ -68,9 +68,9 @@ __device__ __forceinline__ void band_terms_k(float (&x)[128], int E_lo, int E_hi
 //   key_rows = false: row = query i = row0 + rr, column = key j = col0 + c, d = j - i
 //   key_rows = true:  row = key j = row0 + rr, column = query i = col0 + c, d = j - i
 //   dz_base + rr * S + (d - E_lo - e0) is the entry of (row, d)
-template <typename T>
+template <typename T, int NCOL>
 __device__ __forceinline__ void dz_band_store(uint32_t tile, int rbase, int lane, bool key_rows, int row0, int col0,
-                                              int nrows, int nkv, int N, int causal, int E_lo, int E_hi,
+                                              int cbeg, int nrows, int nkv, int N, int causal, int E_lo, int E_hi,
                                               float* dz_base, long long S, int e0, float tau) {
 #pragma unroll 1
   for (int rr = 0; rr < 32; ++rr) {
@@ -78,8 +78,8 @@ __device__ __forceinline__ void dz_band_store(uint32_t tile, int rbase, int lane
     if (row >= nrows) break;
     float* dz_row = dz_base + (long long)row * S - e0 - E_lo;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = lane + 32 * q;
+    for (int q = 0; q < NCOL / 32; ++q) {
+      const int c = cbeg + lane + 32 * q;
       const int col = col0 + c;
       const int i = key_rows ? col : row0 + row;
       const int j = key_rows ? row0 + row : col;
