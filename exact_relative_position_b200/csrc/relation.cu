@@ -160,16 +160,25 @@ __global__ void saturated_rows_kernel(const Plan p, const float* __restrict__ zq
 
 // ------------------------------------------------------------------ relgrad rows
 // out[rows of group g] = acc_in[rows] + dZ_g[rows, :W] A_exp[e0 .. e0 + W)   (tf32 tensor cores)
-constexpr int kRowPitchA = 36;   // floats, dZ chunk [128][32]
-constexpr int kRowPitchB = 72;   // floats, table chunk [32][64]
+// One CTA per (group, batch x head).  The reduction runs over the group's W
+// stored columns, streamed in chunks of 32 columns through a 3-stage cp.async
+// ring; warp w owns rows 16w .. 16w + 15 and all 64 output columns.
+namespace rg {
+constexpr int kKC = 32;        // columns of dZ (rows of the table) per chunk
+constexpr int kStages = 3;
+constexpr int kZP = 36;        // floats per row of a dZ chunk [128][32]: conflict-free fragment reads
+constexpr int kAP = 72;        // elements per row of a table chunk [32][64]
+template <typename T>
+constexpr uint32_t stage_bytes() { return 128u * kZP * 4u + (uint32_t)(kKC * kAP * sizeof(T)); }
+}  // namespace rg
 
 template <typename T>
 __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
                                                            const long long z_head, const T* __restrict__ A,
                                                            const long long a_hs, const float* __restrict__ acc_in,
                                                            T* __restrict__ out) {
-  __shared__ float As[128 * kRowPitchA];
-  __shared__ float Bs[32 * kRowPitchB];
+  extern __shared__ __align__(16) uint8_t rg_smem[];
+  constexpr uint32_t kSB = rg::stage_bytes<T>();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.x, bh = blockIdx.y, h = bh % p.H;
   const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
@@ -177,40 +186,66 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
   const int nrows = imin(kTile, p.N - r0);
   const float* Zg = dZ + (size_t)bh * z_head + gi.base;
   const T* Ah = A + (size_t)h * a_hs + (size_t)gi.e0 * 64;
-  const int g8 = lane >> 2, tq = lane & 3;
+  const int nk = (gi.W + rg::kKC - 1) / rg::kKC;
+  const uint32_t sbase = smem_u32(rg_smem);
+  auto load = [&](int kc) {
+    const uint32_t zs = sbase + (uint32_t)(kc % rg::kStages) * kSB;
+    const uint32_t as = zs + 128u * rg::kZP * 4u;
+    const int c0 = kc * rg::kKC;
+    // dZ: 128 rows x 8 pieces of 4 columns; a piece at or past the row stride
+    // S (a multiple of 4) or a row past the group is zero-filled.  Columns in
+    // [W, S) are stored zeros.
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = u * 256 + tid;
+      const int r = idx >> 3, pc = idx & 7;
+      const int col = c0 + 4 * pc;
+      const bool ok = r < nrows && col < gi.S;
+      cp_async16(zs + (uint32_t)(r * rg::kZP + 4 * pc) * 4u, ok ? Zg + (long long)r * gi.S + col : Zg, ok ? 16 : 0);
+    }
+    // table rows e0 + c0 .. + 31 (8 pieces of 8 elements each); rows past W are zero-filled
+    const int r = tid >> 3, pc = tid & 7;
+    const bool ok = c0 + r < gi.W;
+    cp_async16(as + (uint32_t)(r * rg::kAP + 8 * pc) * (uint32_t)sizeof(T), ok ? Ah + (size_t)(c0 + r) * 64 + 8 * pc : Ah,
+               ok ? 16 : 0);
+  };
+  const int g8 = lane >> 2, tq = lane & 3, rb = warp * 16;
   float acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  for (int c0 = 0; c0 < gi.W; c0 += 32) {
-    for (int idx = tid; idx < 128 * 32; idx += 256) {
-      const int r = idx >> 5, c = idx & 31;
-      As[r * kRowPitchA + c] = (r < nrows && c0 + c < gi.W) ? Zg[(long long)r * gi.S + c0 + c] : 0.f;
-    }
-    for (int idx = tid; idx < 32 * 64; idx += 256) {
-      const int r = idx >> 6, c = idx & 63;
-      Bs[r * kRowPitchB + c] = (c0 + r < gi.W) ? DT<T>::to_f(Ah[(size_t)(c0 + r) * 64 + c]) : 0.f;
-    }
-    __syncthreads();
+#pragma unroll
+  for (int s = 0; s < rg::kStages - 1; ++s) {
+    if (s < nk) load(s);
+    cp_async_commit();
+  }
+  for (int kc = 0; kc < nk; ++kc) {
+    cp_async_wait<rg::kStages - 2>();
+    __syncthreads();   // chunk kc visible to all; the stage of chunk kc - 1 is free again
+    if (kc + rg::kStages - 1 < nk) load(kc + rg::kStages - 1);
+    cp_async_commit();
+    const uint8_t* st = rg_smem + (uint32_t)(kc % rg::kStages) * kSB;
+    const float* Zs = reinterpret_cast<const float*>(st);
+    const T* As = reinterpret_cast<const T*>(st + 128u * rg::kZP * 4u);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      const int rb = warp * 16;
-      const uint32_t a0 = to_tf32(As[(rb + g8) * kRowPitchA + ks * 8 + tq]);
-      const uint32_t a1 = to_tf32(As[(rb + g8 + 8) * kRowPitchA + ks * 8 + tq]);
-      const uint32_t a2 = to_tf32(As[(rb + g8) * kRowPitchA + ks * 8 + tq + 4]);
-      const uint32_t a3 = to_tf32(As[(rb + g8 + 8) * kRowPitchA + ks * 8 + tq + 4]);
+      const uint32_t a0 = to_tf32(Zs[(rb + g8) * rg::kZP + ks * 8 + tq]);
+      const uint32_t a1 = to_tf32(Zs[(rb + g8 + 8) * rg::kZP + ks * 8 + tq]);
+      const uint32_t a2 = to_tf32(Zs[(rb + g8) * rg::kZP + ks * 8 + tq + 4]);
+      const uint32_t a3 = to_tf32(Zs[(rb + g8 + 8) * rg::kZP + ks * 8 + tq + 4]);
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        const uint32_t b0 = to_tf32(Bs[(ks * 8 + tq) * kRowPitchB + nt * 8 + g8]);
-        const uint32_t b1 = to_tf32(Bs[(ks * 8 + tq + 4) * kRowPitchB + nt * 8 + g8]);
+        // a 16-bit value is exact in tf32
+        const uint32_t b0 = __float_as_uint(DT<T>::to_f(As[(ks * 8 + tq) * rg::kAP + nt * 8 + g8]));
+        const uint32_t b1 = __float_as_uint(DT<T>::to_f(As[(ks * 8 + tq + 4) * rg::kAP + nt * 8 + g8]));
         mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
       }
     }
-    __syncthreads();
   }
+  cp_async_wait<0>();
   const size_t off = (size_t)bh * p.N * 64;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
-    const int rr = warp * 16 + g8 + 8 * hf;
+    const int rr = rb + g8 + 8 * hf;
     if (rr >= nrows) continue;
     const size_t ro = off + (size_t)(r0 + rr) * 64;
 #pragma unroll
@@ -225,25 +260,38 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
 // ------------------------------------------------------------------ table partials
 // part[s][hq][c0 + m][:] = sum over the split's (batch, head, group) items, in
 // order, of dZ_g[rows, c0 + m - e0] X[rows, :]   (tf32 tensor cores)
+// Block (e-block of 128 expanded rows, table, split).  The split's positions
+// are streamed in chunks of 32 rows of (dZ, X) through a 4-stage cp.async
+// ring that runs across item boundaries; items whose group stores none of the
+// block's columns are skipped.  Warp w owns expanded rows 16w .. 16w + 15.
+namespace tp {
+constexpr int kEB = 128;       // expanded rows per block
+constexpr int kRC = 32;        // positions per chunk
+constexpr int kStages = 4;
+constexpr int kZP = 136;       // floats per row of a dZ chunk [32][128]: conflict-free transposed fragment reads
+constexpr int kXP = 72;        // elements per row of an X chunk [32][64]
+template <typename T>
+constexpr uint32_t stage_bytes() { return (uint32_t)kRC * kZP * 4u + (uint32_t)(kRC * kXP * sizeof(T)); }
+}  // namespace tp
+
+struct ItemCursor {
+  long long it;   // current item
+  int rc;         // first row of the next chunk inside it
+};
+
 template <typename T>
 __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
                                                          const long long z_head, const T* __restrict__ X,
                                                          const int per_head, const int nsplit,
                                                          float* __restrict__ part) {
-  __shared__ float Zs[32 * kRowPitchB];   // [rows][e]
-  __shared__ float Xs[32 * kRowPitchB];   // [rows][d]
+  extern __shared__ __align__(16) uint8_t tp_smem[];
+  constexpr uint32_t kSB = tp::stage_bytes<T>();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c0 = blockIdx.x * 64, hq = blockIdx.y, s = blockIdx.z;
+  const int c0 = blockIdx.x * tp::kEB, hq = blockIdx.y, s = blockIdx.z;
   const int Hq = per_head ? p.H : 1;
   const long long nitems = per_head ? (long long)p.B * p.nT : (long long)p.B * p.H * p.nT;
   const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
-  const int g8 = lane >> 2, tq = lane & 3;
-  const int eb = (warp & 3) * 16, db = (warp >> 2) * 32;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  for (long long it = it0; it < it1; ++it) {
-    int bh, g;
+  auto item = [&](long long it, int& bh, int& g) {
     if (per_head) {
       const int b = (int)(it / p.nT);
       g = (int)(it - (long long)b * p.nT);
@@ -252,86 +300,185 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
       bh = (int)(it / p.nT);
       g = (int)(it - (long long)bh * p.nT);
     }
+  };
+  auto useful = [&](int g) {
     const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
-    if (c0 + 64 <= gi.e0 || c0 >= gi.e0 + gi.W) continue;   // block-uniform
+    return !(c0 + tp::kEB <= gi.e0 || c0 >= gi.e0 + gi.W);
+  };
+  // number of chunks of this split (block-uniform)
+  int nchunks = 0;
+  for (long long it = it0; it < it1; ++it) {
+    int bh, g;
+    item(it, bh, g);
+    if (useful(g)) nchunks += (imin(kTile, p.N - g * kTile) + tp::kRC - 1) / tp::kRC;
+  }
+  // load cursor: skips items that store none of the block's columns
+  ItemCursor cur{it0, 0};
+  auto skip = [&]() {
+    while (cur.it < it1) {
+      int bh, g;
+      item(cur.it, bh, g);
+      if (useful(g)) break;
+      ++cur.it;
+    }
+  };
+  skip();
+  const uint32_t sbase = smem_u32(tp_smem);
+  auto load = [&](int q) {
+    int bh, g;
+    item(cur.it, bh, g);
+    const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
     const int r0 = g * kTile, nrows = imin(kTile, p.N - r0);
     const float* Zg = dZ + (size_t)bh * z_head + gi.base;
-    const T* Xg = X + (size_t)bh * p.N * 64 + (size_t)r0 * 64;
-    for (int rc = 0; rc < nrows; rc += 32) {
-      for (int idx = tid; idx < 32 * 64; idx += 256) {
-        const int r = idx >> 6, c = idx & 63;
-        const int col = c0 + c - gi.e0;
-        const bool ok = (rc + r < nrows) && col >= 0 && col < gi.W;
-        Zs[r * kRowPitchB + c] = ok ? Zg[(long long)(rc + r) * gi.S + col] : 0.f;
-        Xs[r * kRowPitchB + c] = (rc + r < nrows) ? DT<T>::to_f(Xg[(size_t)(rc + r) * 64 + c]) : 0.f;
-      }
-      __syncthreads();
+    const T* Xg = X + ((size_t)bh * p.N + r0) * 64;
+    const uint32_t zs = sbase + (uint32_t)(q % tp::kStages) * kSB;
+    const uint32_t xs = zs + (uint32_t)tp::kRC * tp::kZP * 4u;
+    // dZ rows rc .. rc + 31, expanded columns c0 .. c0 + 127 (4-byte copies:
+    // the group's first column e0 has no alignment)
+#pragma unroll 4
+    for (int u = 0; u < tp::kRC * tp::kEB / 256; ++u) {
+      const int idx = u * 256 + tid;
+      const int r = idx >> 7, c = idx & 127;
+      const int lc = c0 + c - gi.e0;
+      const bool ok = cur.rc + r < nrows && lc >= 0 && lc < gi.W;
+      cp_async4(zs + (uint32_t)(r * tp::kZP + c) * 4u, ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg, ok ? 4 : 0);
+    }
+    {
+      const int r = tid >> 3, pc = tid & 7;
+      const bool ok = cur.rc + r < nrows;
+      cp_async16(xs + (uint32_t)(r * tp::kXP + 8 * pc) * (uint32_t)sizeof(T),
+                 ok ? Xg + (size_t)(cur.rc + r) * 64 + 8 * pc : Xg, ok ? 16 : 0);
+    }
+    cur.rc += tp::kRC;
+    if (cur.rc >= nrows) {
+      cur.rc = 0;
+      ++cur.it;
+      skip();
+    }
+  };
+  const int g8 = lane >> 2, tq = lane & 3, eb = warp * 16;
+  float acc[8][4];
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint32_t a0 = to_tf32(Zs[(ks * 8 + tq) * kRowPitchB + eb + g8]);
-        const uint32_t a1 = to_tf32(Zs[(ks * 8 + tq) * kRowPitchB + eb + g8 + 8]);
-        const uint32_t a2 = to_tf32(Zs[(ks * 8 + tq + 4) * kRowPitchB + eb + g8]);
-        const uint32_t a3 = to_tf32(Zs[(ks * 8 + tq + 4) * kRowPitchB + eb + g8 + 8]);
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          const uint32_t b0 = to_tf32(Xs[(ks * 8 + tq) * kRowPitchB + db + nt * 8 + g8]);
-          const uint32_t b1 = to_tf32(Xs[(ks * 8 + tq + 4) * kRowPitchB + db + nt * 8 + g8]);
-          mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
-        }
+  for (int q = 0; q < tp::kStages - 1; ++q) {
+    if (q < nchunks) load(q);
+    cp_async_commit();
+  }
+  for (int q = 0; q < nchunks; ++q) {
+    cp_async_wait<tp::kStages - 2>();
+    __syncthreads();   // chunk q visible to all; the stage of chunk q - 1 is free again
+    if (q + tp::kStages - 1 < nchunks) load(q + tp::kStages - 1);
+    cp_async_commit();
+    const uint8_t* st = tp_smem + (uint32_t)(q % tp::kStages) * kSB;
+    const float* Zs = reinterpret_cast<const float*>(st);
+    const T* Xs = reinterpret_cast<const T*>(st + (uint32_t)tp::kRC * tp::kZP * 4u);
+#pragma unroll
+    for (int ks = 0; ks < tp::kRC / 8; ++ks) {
+      // A = dZ^T: rows = expanded offsets, columns = positions
+      const uint32_t a0 = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + eb + g8]);
+      const uint32_t a1 = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + eb + g8 + 8]);
+      const uint32_t a2 = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + eb + g8]);
+      const uint32_t a3 = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + eb + g8 + 8]);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const uint32_t b0 = __float_as_uint(DT<T>::to_f(Xs[(ks * 8 + tq) * tp::kXP + nt * 8 + g8]));
+        const uint32_t b1 = __float_as_uint(DT<T>::to_f(Xs[(ks * 8 + tq + 4) * tp::kXP + nt * 8 + g8]));
+        mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
       }
-      __syncthreads();
     }
   }
+  cp_async_wait<0>();
   float* P = part + ((size_t)s * Hq + hq) * (size_t)p.Rexp * 64;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
     const int e = c0 + eb + g8 + 8 * hf;
     if (e >= p.Rexp) continue;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int d = db + nt * 8 + 2 * tq;
+    for (int nt = 0; nt < 8; ++nt) {
+      const int d = nt * 8 + 2 * tq;
       *reinterpret_cast<float2*>(P + (size_t)e * 64 + d) = make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
     }
   }
 }
 
-// db_part[s][h][e] = sum over the split's (batch, group) items of column e of dZ^Q.
+// db_part[s][h][e] = sum over the split's (batch, group) items of column e of
+// dZ^Q, for the block's 256 expanded columns.  Warp w takes the rows r = w
+// (mod 8) of every item, lane l the columns l + 32 k; the eight warp sums are
+// added in warp order at the end.
 __global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const float* __restrict__ dZ, const long long z_head,
                                                         const int nsplit, float* __restrict__ part) {
-  const int e = blockIdx.x * 256 + threadIdx.x, h = blockIdx.y, s = blockIdx.z;
+  __shared__ float red[8][256];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c0 = blockIdx.x * 256, h = blockIdx.y, s = blockIdx.z;
   const long long nitems = (long long)p.B * p.nT;
   const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
-  float acc = 0.f;
-  if (e < p.Rexp) {
-    for (long long it = it0; it < it1; ++it) {
-      const int b = (int)(it / p.nT), g = (int)(it - (long long)b * p.nT);
-      const GroupInfo gi = p.gq[g];
-      const int col = e - gi.e0;
-      if (col < 0 || col >= gi.W) continue;
-      const int nrows = imin(kTile, p.N - g * kTile);
-      const float* Zg = dZ + (size_t)(b * p.H + h) * z_head + gi.base + col;
-      for (int r = 0; r < nrows; ++r) acc += Zg[(long long)r * gi.S];
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  for (long long it = it0; it < it1; ++it) {
+    const int b = (int)(it / p.nT), g = (int)(it - (long long)b * p.nT);
+    const GroupInfo gi = p.gq[g];
+    if (c0 + 256 <= gi.e0 || c0 >= gi.e0 + gi.W) continue;   // block-uniform
+    const int nrows = imin(kTile, p.N - g * kTile);
+    const float* Zg = dZ + (size_t)(b * p.H + h) * z_head + gi.base;
+    int lc[8];
+    bool okc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      lc[k] = c0 + lane + 32 * k - gi.e0;
+      okc[k] = lc[k] >= 0 && lc[k] < gi.W;
+      if (!okc[k]) lc[k] = 0;
     }
-    part[((size_t)s * p.H + h) * p.Rexp + e] = acc;
+#pragma unroll 4
+    for (int r = warp; r < nrows; r += 8) {
+      const float* zr = Zg + (long long)r * gi.S;
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = okc[k] ? __ldg(zr + lc[k]) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] += v[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) red[warp][lane + 32 * k] = acc[k];
+  __syncthreads();
+  const int e = c0 + tid;
+  if (e < p.Rexp) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += red[w][tid];
+    part[((size_t)s * p.H + h) * p.Rexp + e] = sum;
   }
 }
 
-// out[hq][r][c] = sum_{e in fold range of r, ascending} sum_{s ascending} part[s][hq][e][c]
-__global__ void fold_kernel(const float* __restrict__ part, const int nsplit, const int Hq, const int Rexp, const int R,
-                            const int C, const int* __restrict__ fold_lo, const int* __restrict__ fold_hi,
-                            float* __restrict__ out) {
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)Hq * R * C) return;
-  const int c = (int)(idx % C);
-  const long long hr = idx / C;
-  const int r = (int)(hr % R), hq = (int)(hr / R);
+// out[hq][r][c] = sum over the pairs (e in the fold range of r, split s) of
+// part[s][hq][e][c].  One block per (r, hq); C is 64 (tables) or 1 (bias).
+// The 256 threads form 256 / C groups per column c; group k sums the pairs
+// k, k + 256 / C, ... (pairs ordered by e, then s) and the group sums are
+// added in group order, so the result does not depend on scheduling.
+__global__ void __launch_bounds__(256) fold_kernel(const float* __restrict__ part, const int nsplit, const int Hq,
+                                                   const int Rexp, const int R, const int C,
+                                                   const int* __restrict__ fold_lo, const int* __restrict__ fold_hi,
+                                                   float* __restrict__ out) {
+  __shared__ float red[256];
+  const int r = blockIdx.x, hq = blockIdx.y, tid = threadIdx.x;
+  const int G = 256 / C, c = tid % C, grp = tid / C;
+  const int lo = fold_lo[r];
+  const long long npairs = (long long)(fold_hi[r] - lo) * nsplit;
   float acc = 0.f;
-  for (int e = fold_lo[r]; e < fold_hi[r]; ++e) {
-    float se = 0.f;
-    for (int s = 0; s < nsplit; ++s) se += part[(((size_t)s * Hq + hq) * Rexp + e) * C + c];
-    acc += se;
+#pragma unroll 4
+  for (long long q = grp; q < npairs; q += G) {
+    const int e = lo + (int)(q / nsplit), sp = (int)(q % nsplit);
+    acc += part[(((size_t)sp * Hq + hq) * Rexp + e) * C + c];
   }
-  out[idx] = acc;
+  red[tid] = acc;
+  __syncthreads();
+  if (tid < C) {
+    float sum = 0.f;
+    for (int k = 0; k < G; ++k) sum += red[k * C + tid];
+    out[((size_t)hq * R + r) * C + tid] = sum;
+  }
 }
 
 // ------------------------------------------------------------------ debug
@@ -429,26 +576,32 @@ cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s) {
 template <typename T>
 static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   const int Hq = t.table_per_head ? p.H : 1;
-  const int nE = (p.Rexp + 63) / 64;
+  const int nE = (p.Rexp + tp::kEB - 1) / tp::kEB;
+  constexpr uint32_t kRowsSmem = rg::kStages * rg::stage_bytes<T>();
+  constexpr uint32_t kPartSmem = tp::kStages * tp::stage_bytes<T>();
+  cudaError_t e = cudaFuncSetAttribute(relgrad_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(table_part_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPartSmem);
+  if (e != cudaSuccess) return e;
   if (t.aq_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, 0, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
-                                                                t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
-    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, 0, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
-                                                                   t.table_per_head, t.nsplit_q, t.daq_part); note_launch(1); }
-    { fold_kernel<<<nblk((long long)Hq * t.R * 64, 256), 256, 0, s>>>(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64,
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
+                                                                        t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
+    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
+                                                                           t.table_per_head, t.nsplit_q, t.daq_part); note_launch(1); }
+    { fold_kernel<<<dim3(t.R, Hq), 256, 0, s>>>(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64,
                                                                      t.fold_lo, t.fold_hi, t.daq); note_launch(1); }
   }
   if (t.ak_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, 0, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
-                                                                t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
-    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, 0, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
-                                                                   t.table_per_head, t.nsplit_k, t.dak_part); note_launch(1); }
-    { fold_kernel<<<nblk((long long)Hq * t.R * 64, 256), 256, 0, s>>>(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64,
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
+                                                                        t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
+    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
+                                                                           t.table_per_head, t.nsplit_k, t.dak_part); note_launch(1); }
+    { fold_kernel<<<dim3(t.R, Hq), 256, 0, s>>>(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64,
                                                                      t.fold_lo, t.fold_hi, t.dak); note_launch(1); }
   }
   if (t.b_exp) {
     { bias_part_kernel<<<dim3((p.Rexp + 255) / 256, p.H, t.nsplit_b), 256, 0, s>>>(p, t.dzq, p.zq_head, t.nsplit_b, t.db_part); note_launch(1); }
-    { fold_kernel<<<nblk((long long)p.H * t.R, 256), 256, 0, s>>>(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1,
+    { fold_kernel<<<dim3(t.R, p.H), 256, 0, s>>>(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1,
                                                                  t.fold_lo, t.fold_hi, t.db); note_launch(1); }
   }
   return cudaGetLastError();
