@@ -41,9 +41,6 @@ constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // 16-bit [128 rows x 128 cols] K-major tile as two 64-column swizzle atoms:
 // address of the 16-byte chunk c (0..15) of row r.
@@ -102,8 +99,9 @@ constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 rows][2] saturated sums of column half 1
 constexpr uint32_t kSmemBytes = kOffSat + 1024 + 1024;
-// tensor memory: S buffers [0,128) and [128,256), dP [256,384), dQ [384,448)
-constexpr uint32_t kTmDP = 256, kTmDQ = 384;
+// tensor memory: S buffers [0,128) and [128,256), dP [256,384), dQ [384,448),
+// dS [448,512) (16-bit, two keys per column: the A operand of dQ += dS K)
+constexpr uint32_t kTmDP = 256, kTmDQ = 384, kTmDS = 448;
 // barriers
 constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kStages, kBarSFull = kBarKvEmpty + kStages,
               kBarSFree = kBarSFull + 2, kBarDpFull = kBarSFree + 2, kBarDpFree = kBarDpFull + 1,
@@ -203,8 +201,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         const uint64_t dk0 = sdesc_sw128(sb + kOffKV, 16, 1024);
         const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 16, 1024);
         const uint64_t dkmn0 = sdesc_sw128(sb + kOffKV, 8192, 1024);
-        const uint64_t dds0 = sdesc_sw128(sb + kOffDS, 16, 1024);
-        constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
+        constexpr uint64_t kStage16 = kStageBytes >> 4;
         auto issue_s = [&](int buf, int s) {
           const uint64_t kd = dk0 + (uint64_t)s * kStage16;
   #pragma unroll 1
@@ -219,8 +216,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           const uint64_t kd = dkmn0 + (uint64_t)s * kStage16;
   #pragma unroll 1
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + kTmDQ, dds0 + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), kd + 128 * kk, id_dq,
-                   (acc || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + kTmDQ, tmem + kTmDS + 8 * kk, kd + 128 * kk, id_dq, (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
         if (ok) {
@@ -407,18 +403,27 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
+      // this half's 64 keys of dS, two per tensor-memory column
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int c = 8 * ch;
-        st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), DT<T>::pack(x[c], x[c + 1]), DT<T>::pack(x[c + 2], x[c + 3]),
-                     DT<T>::pack(x[c + 4], x[c + 5]), DT<T>::pack(x[c + 6], x[c + 7]));
+        for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
+        tmem_st32(tmem + t_lane + kTmDS + 32 * hc, pk);
+        if (DZQ && !is_const) {
+          // BAND tile: the same 16-bit values also go to shared memory (rows
+          // of this warp only) for the coalesced by-offset store below
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        }
+        tmem_wait_st();
       }
       if (DZQ && !is_const) {
         __syncwarp();
         dz_band_store<T, 64>(dsb, (warp & 3) * 32, lane, false, q0, j0, cb, nrows_q, nkv, N, p.causal, p.E_lo,
                              p.E_hi, dzq_base, gi.S, gi.e0, p.tau);
       }
-      fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(bar(kBarDsReady));
     }
     // -------------------------------------------------------------- epilogue
@@ -496,19 +501,25 @@ constexpr uint32_t kStageBytes = 2 * kTileBytes + 2048;
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kTileBytes;
 constexpr uint32_t kOffQD = 2 * kTileBytes;
-constexpr uint32_t kOffP = kOffQD + kStages * kStageBytes;
-constexpr uint32_t kOffDS = kOffP + 2 * kTileBytes;
+constexpr uint32_t kOffDS = kOffQD + kStages * kStageBytes;   // dS^T of BAND tiles (relation-gradient stores)
 constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 keys][2] saturated sums of column half 1
 constexpr uint32_t kSmemBytes = kOffSat + 1024 + 1024;
-// tensor memory: S^T buffers [0,128), [128,256), dP^T [256,384), dV [384,448), dK [448,512)
+// tensor memory: S^T buffers [0,128), [128,256), dP^T [256,384), dV [384,448),
+// dK [448,512).  The 16-bit P^T of a tile overwrites its own S^T buffer and
+// dS^T overwrites dP^T: compute half hc (queries 64 hc .. 64 hc + 63) packs
+// its values two per column into columns 64 hc .. 64 hc + 31 of the buffer it
+// has just read, and those columns are the A operands of dV += P^T dO and
+// dK += dS^T Q.  The MMA issuer writes a buffer again only with a GEMM issued
+// after the one that reads it (tcgen05 ops of one thread run in order), and a
+// commit covers every earlier op, so the S / dP "full" barriers also mean
+// that the previous reader of the region is done.
 constexpr uint32_t kTmDP = 256, kTmDV = 384, kTmDK = 448;
 constexpr int kBarKV = 0, kBarQsFull = 1, kBarQsEmpty = kBarQsFull + kStages, kBarSFull = kBarQsEmpty + kStages,
-              kBarSFree = kBarSFull + 2, kBarDpFull = kBarSFree + 2, kBarDpFree = kBarDpFull + 1,
-              kBarPReady = kBarDpFree + 1, kBarPFree = kBarPReady + 1, kBarDsReady = kBarPFree + 1,
-              kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
+              kBarDpFull = kBarSFull + 2, kBarPReady = kBarDpFull + 1, kBarDsReady = kBarPReady + 1,
+              kBarDone = kBarDsReady + 1, kBarDrain = kBarDone + 1;
 }  // namespace kp
 
 template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32>
@@ -539,16 +550,11 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       mbar_init(bar(kBarQsFull + s), 1);
       mbar_init(bar(kBarQsEmpty + s), 1);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(bar(kBarSFull + u), 1);
-      mbar_init(bar(kBarSFree + u), 256);
-    }
+    for (int u = 0; u < 2; ++u) mbar_init(bar(kBarSFull + u), 1);
     mbar_init(bar(kBarDpFull), 1);
-    mbar_init(bar(kBarDpFree), 256);
     mbar_init(bar(kBarPReady), 256);
-    mbar_init(bar(kBarPFree), 1);
     mbar_init(bar(kBarDsReady), 256);
-    mbar_init(bar(kBarDsFree), 1);
+    mbar_init(bar(kBarDone), 1);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -609,9 +615,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         const uint64_t ddo0 = sdesc_sw128(sb + kOffQD + kTileBytes, 16, 1024);
         const uint64_t dqmn0 = sdesc_sw128(sb + kOffQD, 8192, 1024);
         const uint64_t ddomn0 = sdesc_sw128(sb + kOffQD + kTileBytes, 8192, 1024);
-        const uint64_t dp_ = sdesc_sw128(sb + kOffP, 16, 1024);
-        const uint64_t dds = sdesc_sw128(sb + kOffDS, 16, 1024);
-        constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
+        constexpr uint64_t kStage16 = kStageBytes >> 4;
         auto issue_s = [&](int buf, int s) {
           const uint64_t qd = dq0 + (uint64_t)s * kStage16;
   #pragma unroll 1
@@ -622,11 +626,12 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
   #pragma unroll 1
           for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, dv + 2 * kk, od + 2 * kk, id_s, kk > 0);
         };
-        // D[keys x 64] (+)= A[keys x queries] (shared) * B[queries x 64] (MN-major)
-        auto issue_g = [&](uint32_t d, uint64_t a, uint64_t bmn, bool acc) {
+        // D[keys x 64] (+)= A[keys x queries] (tensor memory, region a) * B[queries x 64] (MN-major);
+        // queries 16 kk .. 16 kk + 15 sit in columns 64 (kk / 4) + 8 (kk % 4) of the region
+        auto issue_g = [&](uint32_t d, uint32_t a, uint64_t bmn, bool acc) {
   #pragma unroll 1
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(d, a + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
+            mma_ts(d, a + 64 * (kk >> 2) + 8 * (kk & 3), bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = mbar_wait(bar(kBarKV), 0, abort_flag) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag);
         if (ok) {
@@ -644,31 +649,29 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
             }
           }
         }
+        // per tile t: dV(t) once P^T(t) is in its S^T buffer, dK(t) once dS^T(t)
+        // is in the dP^T region, then dP(t+1) over dS^T(t) and S(t+2) over P^T(t)
   #pragma unroll 1
         for (int it = 0; it < nq && ok; ++it) {
           const int s = it % kStages;
-          if (it + 1 < nq) {
-            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_dp((it + 1) % kStages);
-            mma_commit(bar(kBarDpFull));
-          }
           ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_g(tmem + kTmDV, dp_, ddomn0 + (uint64_t)s * kStage16, it > 0);
-          mma_commit(bar(kBarPFree));
+          issue_g(tmem + kTmDV, tmem + (uint32_t)(it & 1) * 128, ddomn0 + (uint64_t)s * kStage16, it > 0);
           ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_g(tmem + kTmDK, dds, dqmn0 + (uint64_t)s * kStage16, it > 0);
-          mma_commit(bar(kBarDsFree));
+          issue_g(tmem + kTmDK, tmem + kTmDP, dqmn0 + (uint64_t)s * kStage16, it > 0);
           mma_commit(bar(kBarQsEmpty + s));
+          if (it + 1 < nq) {
+            issue_dp((it + 1) % kStages);
+            mma_commit(bar(kBarDpFull));
+          } else {
+            mma_commit(bar(kBarDone));
+          }
           if (it + 2 < nq) {
             const int s2 = (it + 2) % kStages;
-            ok = mbar_wait(bar(kBarQsFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
-                 mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
+            ok = mbar_wait(bar(kBarQsFull + s2), ((it + 2) / kStages) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             issue_s(it & 1, s2);
@@ -707,7 +710,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     float* dzk_row = DZK ? dzk_base + (long long)krow * gk.S - gk.e0 : nullptr;
     const int nrows_k = imin(kT, N - k0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
-    const uint32_t pb = sb + kOffP, dsb = sb + kOffDS;
+    const uint32_t dsb = sb + kOffDS;
     float sat_lo = 0.f, sat_hi = 0.f;
     bool ok = true;
 #pragma unroll 1
@@ -732,8 +735,6 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
         tmem_wait_ld();
       }
-      tc_fence_before();
-      mbar_arrive(bar(kBarSFree + buf));
       // P^T = 2^(S^T tau log2e + relation terms - LSE_i log2e), column c = query qb + cb + c
       if (is_const) {
         const float rowk = cls == RELPOS_TILE_CONST_LO ? rowk_lo : rowk_hi;
@@ -778,18 +779,16 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           if (!jkeep || (p.causal && j > qb + cb + c)) x[c] = 0.f;
         }
       }
-      // P^T to shared memory: the A operand of dV += P^T dO
-      if (it > 0) {
-        const bool got = mbar_wait(bar(kBarPFree), (it - 1) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      }
+      // P^T, two queries per column, over the first half of this half's S^T
+      // columns: the A operand of dV += P^T dO
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int c = 8 * ch;
-        st_shared_v4(op_chunk(pb, r, 8 * hc + ch), DT<T>::pack(x[c], x[c + 1]), DT<T>::pack(x[c + 2], x[c + 3]),
-                     DT<T>::pack(x[c + 4], x[c + 5]), DT<T>::pack(x[c + 6], x[c + 7]));
+        for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
+        tmem_st32(tmem + t_lane + (uint32_t)buf * 128 + cb, pk);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(bar(kBarPReady));
       // dS^T = P^T (dP^T - D_i): the A operand of dK += dS^T Q, and the
       // key-side relation gradient of this key row
@@ -802,8 +801,6 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         tmem_ld32(td, dp);
         tmem_ld32(td + 32, dp + 32);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(kBarDpFree));
         if (!DZK || is_const) {
           float ssum[2] = {0.f, 0.f};
 #pragma unroll
@@ -845,22 +842,28 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           }
         }
       }
-      if (it > 0) {
-        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      }
+      // dS^T, two queries per column, over the first half of this half's dP^T
+      // columns: the A operand of dK += dS^T Q
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int c = 8 * ch;
-        st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), DT<T>::pack(x[c], x[c + 1]), DT<T>::pack(x[c + 2], x[c + 3]),
-                     DT<T>::pack(x[c + 4], x[c + 5]), DT<T>::pack(x[c + 6], x[c + 7]));
+        for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
+        tmem_st32(tmem + t_lane + kTmDP + cb, pk);
+        if (DZK && !is_const) {
+          // BAND tile: the same 16-bit values also go to shared memory (rows
+          // of this warp only) for the coalesced by-offset store below
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        }
+        tmem_wait_st();
       }
       if (DZK && !is_const) {
         __syncwarp();
         dz_band_store<T, 64>(dsb, (warp & 3) * 32, lane, true, k0, qb, cb, nrows_k, nkv, N, p.causal, p.E_lo,
                              p.E_hi, dzk_base, gk.S, gk.e0, p.tau);
       }
-      fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(bar(kBarDsReady));
     }
     // -------------------------------------------------------------- epilogue
@@ -887,7 +890,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     float dv[32], dk[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) dv[c] = dk[c] = 0.f;
-    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDsFree), (nq - 1) & 1, abort_flag);
+    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDone), 0, abort_flag);
     if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
       uint32_t u[32];

@@ -9,14 +9,16 @@
 //   warp 0       TMA producer: Q0/Q1 once, then K/V tiles (and the key
 //                tile's saturated relation columns) into a 3-stage ring
 //   warp 1       MMA issuer (one thread): S_g = Q_g K^T into tensor memory,
-//                O_g += P_g V with P_g from shared memory
+//                O_g += P_g V with P_g read from tensor memory
 //   warp 2       allocates / frees the tensor-memory columns
 //   warps 4..7   softmax of Q0 (thread r owns row r = TMEM lane r)
 //   warps 8..11  softmax of Q1
-// Tensor memory: S0 cols [0,128), S1 [128,256), O0 [256,320), O1 [320,384).
-// A softmax warpgroup releases S_g as soon as it has read it into registers,
-// so the GEMM of the next key tile runs while it computes; its 16-bit P_g
-// goes to a 128-byte-swizzled shared-memory tile that the PV GEMM reads.
+// Tensor memory: S0 cols [0,128), S1 [128,256), O0 [256,320), O1 [320,384),
+// P0 [384,448), P1 [448,512).  A softmax warpgroup releases S_g as soon as
+// it has read it into registers, so the GEMM of the next key tile runs while
+// it computes; its 16-bit P_g (two keys per column) goes back to tensor
+// memory, where the PV GEMM reads it as its A operand.  Shared memory then
+// only carries the operands TMA brings in.
 //
 // Relation terms are added to the scores in registers.  A key tile whose
 // every offset saturates (CONST_LO / CONST_HI: two comparisons of the tile's
@@ -50,10 +52,7 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kColvBytes = 2 * kBK * 4;
 constexpr uint32_t kStageBytes = 2 * kTileBytes + 1024;   // keeps every K/V tile 1024-byte aligned
 constexpr uint32_t kOffKV = 2 * kTileBytes;
-// P_g: [128 rows x 128 keys] 16-bit, two 64-key swizzle atoms of 16 KB
-constexpr uint32_t kOffP = kOffKV + kStages * kStageBytes;
-constexpr uint32_t kPBytes = 2 * kTileBytes;
-constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
+constexpr uint32_t kOffBar = kOffKV + kStages * kStageBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kSmemBytes = kOffTmem + 16 + 1024;   // + alignment slack
@@ -66,7 +65,7 @@ constexpr int kBarKvFull = 1;
 constexpr int kBarKvEmpty = kBarKvFull + kStages;
 constexpr int kBarSFull = kBarKvEmpty + kStages;   // 2: S_g written (MMA commit)
 constexpr int kBarSFree = kBarSFull + 2;           // 2: S_g read into registers (128 arrivals)
-constexpr int kBarPReady = kBarSFree + 2;          // 2: P_g written to shared memory (128 arrivals)
+constexpr int kBarPReady = kBarSFree + 2;          // 2: P_g written to tensor memory (128 arrivals)
 constexpr int kBarPFree = kBarPReady + 2;          // 2: PV_g done: P_g buffer and O_g free (MMA commit)
 constexpr int kBarDrain = kBarPFree + 2;
 
@@ -76,12 +75,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 template <typename OutT> struct RowStore;
 template <> struct RowStore<float> {
@@ -189,8 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq0 = sdesc_sw128(sb + kOffQ, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(sb + kOffKV, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 8192, 1024);
-      const uint64_t dp0 = sdesc_sw128(sb + kOffP, 16, 1024);
-      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4, kP16 = kPBytes >> 4;
+      constexpr uint64_t kTile16 = kTileBytes >> 4, kStage16 = kStageBytes >> 4;
       auto issue_qk = [&](int g, int s) {
         const uint64_t a = dq0 + (uint64_t)g * kTile16;
         const uint64_t k = dk0 + (uint64_t)s * kStage16;
@@ -198,13 +190,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int kk = 0; kk < 4; ++kk) mma_ss(d, a + 2 * kk, k + 2 * kk, id_qk, kk > 0);
       };
+      // keys 16 kk .. 16 kk + 15 of P_g are its columns 8 kk .. 8 kk + 7
       auto issue_pv = [&](int g, int s, bool acc) {
         const uint64_t v = dv0 + (uint64_t)s * kStage16;
-        const uint64_t pp = dp0 + (uint64_t)g * kP16;
+        const uint32_t pt = tmem + 384 + (uint32_t)g * 64;
         const uint32_t d = tmem + 256 + (uint32_t)g * 64;
 #pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(d, pp + (uint64_t)(kk >> 2) * kTile16 + 2 * (kk & 3), v + 128 * kk, id_pv, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(d, pt + 8 * kk, v + 128 * kk, id_pv, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
       if (ok) {
@@ -257,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = (uint32_t)(wl * 32) << 16;
     const uint32_t tS = tmem + t_lane + (uint32_t)g * 128;
     const uint32_t tO = tmem + t_lane + 256 + (uint32_t)g * 64;
-    const uint32_t pbase = sb + kOffP + (uint32_t)g * kPBytes + (uint32_t)r * 128;
+    const uint32_t tP = tmem + t_lane + 384 + (uint32_t)g * 64;
     const float sc = p.tau * kLog2e;
     // projection group of this query tile (the last one for a tile past N,
     // whose rows are all discarded); rows past N read row 0 (in bounds)
@@ -385,28 +377,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
-      // p = 2^(x * xs + rowc - m_run), streamed 8 keys at a time into row r of
-      // P (16-byte chunks of two 64-key swizzle atoms)
+      // p = 2^(x * xs + rowc - m_run), 64 keys at a time packed two per
+      // column into row r of P_g in tensor memory
       const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float e8[8];
+      for (int hk = 0; hk < 2; ++hk) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) e8[u] = fast_exp2(fmaf(x[8 * c + u], xs, -msub));
-        uint32_t pk[4];
+        for (int c = 0; c < 8; ++c) {
+          float e8[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          pk[u] = DT<T>::pack(e8[2 * u], e8[2 * u + 1]);
-          // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
-          // enough to sum the fp32 values and spare the conversions
-          ps[u] += DT<T>::kCoarse ? DT<T>::pair_sum(pk[u]) : e8[2 * u] + e8[2 * u + 1];
+          for (int u = 0; u < 8; ++u) e8[u] = fast_exp2(fmaf(x[64 * hk + 8 * c + u], xs, -msub));
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            pk[4 * c + u] = DT<T>::pack(e8[2 * u], e8[2 * u + 1]);
+            // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
+            // enough to sum the fp32 values and spare the conversions
+            ps[u] += DT<T>::kCoarse ? DT<T>::pair_sum(pk[4 * c + u]) : e8[2 * u] + e8[2 * u + 1];
+          }
         }
-        const uint32_t addr = pbase + (uint32_t)(c >> 3) * kTileBytes + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-        st_shared_v4(addr, pk[0], pk[1], pk[2], pk[3]);
+        tmem_st32(tP + 32 * hk, pk);
       }
       l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(bar(kBarPReady + g));
     }
     // ------------------------------------------------------------ epilogue
