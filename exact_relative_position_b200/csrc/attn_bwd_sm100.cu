@@ -42,11 +42,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// 16-bit [128 rows x 128 cols] K-major tile as two 64-column swizzle atoms:
-// address of the 16-byte chunk c (0..15) of row r.
-__device__ __forceinline__ uint32_t op_chunk(uint32_t base, int r, int c) {
-  return base + (uint32_t)(c >> 3) * kTileBytes + (uint32_t)r * 128 + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-}
 
 // ------------------------------------------------------------------ prep
 // dsum[bh][i] = sum_c dO_ic O_ic and lse2[bh][i] = LSE_i log2 e for i < N;
@@ -93,8 +88,9 @@ constexpr uint32_t kStageBytes = 2 * kTileBytes + 1024;   // K, V, saturated key
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffDO = kTileBytes;
 constexpr uint32_t kOffKV = 2 * kTileBytes;
-constexpr uint32_t kOffDS = kOffKV + kStages * kStageBytes;
-constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
+// warp-private staging areas of BAND tiles: 16-bit dS rows for the by-offset store
+constexpr uint32_t kOffStage = kOffKV + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffStage + 8 * kStageWarpBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 rows][2] saturated sums of column half 1
@@ -289,12 +285,12 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     // projection group of this query tile; rows past N use row 0 (in bounds)
     const GroupInfo gi = p.gq[qt];
     const int rrow = rok ? r : 0;
-    const float* zq_row = AQ ? t.zq + (size_t)bh * p.zq_head + gi.base + (long long)rrow * gi.S - gi.e0 : nullptr;
     float* dzq_base = DZQ ? t.dzq + (size_t)bh * p.zq_head + gi.base : nullptr;
     float* dzq_row = DZQ ? dzq_base + (long long)rrow * gi.S - gi.e0 : nullptr;
     const int nrows_q = imin(kT, N - q0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
-    const uint32_t dsb = sb + kOffDS;
+    T* stg = reinterpret_cast<T*>(sg + kOffStage + (uint32_t)(warp - 4) * kStageWarpBytes);
+    const float* zq_row = AQ ? t.zq + (size_t)bh * p.zq_head + gi.base + (long long)rrow * gi.S - gi.e0 : nullptr;
     float sat_lo = 0.f, sat_hi = 0.f;
     bool ok = true;
 #pragma unroll 1
@@ -410,18 +406,19 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
         tmem_st32(tmem + t_lane + kTmDS + 32 * hc, pk);
         if (DZQ && !is_const) {
-          // BAND tile: the same 16-bit values also go to shared memory (rows
-          // of this warp only) for the coalesced by-offset store below
+          // BAND tile: the same 16-bit values also go to the warp's staging
+          // area (its own rows) for the coalesced by-offset store below
+          __syncwarp();
+          const uint32_t row16 = smem_u32(stg) + (uint32_t)(lane * kDsPitch) * 2u;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          for (int ch = 0; ch < 8; ++ch) st_shared_v4(row16 + 16u * ch, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
         tmem_wait_st();
       }
       if (DZQ && !is_const) {
         __syncwarp();
-        dz_band_store<T, 64>(dsb, (warp & 3) * 32, lane, false, q0, j0, cb, nrows_q, nkv, N, p.causal, p.E_lo,
-                             p.E_hi, dzq_base, gi.S, gi.e0, p.tau);
+        dz_band_store<T>(stg, (warp & 3) * 32, lane, false, q0, j0, cb, nrows_q, nkv, N,
+                         p.causal, p.E_lo, p.E_hi, dzq_base, gi.S, gi.e0, p.tau);
       }
       tc_fence_before();
       mbar_arrive(bar(kBarDsReady));
@@ -501,25 +498,25 @@ constexpr uint32_t kStageBytes = 2 * kTileBytes + 2048;
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kTileBytes;
 constexpr uint32_t kOffQD = 2 * kTileBytes;
-constexpr uint32_t kOffDS = kOffQD + kStages * kStageBytes;   // dS^T of BAND tiles (relation-gradient stores)
-constexpr uint32_t kOffBar = kOffDS + 2 * kTileBytes;
+// warp-private staging areas of BAND tiles: 16-bit dS^T rows for the by-offset store
+constexpr uint32_t kOffStage = kOffQD + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffStage + 8 * kStageWarpBytes;
 constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 keys][2] saturated sums of column half 1
 constexpr uint32_t kSmemBytes = kOffSat + 1024 + 1024;
-// tensor memory: S^T buffers [0,128), [128,256), dP^T [256,384), dV [384,448),
-// dK [448,512).  The 16-bit P^T of a tile overwrites its own S^T buffer and
-// dS^T overwrites dP^T: compute half hc (queries 64 hc .. 64 hc + 63) packs
-// its values two per column into columns 64 hc .. 64 hc + 31 of the buffer it
-// has just read, and those columns are the A operands of dV += P^T dO and
-// dK += dS^T Q.  The MMA issuer writes a buffer again only with a GEMM issued
-// after the one that reads it (tcgen05 ops of one thread run in order), and a
-// commit covers every earlier op, so the S / dP "full" barriers also mean
-// that the previous reader of the region is done.
-constexpr uint32_t kTmDP = 256, kTmDV = 384, kTmDK = 448;
+// tensor memory: S^T [0,128), P^T [128,192), dS^T [192,256), dP^T [256,384),
+// dV [384,448), dK [448,512).  P^T and dS^T are 16-bit, two queries per
+// column; compute half hc (queries 64 hc .. 64 hc + 63) owns columns
+// 32 hc .. 32 hc + 31 of each.  They are the A operands of dV += P^T dO and
+// dK += dS^T Q.  Every region a GEMM reads is rewritten only after a commit
+// that follows that GEMM (PFree, DsFree), and every region the compute warps
+// read is rewritten by a GEMM only after their arrival (SFree, DpFree).
+constexpr uint32_t kTmP = 128, kTmDS = 192, kTmDP = 256, kTmDV = 384, kTmDK = 448;
 constexpr int kBarKV = 0, kBarQsFull = 1, kBarQsEmpty = kBarQsFull + kStages, kBarSFull = kBarQsEmpty + kStages,
-              kBarDpFull = kBarSFull + 2, kBarPReady = kBarDpFull + 1, kBarDsReady = kBarPReady + 1,
-              kBarDone = kBarDsReady + 1, kBarDrain = kBarDone + 1;
+              kBarSFree = kBarSFull + 1, kBarDpFull = kBarSFree + 1, kBarDpFree = kBarDpFull + 1,
+              kBarPReady = kBarDpFree + 1, kBarPFree = kBarPReady + 1, kBarDsReady = kBarPFree + 1,
+              kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
 }  // namespace kp
 
 template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32>
@@ -550,11 +547,14 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       mbar_init(bar(kBarQsFull + s), 1);
       mbar_init(bar(kBarQsEmpty + s), 1);
     }
-    for (int u = 0; u < 2; ++u) mbar_init(bar(kBarSFull + u), 1);
+    mbar_init(bar(kBarSFull), 1);
+    mbar_init(bar(kBarSFree), 256);
     mbar_init(bar(kBarDpFull), 1);
+    mbar_init(bar(kBarDpFree), 256);
     mbar_init(bar(kBarPReady), 256);
+    mbar_init(bar(kBarPFree), 1);
     mbar_init(bar(kBarDsReady), 256);
-    mbar_init(bar(kBarDone), 1);
+    mbar_init(bar(kBarDsFree), 1);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -616,67 +616,61 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         const uint64_t dqmn0 = sdesc_sw128(sb + kOffQD, 8192, 1024);
         const uint64_t ddomn0 = sdesc_sw128(sb + kOffQD + kTileBytes, 8192, 1024);
         constexpr uint64_t kStage16 = kStageBytes >> 4;
-        auto issue_s = [&](int buf, int s) {
+        auto issue_s = [&](int s) {
           const uint64_t qd = dq0 + (uint64_t)s * kStage16;
   #pragma unroll 1
-          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dk + 2 * kk, qd + 2 * kk, id_s, kk > 0);
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem, dk + 2 * kk, qd + 2 * kk, id_s, kk > 0);
         };
         auto issue_dp = [&](int s) {
           const uint64_t od = ddo0 + (uint64_t)s * kStage16;
   #pragma unroll 1
           for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, dv + 2 * kk, od + 2 * kk, id_s, kk > 0);
         };
-        // D[keys x 64] (+)= A[keys x queries] (tensor memory, region a) * B[queries x 64] (MN-major);
-        // queries 16 kk .. 16 kk + 15 sit in columns 64 (kk / 4) + 8 (kk % 4) of the region
+        // D[keys x 64] (+)= A[keys x queries] (tensor memory at a, queries
+        // 16 kk .. 16 kk + 15 in columns 8 kk .. 8 kk + 7) * B[queries x 64] (MN-major)
         auto issue_g = [&](uint32_t d, uint32_t a, uint64_t bmn, bool acc) {
   #pragma unroll 1
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(d, a + 64 * (kk >> 2) + 8 * (kk & 3), bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) mma_ts(d, a + 8 * kk, bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = mbar_wait(bar(kBarKV), 0, abort_flag) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag);
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0);
-          mma_commit(bar(kBarSFull + 0));
+          issue_s(0);
+          mma_commit(bar(kBarSFull));
           issue_dp(0);
           mma_commit(bar(kBarDpFull));
-          if (nq > 1) {
-            ok = mbar_wait(bar(kBarQsFull + 1), 0, abort_flag);
-            if (ok) {
-              tc_fence_after();
-              issue_s(1, 1);
-              mma_commit(bar(kBarSFull + 1));
-            }
-          }
         }
-        // per tile t: dV(t) once P^T(t) is in its S^T buffer, dK(t) once dS^T(t)
-        // is in the dP^T region, then dP(t+1) over dS^T(t) and S(t+2) over P^T(t)
+        // per tile t: S(t+1) once S(t) has been read, dV(t) once P^T(t) is
+        // written, dP(t+1) once dP(t) has been read, dK(t) once dS^T(t) is written
   #pragma unroll 1
         for (int it = 0; it < nq && ok; ++it) {
-          const int s = it % kStages;
+          const int s = it % kStages, s1 = (it + 1) % kStages;
+          if (it + 1 < nq) {
+            ok = mbar_wait(bar(kBarQsFull + s1), ((it + 1) / kStages) & 1, abort_flag) &&
+                 mbar_wait(bar(kBarSFree), it & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(s1);
+            mma_commit(bar(kBarSFull));
+          }
           ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_g(tmem + kTmDV, tmem + (uint32_t)(it & 1) * 128, ddomn0 + (uint64_t)s * kStage16, it > 0);
+          issue_g(tmem + kTmDV, tmem + kTmP, ddomn0 + (uint64_t)s * kStage16, it > 0);
+          mma_commit(bar(kBarPFree));
+          if (it + 1 < nq) {
+            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp(s1);
+            mma_commit(bar(kBarDpFull));
+          }
           ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_g(tmem + kTmDK, tmem + kTmDP, dqmn0 + (uint64_t)s * kStage16, it > 0);
+          issue_g(tmem + kTmDK, tmem + kTmDS, dqmn0 + (uint64_t)s * kStage16, it > 0);
+          mma_commit(bar(kBarDsFree));
           mma_commit(bar(kBarQsEmpty + s));
-          if (it + 1 < nq) {
-            issue_dp((it + 1) % kStages);
-            mma_commit(bar(kBarDpFull));
-          } else {
-            mma_commit(bar(kBarDone));
-          }
-          if (it + 2 < nq) {
-            const int s2 = (it + 2) % kStages;
-            ok = mbar_wait(bar(kBarQsFull + s2), ((it + 2) / kStages) & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(it & 1, s2);
-            mma_commit(bar(kBarSFull + (it & 1)));
-          }
         }
         if (!ok) {
           mma_commit(bar(kBarDrain));
@@ -705,12 +699,12 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     // projection group of this key tile; keys past N use row 0 (in bounds)
     const GroupInfo gk = p.gk[kt];
     const int krow = jok ? r : 0;
-    const float* zk_row = AK ? t.zk + (size_t)bh * p.zk_head + gk.base + (long long)krow * gk.S - gk.e0 : nullptr;
     float* dzk_base = DZK ? t.dzk + (size_t)bh * p.zk_head + gk.base : nullptr;
     float* dzk_row = DZK ? dzk_base + (long long)krow * gk.S - gk.e0 : nullptr;
     const int nrows_k = imin(kT, N - k0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
-    const uint32_t dsb = sb + kOffDS;
+    T* stg = reinterpret_cast<T*>(sg + kOffStage + (uint32_t)(warp - 4) * kStageWarpBytes);
+    const float* zk_row = AK ? t.zk + (size_t)bh * p.zk_head + gk.base + (long long)krow * gk.S - gk.e0 : nullptr;
     float sat_lo = 0.f, sat_hi = 0.f;
     bool ok = true;
 #pragma unroll 1
@@ -718,23 +712,25 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       const int qi = qt0 + it, qb = qi * kT;
       const int cls = tile_class(qi, kt, N, nkv, p.causal, p.E_lo, p.E_hi);
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
-      const int stage = it % kStages, buf = it & 1;
+      const int stage = it % kStages;
       const float* vec = reinterpret_cast<const float*>(sg + kOffQD + (uint32_t)stage * kStageBytes + 2 * kTileBytes);
       const float* lse2v = vec + cb;
       const float* dvec = vec + kT + cb;
       const float* cvq = vec + (cls == RELPOS_TILE_CONST_LO ? 2 * kT : 3 * kT) + cb;
       // the stage's own barrier makes its TMA-written vectors visible to these threads
-      const bool got_s = mbar_wait(bar(kBarSFull + buf), (it >> 1) & 1, abort_flag) &&
+      const bool got_s = mbar_wait(bar(kBarSFull), it & 1, abort_flag) &&
                          mbar_wait(bar(kBarQsFull + stage), (it / kStages) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       float x[64];
       {
-        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128 + cb;
+        const uint32_t ts = tmem + t_lane + cb;
         tmem_ld32(ts + 0, reinterpret_cast<uint32_t*>(x) + 0);
         tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
         tmem_wait_ld();
       }
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree));   // S(t + 1) may now be written
       // P^T = 2^(S^T tau log2e + relation terms - LSE_i log2e), column c = query qb + cb + c
       if (is_const) {
         const float rowk = cls == RELPOS_TILE_CONST_LO ? rowk_lo : rowk_hi;
@@ -779,13 +775,17 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           if (!jkeep || (p.causal && j > qb + cb + c)) x[c] = 0.f;
         }
       }
-      // P^T, two queries per column, over the first half of this half's S^T
-      // columns: the A operand of dV += P^T dO
+      // P^T, two queries per column, once dV(t - 1) has read P^T(t - 1)
+      if (it > 0) {
+        const bool got = mbar_wait(bar(kBarPFree), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+      }
       {
         uint32_t pk[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
-        tmem_st32(tmem + t_lane + (uint32_t)buf * 128 + cb, pk);
+        tmem_st32(tmem + t_lane + kTmP + 32 * hc, pk);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -801,6 +801,8 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         tmem_ld32(td, dp);
         tmem_ld32(td + 32, dp + 32);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(kBarDpFree));   // dP(t + 1) may now be written
         if (!DZK || is_const) {
           float ssum[2] = {0.f, 0.f};
 #pragma unroll
@@ -842,26 +844,31 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           }
         }
       }
-      // dS^T, two queries per column, over the first half of this half's dP^T
-      // columns: the A operand of dK += dS^T Q
+      // dS^T, two queries per column, once dK(t - 1) has read dS^T(t - 1)
+      if (it > 0) {
+        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+      }
       {
         uint32_t pk[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
-        tmem_st32(tmem + t_lane + kTmDP + cb, pk);
+        tmem_st32(tmem + t_lane + kTmDS + 32 * hc, pk);
         if (DZK && !is_const) {
-          // BAND tile: the same 16-bit values also go to shared memory (rows
-          // of this warp only) for the coalesced by-offset store below
+          // BAND tile: the same 16-bit values also go to the warp's staging
+          // area (its own rows) for the coalesced by-offset store below
+          __syncwarp();
+          const uint32_t row16 = smem_u32(stg) + (uint32_t)(lane * kDsPitch) * 2u;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            st_shared_v4(op_chunk(dsb, r, 8 * hc + ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          for (int ch = 0; ch < 8; ++ch) st_shared_v4(row16 + 16u * ch, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
         tmem_wait_st();
       }
       if (DZK && !is_const) {
         __syncwarp();
-        dz_band_store<T, 64>(dsb, (warp & 3) * 32, lane, true, k0, qb, cb, nrows_k, nkv, N, p.causal, p.E_lo,
-                             p.E_hi, dzk_base, gk.S, gk.e0, p.tau);
+        dz_band_store<T>(stg, (warp & 3) * 32, lane, true, k0, qb, cb, nrows_k, nkv, N,
+                         p.causal, p.E_lo, p.E_hi, dzk_base, gk.S, gk.e0, p.tau);
       }
       tc_fence_before();
       mbar_arrive(bar(kBarDsReady));
@@ -890,7 +897,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     float dv[32], dk[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) dv[c] = dk[c] = 0.f;
-    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDone), 0, abort_flag);
+    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDsFree), (nq - 1) & 1, abort_flag);
     if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
       uint32_t u[32];

@@ -5,22 +5,29 @@
 //
 // A BAND tile straddles the diagonal band of interior offsets, so its scores
 // need one scalar per cell: Z^Q[i, e], Z^K[j, e] and b[e] with
-// e = clamp(j - i, E_lo, E_hi) - E_lo.  The gathers are branch-free: every
-// index is clamped into the stored columns (and rows) of its projection group,
-// so a masked cell reads a harmless in-bounds value that the caller's mask
-// overwrites, and the code stays small enough for the instruction cache.
+// e = clamp(j - i, E_lo, E_hi) - E_lo.
+//
+// The gathers are branch-free: every index is clamped into the stored
+// columns (and rows) of its projection group, so a masked cell reads a
+// harmless in-bounds value that the caller's mask overwrites, and the code
+// stays small enough for the instruction cache.
 #pragma once
 
 #include "common.cuh"
 
 namespace relpos {
 
+// Bytes of one warp's staging area: the 16-bit dS rows of the by-offset
+// store (32 rows x 64 columns, kDsPitch elements per row).
+constexpr int kDsPitch = 72;
+constexpr uint32_t kStageWarpBytes = 32u * kDsPitch * 2u;
+
 // Row = query i (forward, Q-parallel backward).  x[c] (c < NC) holds the raw
 // score of key j0 + coff + c and becomes (score + relation terms) * sc.
 //   zq_row: Z^Q row of i, indexable by expanded column in [eq0, eq1]
 //   zk_tile: Z^K of the key tile's key t at zk_tile[t * zS + e], e in [ek0, ek1], t <= kmax
 template <bool AQ, bool AK, bool BIAS, int NC>
-__device__ __forceinline__ void band_terms_q(float (&x)[NC], int E_lo, int E_hi, int i, int j0, int coff,
+__device__ __forceinline__ void band_terms_q(float* x, int E_lo, int E_hi, int i, int j0, int coff,
                                              const float* zq_row, int eq0, int eq1, const float* zk_tile, int zS,
                                              int kmax, int ek0, int ek1, const float* bexp, float sc) {
 #pragma unroll
@@ -40,7 +47,7 @@ __device__ __forceinline__ void band_terms_q(float (&x)[NC], int E_lo, int E_hi,
 
 // Row = key j (K-parallel backward).  x[c] holds the raw score of query qb + coff + c.
 template <bool AQ, bool AK, bool BIAS, int NC>
-__device__ __forceinline__ void band_terms_k(float (&x)[NC], int E_lo, int E_hi, int j, int qb, int coff,
+__device__ __forceinline__ void band_terms_k(float* x, int E_lo, int E_hi, int j, int qb, int coff,
                                              const float* zk_row, int ek0, int ek1, const float* zq_tile, int zS,
                                              int qmax, int eq0, int eq1, const float* bexp, float sc) {
 #pragma unroll
@@ -59,41 +66,32 @@ __device__ __forceinline__ void band_terms_k(float (&x)[NC], int E_lo, int E_hi,
 }
 
 // Interior relation-gradient entries of one BAND tile, stored by offset from
-// the 16-bit dS tile in shared memory (two 64-column 128-byte-swizzle atoms,
-// rows = this side's positions, columns = the other side's).  Warp-cooperative
-// and coalesced: the warp walks its 32 rows one by one and its lanes cover the
-// 128 columns, whose offsets are consecutive.  Interior offsets E_lo < d < E_hi
-// have exactly one cell per (row, offset), so every entry has one writer; the
-// two saturated offsets are summed by the caller.
-//   key_rows = false: row = query i = row0 + rr, column = key j = col0 + c, d = j - i
-//   key_rows = true:  row = key j = row0 + rr, column = query i = col0 + c, d = j - i
-//   dz_base + rr * S + (d - E_lo - e0) is the entry of (row, d)
-template <typename T, int NCOL>
-__device__ __forceinline__ void dz_band_store(uint32_t tile, int rbase, int lane, bool key_rows, int row0, int col0,
+// the warp's 16-bit dS rows (rows = this side's positions, 64 columns = the
+// other side's).  Warp-cooperative and coalesced: the warp walks its 32 rows
+// and its lanes cover the columns, whose offsets are consecutive.  Interior
+// offsets E_lo < d < E_hi have exactly one cell per (row, offset), so every
+// entry has one writer; the two saturated offsets are summed by the caller.
+//   key_rows = false: row = query i = row0 + rbase + rr, column = key j = col0 + cbeg + c, d = j - i
+//   key_rows = true:  row = key j = row0 + rbase + rr, column = query i = col0 + cbeg + c, d = j - i
+//   dz_base + (rbase + rr) * S + (d - E_lo - e0) is the entry of (row, d)
+template <typename T>
+__device__ __forceinline__ void dz_band_store(const T* stage16, int rbase, int lane, bool key_rows, int row0, int col0,
                                               int cbeg, int nrows, int nkv, int N, int causal, int E_lo, int E_hi,
                                               float* dz_base, long long S, int e0, float tau) {
-#pragma unroll 1
+#pragma unroll 4
   for (int rr = 0; rr < 32; ++rr) {
     const int row = rbase + rr;
     if (row >= nrows) break;
     float* dz_row = dz_base + (long long)row * S - e0 - E_lo;
 #pragma unroll
-    for (int q = 0; q < NCOL / 32; ++q) {
-      const int c = cbeg + lane + 32 * q;
-      const int col = col0 + c;
+    for (int q = 0; q < 2; ++q) {
+      const int c = lane + 32 * q;
+      const int col = col0 + cbeg + c;
       const int i = key_rows ? col : row0 + row;
       const int j = key_rows ? row0 + row : col;
       const int d = j - i;
       const bool kept = i < N && j < nkv && !(causal && j > i) && d > E_lo && d < E_hi;
-      if (kept) {
-        const uint32_t addr = tile + (uint32_t)(c >> 6) * 16384u + (uint32_t)row * 128u +
-                              ((uint32_t)(((c >> 3) & 7) ^ (row & 7)) << 4) + (uint32_t)(c & 7) * 2u;
-        unsigned short h;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(addr));
-        T v;
-        *reinterpret_cast<unsigned short*>(&v) = h;
-        dz_row[d] = tau * DT<T>::to_f(v);
-      }
+      if (kept) dz_row[d] = tau * DT<T>::to_f(stage16[rr * kDsPitch + c]);
     }
   }
 }
