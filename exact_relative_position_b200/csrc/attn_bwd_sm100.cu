@@ -95,13 +95,18 @@ constexpr uint32_t kOffAbort = kOffBar + 256;
 constexpr uint32_t kOffTmem = kOffAbort + 16;
 constexpr uint32_t kOffSat = kOffTmem + 16;          // [128 rows][2] saturated sums of column half 1
 constexpr uint32_t kSmemBytes = kOffSat + 1024 + 1024;
-// tensor memory: S buffers [0,128) and [128,256), dP [256,384), dQ [384,448),
-// dS [448,512) (16-bit, two keys per column: the A operand of dQ += dS K)
-constexpr uint32_t kTmDP = 256, kTmDQ = 384, kTmDS = 448;
+// tensor memory: S [0,128), dS buffers [128,192) and [192,256) (16-bit, two
+// keys per column: the A operand of dQ += dS K; compute half hc owns columns
+// 32 hc .. 32 hc + 31 of each), dP [256,384), dQ [384,448).  dS is double-
+// buffered so that writing dS(t + 1) waits for dQ(t - 1), not dQ(t).
+constexpr uint32_t kTmDS = 128, kTmDP = 256, kTmDQ = 384;
 // barriers
 constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kStages, kBarSFull = kBarKvEmpty + kStages,
-              kBarSFree = kBarSFull + 2, kBarDpFull = kBarSFree + 2, kBarDpFree = kBarDpFull + 1,
-              kBarDsReady = kBarDpFree + 1, kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
+              kBarSFree = kBarSFull + 1, kBarDpFull = kBarSFree + 1, kBarDpFree = kBarDpFull + 1,
+              // DsReady / DsFree: one per dS buffer.  With two buffers the compute
+              // warps can finish tile t + 1 before the MMA issuer has waited for
+              // tile t; per-buffer barriers keep every waiter within one phase.
+              kBarDsReady = kBarDpFree + 1, kBarDsFree = kBarDsReady + 2, kBarDrain = kBarDsFree + 2;
 }  // namespace qp
 
 template <typename T, bool AQ, bool AK, bool BIAS, bool DZQ, bool DQ32>
@@ -133,14 +138,14 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       mbar_init(bar(kBarKvFull + s), 1);
       mbar_init(bar(kBarKvEmpty + s), 1);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(bar(kBarSFull + u), 1);
-      mbar_init(bar(kBarSFree + u), 256);
-    }
+    mbar_init(bar(kBarSFull), 1);
+    mbar_init(bar(kBarSFree), 256);
     mbar_init(bar(kBarDpFull), 1);
     mbar_init(bar(kBarDpFree), 256);
-    mbar_init(bar(kBarDsReady), 256);
-    mbar_init(bar(kBarDsFree), 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(kBarDsReady + u), 256);
+      mbar_init(bar(kBarDsFree + u), 1);
+    }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -187,8 +192,8 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     } else if (warp == 1) {
       if (lane == 0 && nkt > 0) {
         // ------------------------------------------------------------ MMA issuer
-        // per tile t: dP(t+1) once dP(t) has been read, dQ += dS(t) K(t) once
-        // dS(t) is in shared memory, S(t+2) once S(t) has been read
+        // per tile t: S(t+1) once S(t) has been read, dP(t+1) once dP(t) has
+        // been read, dQ += dS(t) K(t) once dS(t) is in its tensor-memory buffer
         const bool bf = t.is_bf16 != 0;
         const uint32_t id_s = idesc_f16(bf, 128, 128, false, false);
         const uint32_t id_dq = idesc_f16(bf, 128, 64, false, true);
@@ -198,63 +203,53 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         const uint64_t dv0 = sdesc_sw128(sb + kOffKV + kTileBytes, 16, 1024);
         const uint64_t dkmn0 = sdesc_sw128(sb + kOffKV, 8192, 1024);
         constexpr uint64_t kStage16 = kStageBytes >> 4;
-        auto issue_s = [&](int buf, int s) {
+        auto issue_s = [&](int s) {
           const uint64_t kd = dk0 + (uint64_t)s * kStage16;
   #pragma unroll 1
-          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + (uint32_t)buf * 128, dq0 + 2 * kk, kd + 2 * kk, id_s, kk > 0);
+          for (int kk = 0; kk < 4; ++kk) mma_ss(tmem, dq0 + 2 * kk, kd + 2 * kk, id_s, kk > 0);
         };
         auto issue_dp = [&](int s) {
           const uint64_t vd = dv0 + (uint64_t)s * kStage16;
   #pragma unroll 1
           for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + kTmDP, ddo0 + 2 * kk, vd + 2 * kk, id_s, kk > 0);
         };
-        auto issue_dq = [&](int s, bool acc) {
+        // keys 16 kk .. 16 kk + 15 of dS are columns 8 kk .. 8 kk + 7 of its buffer
+        auto issue_dq = [&](int s, int db, bool acc) {
           const uint64_t kd = dkmn0 + (uint64_t)s * kStage16;
+          const uint32_t a = tmem + kTmDS + 64u * (uint32_t)db;
   #pragma unroll 1
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kTmDQ, tmem + kTmDS + 8 * kk, kd + 128 * kk, id_dq, (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) mma_ts(tmem + kTmDQ, a + 8 * kk, kd + 128 * kk, id_dq, (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0);
-          mma_commit(bar(kBarSFull + 0));
+          issue_s(0);
+          mma_commit(bar(kBarSFull));
           issue_dp(0);
           mma_commit(bar(kBarDpFull));
-          if (nkt > 1) {
-            ok = mbar_wait(bar(kBarKvFull + 1), 0, abort_flag);
-            if (ok) {
-              tc_fence_after();
-              issue_s(1, 1);
-              mma_commit(bar(kBarSFull + 1));
-            }
-          }
         }
   #pragma unroll 1
         for (int it = 0; it < nkt && ok; ++it) {
-          const int s = it % kStages;
+          const int s = it % kStages, s1 = (it + 1) % kStages;
           if (it + 1 < nkt) {
+            ok = mbar_wait(bar(kBarKvFull + s1), ((it + 1) / kStages) & 1, abort_flag) &&
+                 mbar_wait(bar(kBarSFree), it & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(s1);
+            mma_commit(bar(kBarSFull));
             ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            issue_dp((it + 1) % kStages);
+            issue_dp(s1);
             mma_commit(bar(kBarDpFull));
           }
-          ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
+          ok = mbar_wait(bar(kBarDsReady + (it & 1)), (it >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_dq(s, it > 0);
-          mma_commit(bar(kBarDsFree));
+          issue_dq(s, it & 1, it > 0);
+          mma_commit(bar(kBarDsFree + (it & 1)));
           mma_commit(bar(kBarKvEmpty + s));
-          if (it + 2 < nkt) {
-            const int s2 = (it + 2) % kStages;
-            ok = mbar_wait(bar(kBarKvFull + s2), ((it + 2) / kStages) & 1, abort_flag) &&
-                 mbar_wait(bar(kBarSFree + (it & 1)), (it >> 1) & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(it & 1, s2);
-            mma_commit(bar(kBarSFull + (it & 1)));
-          }
         }
         if (!ok) {
           mma_commit(bar(kBarDrain));
@@ -298,22 +293,22 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       const int j0 = it * kT;
       const int cls = tile_class(qt, it, N, nkv, p.causal, p.E_lo, p.E_hi);
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
-      const int stage = it % kStages, buf = it & 1;
+      const int stage = it % kStages;
       const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
                         (cls == RELPOS_TILE_CONST_LO ? 0 : kT) + cb;
-      const bool got_s = mbar_wait(bar(kBarSFull + buf), (it >> 1) & 1, abort_flag) &&
+      const bool got_s = mbar_wait(bar(kBarSFull), it & 1, abort_flag) &&
                          (!(AK && is_const) || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       float x[64];
       {
-        const uint32_t ts = tmem + t_lane + (uint32_t)buf * 128 + cb;
+        const uint32_t ts = tmem + t_lane + cb;
         tmem_ld32(ts + 0, reinterpret_cast<uint32_t*>(x) + 0);
         tmem_ld32(ts + 32, reinterpret_cast<uint32_t*>(x) + 32);
         tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarSFree + buf));   // S(t + 2) may now be written here
+      mbar_arrive(bar(kBarSFree));   // S(t + 1) may now be written
       // P = 2^(S tau log2e + relation terms - LSE log2e)
       if (is_const) {
         const float off = (cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi) - lse2;
@@ -395,16 +390,18 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           }
         }
       }
-      if (it > 0) {
-        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+      // dS buffer (t & 1) is free once dQ(t - 2) has read it
+      if (it > 1) {
+        const bool got = mbar_wait(bar(kBarDsFree + (it & 1)), ((it >> 1) - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
       }
       // this half's 64 keys of dS, two per tensor-memory column
       {
         uint32_t pk[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
-        tmem_st32(tmem + t_lane + kTmDS + 32 * hc, pk);
+        tmem_st32(tmem + t_lane + kTmDS + 64u * (uint32_t)(it & 1) + 32 * hc, pk);
         if (DZQ && !is_const) {
           // BAND tile: the same 16-bit values also go to the warp's staging
           // area (its own rows) for the coalesced by-offset store below
@@ -421,7 +418,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
                          p.causal, p.E_lo, p.E_hi, dzq_base, gi.S, gi.e0, p.tau);
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarDsReady));
+      mbar_arrive(bar(kBarDsReady + (it & 1)));
     }
     // -------------------------------------------------------------- epilogue
     if (DZQ) {
@@ -447,7 +444,8 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     float dq[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) dq[c] = 0.f;
-    const bool got_q = nkt > 0 && ok && mbar_wait(bar(kBarDsFree), (nkt - 1) & 1, abort_flag);
+    // the last dQ GEMM's commit covers every earlier one
+    const bool got_q = nkt > 0 && ok && mbar_wait(bar(kBarDsFree + ((nkt - 1) & 1)), ((nkt - 1) >> 1) & 1, abort_flag);
     if (__all_sync(0xffffffffu, got_q)) {
       tc_fence_after();
       uint32_t u[32];

@@ -303,13 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (is_const) {
         rowc = cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi;
         if (AK) {
+          const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
           for (int c = 0; c < 128; c += 4) {
             const float4 v4 = *reinterpret_cast<const float4*>(cv + c);
-            x[c] = fmaf(x[c], sc, v4.x);
-            x[c + 1] = fmaf(x[c + 1], sc, v4.y);
-            x[c + 2] = fmaf(x[c + 2], sc, v4.z);
-            x[c + 3] = fmaf(x[c + 3], sc, v4.w);
+            const float2 a = ffma2(make_float2(x[c], x[c + 1]), sc2, make_float2(v4.x, v4.y));
+            const float2 b2 = ffma2(make_float2(x[c + 2], x[c + 3]), sc2, make_float2(v4.z, v4.w));
+            x[c] = a.x; x[c + 1] = a.y; x[c + 2] = b2.x; x[c + 3] = b2.y;
           }
         } else {
           xs = sc;
@@ -372,34 +372,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run *= alpha;
         m_run = m_new;
       }
-      // P_g of the previous key tile must have been consumed by its PV GEMM
+      // p = 2^(x * xs + rowc - m_run), packed two keys per word; the words go
+      // to row r of P_g in tensor memory once the previous PV has read P_g,
+      // so that PV overlaps these exponentials
+      const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
+      const float2 xs2 = make_float2(xs, xs), ms2 = make_float2(-msub, -msub);
+      float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float ps[2] = {0.f, 0.f};
+      uint32_t pk[64];
+#pragma unroll
+      for (int w = 0; w < 64; ++w) {
+        const float2 z = ffma2(make_float2(x[2 * w], x[2 * w + 1]), xs2, ms2);
+        const float2 e = make_float2(fast_exp2(z.x), fast_exp2(z.y));
+        pk[w] = DT<T>::pack(e.x, e.y);
+        // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
+        // enough to sum the fp32 values and spare the conversions
+        if (DT<T>::kCoarse) ps[w & 1] += DT<T>::pair_sum(pk[w]);
+        else ps2[w & 1] = fadd2(ps2[w & 1], e);
+      }
+      l_run += DT<T>::kCoarse ? ps[0] + ps[1] : (ps2[0].x + ps2[1].x) + (ps2[0].y + ps2[1].y);
       if (!pfree_seen) {
         const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
       }
-      // p = 2^(x * xs + rowc - m_run), 64 keys at a time packed two per
-      // column into row r of P_g in tensor memory
-      const float msub = m_run == -INFINITY ? 0.f : m_run - rowc;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int hk = 0; hk < 2; ++hk) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float e8[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) e8[u] = fast_exp2(fmaf(x[64 * hk + 8 * c + u], xs, -msub));
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            pk[4 * c + u] = DT<T>::pack(e8[2 * u], e8[2 * u + 1]);
-            // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
-            // enough to sum the fp32 values and spare the conversions
-            ps[u] += DT<T>::kCoarse ? DT<T>::pair_sum(pk[4 * c + u]) : e8[2 * u] + e8[2 * u + 1];
-          }
-        }
-        tmem_st32(tP + 32 * hk, pk);
-      }
-      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      tmem_st32(tP, pk);
+      tmem_st32(tP + 32, pk + 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarPReady + g));
