@@ -135,6 +135,19 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank timings (a list of floats) over every rank
+    of the default process group; identity without one.  Each rank takes the same
+    collective step, so ranks that disagree on the list length fail loudly."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def cpu_baseline(w, R_exp, seconds=15.0, block=256):
     """The fp64 oracle on the host cores over blocks of query rows of head 0."""
     import numpy as np
@@ -305,10 +318,7 @@ def main():
     t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev)
     t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev)
     t_step = t_fwd + t_bwd
-    if world > 1:
-        tt = torch.tensor([t_step, t_fwd, t_bwd], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, t_fwd, t_bwd = tt.tolist()
+    t_step, t_fwd, t_bwd = max_over_ranks([t_step, t_fwd, t_bwd], dev)
     peak_mem = torch.cuda.max_memory_allocated(dev)
 
     # ---- end-to-end through the public API with host buffers
@@ -337,10 +347,7 @@ def main():
         if s > 0:
             e2e_ms += e0.elapsed_time(e1)
     e2e_ms /= e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = tt.item()
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
 
     if rank == 0:
         peaks = load_peaks()
