@@ -275,7 +275,8 @@ def main():
         rp.relpos_attn_fwd(q, k, v, aq, ak, b, out_f32=out_f32, workspace=ws, o=o, lse=lse, **kw)
 
     def bwd():
-        rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, workspace=ws, grads=grads, **kw)
+        # the backward reads the forward's tables and projections from `ws`
+        rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, workspace=ws, grads=grads, reuse_forward=True, **kw)
 
     if args.ncu:
         fwd()

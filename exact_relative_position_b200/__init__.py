@@ -22,9 +22,15 @@ class RelPosAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, aq, ak, b, tau, rmap, causal, key_len):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        o, lse = relpos_attn_fwd(q, k, v, aq, ak, b, tau=tau, map=rmap, causal=causal, key_len=key_len)
+        # one workspace for both passes: the backward reads the forward's
+        # tables and projections from it instead of recomputing them
+        kl = None if key_len is None else key_len.to(device=q.device, dtype=torch.int32)
+        fws, bws = workspace_size(q, aq, ak, b, tau, rmap, causal=causal, key_len=kl)
+        ws = torch.empty(max(fws, bws, 256), device=q.device, dtype=torch.uint8)
+        o, lse = relpos_attn_fwd(q, k, v, aq, ak, b, tau=tau, map=rmap, causal=causal, key_len=key_len, workspace=ws)
         ctx.save_for_backward(q, k, v, o, lse, aq, ak, b, key_len)
         ctx.cfg = (tau, rmap, causal)
+        ctx.ws = ws
         return o
 
     @staticmethod
@@ -32,7 +38,9 @@ class RelPosAttention(torch.autograd.Function):
         q, k, v, o, lse, aq, ak, b, key_len = ctx.saved_tensors
         tau, rmap, causal = ctx.cfg
         dq, dk, dv, daq, dak, db = relpos_attn_bwd(do.contiguous(), q, k, v, o, lse, aq, ak, b, tau=tau, map=rmap,
-                                                   causal=causal, key_len=key_len)
+                                                   causal=causal, key_len=key_len, workspace=ctx.ws,
+                                                   reuse_forward=True)
+        ctx.ws = None
         cast = lambda g, t: None if g is None else g.to(t.dtype)
         return dq, dk, dv, cast(daq, aq), cast(dak, ak), db, None, None, None, None
 

@@ -41,7 +41,7 @@ class relpos_fwd_args(ctypes.Structure):
 class relpos_bwd_args(ctypes.Structure):
     _fields_ = [("fwd", relpos_fwd_args), ("dout", ctypes.c_void_p), ("dq", ctypes.c_void_p),
                 ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p), ("daq", ctypes.c_void_p),
-                ("dak", ctypes.c_void_p), ("db", ctypes.c_void_p)]
+                ("dak", ctypes.c_void_p), ("db", ctypes.c_void_p), ("reuse_forward_workspace", ctypes.c_int32)]
 
 
 class relpos_phase_stat(ctypes.Structure):
@@ -212,8 +212,12 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
 
 
 def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap,
-                    causal: bool = False, key_len=None, workspace=None, grads=None):
-    """Backward through the C ABI.  Returns (dq, dk, dv, daq, dak, db)."""
+                    causal: bool = False, key_len=None, workspace=None, grads=None, reuse_forward: bool = False):
+    """Backward through the C ABI.  Returns (dq, dk, dv, daq, dak, db).
+
+    reuse_forward: `workspace` is the one the forward with these same arguments
+    ran in and still holds its tables and projections, so the backward reads
+    them instead of recomputing them."""
     if key_len is not None:
         key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
     out_f32 = o.dtype == torch.float32
@@ -234,7 +238,10 @@ def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: flo
     f, bw = ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
     if workspace is None or workspace.numel() < bw.value:
+        if reuse_forward:
+            raise RelPosError("reuse_forward needs the forward's workspace, at least the backward's size")
         workspace = torch.empty(max(bw.value, 256), device=q.device, dtype=torch.uint8)
+    g.reuse_forward_workspace = 1 if reuse_forward else 0
     _check(lib().relpos_attn_bwd(ctypes.byref(g), workspace.data_ptr(), workspace.numel(), _stream(q.device)),
            "relpos_attn_bwd")
     return dq, dk, dv, daq, dak, db

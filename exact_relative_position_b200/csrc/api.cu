@@ -214,7 +214,12 @@ int check_fwd_ptrs(const relpos_fwd_args* a) {
 
 // Resolve workspace regions and the expanded-table pointers; launch the
 // table builder and the projections (shared by forward and backward).
-int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Tensors& t, cudaStream_t s) {
+// Pointers into the workspace for a call with these arguments; when `build`
+// is set, also (re)computes the tables, group records and projections there
+// (the forward always builds; the backward skips it when the caller declares
+// the forward's state still in the workspace).
+int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Tensors& t, cudaStream_t s,
+            bool build = true) {
   memset(&t, 0, sizeof(t));
   GroupInfo* gq = reinterpret_cast<GroupInfo*>(ws + L.gq);
   GroupInfo* gk = reinterpret_cast<GroupInfo*>(ws + L.gk);
@@ -252,6 +257,7 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
     t.zk = reinterpret_cast<float*>(ws + L.zk);
     t.zk_sat = reinterpret_cast<float*>(ws + L.zksat);
   }
+  if (!build) return RELPOS_OK;
   cudaError_t e = run_phase(PH_TABLES, s, [&] {
     return launch_build_tables(p, a->map, gq, gk, phi_exp, L.R, a->aq, a->ak, a->table_per_head, ws + L.aqe,
                                ws + L.ake, a->b, const_cast<float*>(t.b_exp), t.is_bf16, L.expand, s);
@@ -330,8 +336,9 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   if (!workspace || ws_bytes < L.bwd_end || (reinterpret_cast<uintptr_t>(workspace) & 255)) return RELPOS_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (g->reuse_forward_workspace != 0 && g->reuse_forward_workspace != 1) return RELPOS_ERR_INVALID_ARG;
   Tensors t;
-  st = prepare(a, p, L, ws, t, s);
+  st = prepare(a, p, L, ws, t, s, /*build=*/g->reuse_forward_workspace == 0);
   if (st) return st;
   t.dout = g->dout;
   t.dsum = reinterpret_cast<float*>(ws + L.dsum);

@@ -121,6 +121,14 @@ typedef struct {
   float* daq;                /* device float32, shape of aq; required iff aq != NULL; overwritten */
   float* dak;                /* device float32, shape of ak; required iff ak != NULL; overwritten */
   float* db;                 /* device [H,R] float32; required iff b != NULL; overwritten */
+  int32_t reuse_forward_workspace;
+                             /* 1: `workspace` still holds what relpos_attn_fwd left in it
+                                for these same forward arguments (expanded tables, group
+                                records, projections Z^Q / Z^K and their saturated columns);
+                                the backward then reads them instead of rebuilding them (the
+                                digest's retained projection).  0: rebuild them.  With 1 and
+                                a workspace that does not hold that state the gradients are
+                                garbage: the library cannot tell. */
 } relpos_bwd_args;
 
 /* Number of rows R of a relation table for `map` at sequence length N (host only).

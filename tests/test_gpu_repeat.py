@@ -52,3 +52,31 @@ def test_repeated_calls_clean_and_identical(name, overrides):
                 assert b is None
             else:
                 assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name,overrides", [
+    ("deberta_log256_n2048", {"H": 4}),
+    ("shaw_clip64_n8192", {"H": 2}),
+    ("t5_bucket32_n8192", {"H": 2}),
+    ("shaw_clip16_n256", {"causal": True}),
+])
+def test_backward_reusing_forward_workspace_matches_rebuild(name, overrides):
+    """reuse_forward_workspace = 1 reads the forward's tables and projections
+    from the workspace; the gradients must equal a backward that rebuilds them."""
+    w = make_workload(name, **overrides)
+    dev = to_dev(w)
+    kw = dict(tau=w.tau, map=lmap(w), causal=w.causal, key_len=dev["key_len"])
+    fws, bws = rp.workspace_size(dev["q"], dev["aq"], dev["ak"], dev["b"], w.tau, lmap(w), causal=w.causal,
+                                 key_len=dev["key_len"])
+    ws = torch.empty(max(fws, bws), dtype=torch.uint8, device=dev["q"].device)
+    args = (dev["q"], dev["k"], dev["v"])
+    terms = (dev["aq"], dev["ak"], dev["b"])
+    o, lse = rp.relpos_attn_fwd(*args, *terms, workspace=ws, **kw)
+    reused = rp.relpos_attn_bwd(dev["do"], *args, o, lse, *terms, workspace=ws, reuse_forward=True, **kw)
+    assert rp.check_workspace(ws) == 0
+    rebuilt = rp.relpos_attn_bwd(dev["do"], *args, o, lse, *terms, **kw)
+    for a, b in zip(reused, rebuilt):
+        if a is None:
+            assert b is None
+        else:
+            assert torch.equal(a, b)
