@@ -50,7 +50,8 @@ def kernel_flops(w):
     """Tensor-core FLOPs each attention kernel's algorithm performs per launch."""
     cf = 0.5 if w.causal else 1.0
     base = 2.0 * w.B * w.H * w.N * w.N * w.d * cf    # one N x N x d GEMM
-    return {"fwd_attention": 2 * base, "bwd_dq": 3 * base, "bwd_dkdv": 4 * base}
+    # the two backward passes run concurrently (two streams): timed together
+    return {"fwd_attention": 2 * base, "bwd_attention": 7 * base}
 
 
 def load_peaks():
@@ -63,10 +64,16 @@ def load_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
+# the sources the attention kernels are compiled from (their code and every
+# header they include); a change to any of them invalidates the traffic record
+KERNEL_SOURCES = ("attn_fwd.cu", "attn_bwd_sm100.cu", "band.cuh", "common.cuh", "kernels.cuh", "sm100.cuh",
+                  "warp_mma.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_relative_position_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -81,8 +88,11 @@ def traffic_for(phase):
         j = json.load(f)
     if j.get("kernel_source_hash") != kernel_source_hash():
         return None
-    ent = j.get("kernels", {}).get(phase)
-    return None if ent is None else ent.get("dram_bytes_per_launch")
+    k = j.get("kernels", {})
+    parts = ("bwd_dq", "bwd_dkdv") if phase == "bwd_attention" else (phase,)
+    if any(k.get(ph) is None for ph in parts):
+        return None
+    return sum(k[ph]["dram_bytes_per_launch"] for ph in parts)
 
 
 class ClockSampler:

@@ -36,12 +36,13 @@ int relpos::cuda_status(cudaError_t e) { return cuda_fail(e); }
 namespace {
 
 // ---- optional per-phase event timing (relpos_profile_start / _stop)
-enum Phase { PH_TABLES, PH_PROJ, PH_FWD, PH_PREP, PH_DQ, PH_DKDV, PH_FOLD, PH_RELGRAD, PH_COUNT };
-const char* const kPhaseNames[PH_COUNT] = {"tables", "projection", "fwd_attention", "bwd_prep",
-                                           "bwd_dq", "bwd_dkdv", "fold_ranges", "relation_grads"};
+enum Phase { PH_TABLES, PH_PROJ, PH_FWD, PH_PREP, PH_DQ, PH_DKDV, PH_FOLD, PH_RELGRAD, PH_BWD_ATTN, PH_COUNT };
+const char* const kPhaseNames[PH_COUNT] = {"tables",  "projection", "fwd_attention", "bwd_prep",     "bwd_dq",
+                                           "bwd_dkdv", "fold_ranges", "relation_grads", "bwd_attention"};
+// Duration a -> b, or a -> the later of b and c when c is set (two streams).
 struct PhaseEvent {
   int phase, kernels;
-  cudaEvent_t a, b;
+  cudaEvent_t a, b, c;
 };
 std::mutex g_prof_mu;
 std::atomic<bool> g_prof_on{false};
@@ -57,9 +58,81 @@ cudaError_t run_phase(int ph, cudaStream_t s, F&& f) {
   const cudaError_t e = f();
   cudaEventRecord(b, s);
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  g_prof_events.push_back({ph, (int)(g_kernel_launches.load() - before), a, b});
+  g_prof_events.push_back({ph, (int)(g_kernel_launches.load() - before), a, b, nullptr});
   return e;
 }
+
+// "bwd_attention": both backward passes, which run concurrently on two
+// streams, from the start of the first to the end of the later one.
+struct PairTimer {
+  cudaEvent_t a = nullptr, b = nullptr, c = nullptr;
+  PairTimer() {
+    if (!g_prof_on.load()) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess ||
+        cudaEventCreate(&c) != cudaSuccess) {
+      cudaGetLastError();
+      a = b = c = nullptr;
+    }
+  }
+  void start(cudaStream_t s) { if (a) cudaEventRecord(a, s); }
+  void end_first(cudaStream_t s) { if (b) cudaEventRecord(b, s); }
+  void end_second(cudaStream_t s) { if (c) cudaEventRecord(c, s); }
+  void commit(int kernels) {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_events.push_back({PH_BWD_ATTN, kernels, a, b, c});
+  }
+};
+
+// A second stream per device, created once (non-blocking, never destroyed).
+// A fork records an event on the caller's stream and makes the side stream
+// wait for it; join does the reverse, so work issued on the side stream in
+// between is ordered before anything the caller issues afterwards (also under
+// stream capture).  If the side stream or the events cannot be created the
+// fork degrades to the caller's stream alone.
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    streams[dev] = nullptr;
+  }
+  return streams[dev];
+}
+
+class Fork {
+ public:
+  explicit Fork(cudaStream_t s) : s_(s), side_(s) {
+    cudaStream_t s2 = side_stream();
+    if (!s2 || cudaEventCreateWithFlags(&fork_, cudaEventDisableTiming) != cudaSuccess) return;
+    if (cudaEventCreateWithFlags(&join_, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventRecord(fork_, s) != cudaSuccess || cudaStreamWaitEvent(s2, fork_, 0) != cudaSuccess) {
+      cudaGetLastError();
+      return;
+    }
+    side_ = s2;
+  }
+  cudaStream_t side() const { return side_; }
+  cudaError_t join() {
+    cudaError_t e = cudaSuccess;
+    if (side_ != s_) {
+      e = cudaEventRecord(join_, side_);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s_, join_, 0);
+    }
+    return e;
+  }
+  ~Fork() {
+    if (fork_) cudaEventDestroy(fork_);
+    if (join_) cudaEventDestroy(join_);
+  }
+
+ private:
+  cudaStream_t s_, side_;
+  cudaEvent_t fork_ = nullptr, join_ = nullptr;
+};
 
 thread_local int g_last_cuda_error = 0;
 
@@ -366,13 +439,31 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   if (a->b) t.db_part = reinterpret_cast<float*>(ws + L.dbp);
   t.nsplit_q = L.nsq; t.nsplit_k = L.nsk; t.nsplit_b = L.nsb;
   if ((e = run_phase(PH_PREP, s, [&] { return launch_bwd_prep(p, t, s); })) != cudaSuccess) return cuda_fail(e);
-  if ((e = run_phase(PH_DQ, s, [&] { return launch_bwd_dq(p, t, s); })) != cudaSuccess) return cuda_fail(e);
-  if ((e = run_phase(PH_DKDV, s, [&] { return launch_bwd_dkdv(p, t, s); })) != cudaSuccess) return cuda_fail(e);
-  if (a->aq || a->ak || a->b) {
+  const bool terms = a->aq || a->ak || a->b;
+  if (terms) {
     e = run_phase(PH_FOLD, s, [&] { return launch_fold_ranges(p, t.phi_exp, L.R, t.fold_lo, t.fold_hi, s); });
     if (e != cudaSuccess) return cuda_fail(e);
-    if ((e = run_phase(PH_RELGRAD, s, [&] { return launch_relgrad(p, t, s); })) != cudaSuccess) return cuda_fail(e);
   }
+  // The Q-parallel pass (then the query-side relation gradients) stays on the
+  // caller's stream; the K-parallel pass (then the key side) runs on a second
+  // stream forked from it, so that its CTAs fill the SMs the other pass leaves
+  // idle in its last partial wave.  The caller's stream waits for both.
+  Fork fork(s);
+  cudaStream_t s2 = fork.side();
+  cudaError_t e2 = cudaSuccess;
+  PairTimer pair;
+  pair.start(s);
+  e = run_phase(PH_DQ, s, [&] { return launch_bwd_dq(p, t, s); });
+  pair.end_first(s);
+  e2 = run_phase(PH_DKDV, s2, [&] { return launch_bwd_dkdv(p, t, s2); });
+  pair.end_second(s2);
+  pair.commit(2);
+  if (terms && e == cudaSuccess) e = run_phase(PH_RELGRAD, s, [&] { return launch_relgrad(p, t, 0, s); });
+  if (a->ak && e2 == cudaSuccess) e2 = run_phase(PH_RELGRAD, s2, [&] { return launch_relgrad(p, t, 1, s2); });
+  const cudaError_t ej = fork.join();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (e2 != cudaSuccess) return cuda_fail(e2);
+  if (ej != cudaSuccess) return cuda_fail(ej);
   return RELPOS_OK;
 }
 
@@ -406,6 +497,7 @@ RELPOS_EXPORT int relpos_profile_start(void) {
   for (auto& ev : g_prof_events) {
     cudaEventDestroy(ev.a);
     cudaEventDestroy(ev.b);
+    if (ev.c) cudaEventDestroy(ev.c);
   }
   g_prof_events.clear();
   g_prof_on = true;
@@ -422,12 +514,19 @@ RELPOS_EXPORT int relpos_profile_stop(relpos_phase_stat* stats, int32_t max_stat
     float ms = 0.f;
     cudaError_t e = cudaEventSynchronize(ev.b);
     if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, ev.a, ev.b);
+    if (e == cudaSuccess && ev.c) {
+      float ms2 = 0.f;
+      e = cudaEventSynchronize(ev.c);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms2, ev.a, ev.c);
+      ms = std::max(ms, ms2);
+    }
     if (e != cudaSuccess) status = cuda_fail(e);
     agg[ev.phase].calls += 1;
     agg[ev.phase].kernels += ev.kernels;
     agg[ev.phase].total_ms += ms;
     cudaEventDestroy(ev.a);
     cudaEventDestroy(ev.b);
+    if (ev.c) cudaEventDestroy(ev.c);
   }
   g_prof_events.clear();
   int n = 0;

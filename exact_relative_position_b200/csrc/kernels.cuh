@@ -63,7 +63,9 @@ cudaError_t launch_forward(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dkdv(const Plan& p, const Tensors& t, cudaStream_t s);
-cudaError_t launch_relgrad(const Plan& p, const Tensors& t, cudaStream_t s);
+// side 0: query-side relation gradients (dQ += dZ^Q aQ_exp, daQ, db);
+// side 1: key side (dK += dZ^K aK_exp, daK)
+cudaError_t launch_relgrad(const Plan& p, const Tensors& t, int side, cudaStream_t s);
 cudaError_t launch_debug_phi(const relpos_map_desc& map, int N, int* out, cudaStream_t s);
 cudaError_t launch_debug_tile_plan(int B, int N, int causal, const int* key_len, int E_lo, int E_hi,
                                    int* classes, int* segs, cudaStream_t s);

@@ -573,8 +573,9 @@ cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s) {
   return t.is_bf16 ? projection_typed<__nv_bfloat16>(p, t, s) : projection_typed<__half>(p, t, s);
 }
 
+// side 0: the query side (aQ rows, aQ table, bias); side 1: the key side (aK).
 template <typename T>
-static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
+static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cudaStream_t s) {
   const int Hq = t.table_per_head ? p.H : 1;
   const int nE = (p.Rexp + tp::kEB - 1) / tp::kEB;
   constexpr uint32_t kRowsSmem = rg::kStages * rg::stage_bytes<T>();
@@ -583,7 +584,7 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(table_part_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPartSmem);
   if (e != cudaSuccess) return e;
-  if (t.aq_exp) {
+  if (side == 0 && t.aq_exp) {
     { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
                                                                         t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
     { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
@@ -591,7 +592,7 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s
     { fold_kernel<<<dim3(t.R, Hq), 256, 0, s>>>(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64,
                                                                      t.fold_lo, t.fold_hi, t.daq); note_launch(1); }
   }
-  if (t.ak_exp) {
+  if (side == 1 && t.ak_exp) {
     { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
                                                                         t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
     { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
@@ -599,7 +600,7 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s
     { fold_kernel<<<dim3(t.R, Hq), 256, 0, s>>>(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64,
                                                                      t.fold_lo, t.fold_hi, t.dak); note_launch(1); }
   }
-  if (t.b_exp) {
+  if (side == 0 && t.b_exp) {
     { bias_part_kernel<<<dim3((p.Rexp + 255) / 256, p.H, t.nsplit_b), 256, 0, s>>>(p, t.dzq, p.zq_head, t.nsplit_b, t.db_part); note_launch(1); }
     { fold_kernel<<<dim3(t.R, p.H), 256, 0, s>>>(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1,
                                                                  t.fold_lo, t.fold_hi, t.db); note_launch(1); }
@@ -607,8 +608,8 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, cudaStream_t s
   return cudaGetLastError();
 }
 
-cudaError_t launch_relgrad(const Plan& p, const Tensors& t, cudaStream_t s) {
-  return t.is_bf16 ? relgrad_typed<__nv_bfloat16>(p, t, s) : relgrad_typed<__half>(p, t, s);
+cudaError_t launch_relgrad(const Plan& p, const Tensors& t, int side, cudaStream_t s) {
+  return t.is_bf16 ? relgrad_typed<__nv_bfloat16>(p, t, side, s) : relgrad_typed<__half>(p, t, side, s);
 }
 
 cudaError_t launch_debug_phi(const relpos_map_desc& map, int N, int* out, cudaStream_t s) {

@@ -197,12 +197,18 @@ int relpos_attn_fwd_noalloc(const relpos_fwd_args* a, relpos_stream_t stream);
 
 /* Per-phase device time collected between relpos_profile_start and
  * relpos_profile_stop.  Phases: "tables", "projection", "fwd_attention",
- * "bwd_prep", "bwd_dq", "bwd_dkdv", "fold_ranges", "relation_grads". */
+ * "bwd_prep", "bwd_dq", "bwd_dkdv", "fold_ranges", "relation_grads",
+ * "bwd_attention".  The backward runs its Q-parallel pass (then the query-side
+ * relation gradients) on the caller's stream and its K-parallel pass (then the
+ * key side) concurrently on a second stream, so "bwd_dkdv" and the key-side
+ * "relation_grads" are measured on that stream and overlap other phases;
+ * "bwd_attention" spans both passes, from the start of the first to the end
+ * of the later one. */
 typedef struct {
   char name[32];
   int32_t calls;       /* times the phase ran */
   int32_t kernels;     /* kernels it launched in total */
-  float total_ms;      /* summed device time (CUDA events on the caller's stream) */
+  float total_ms;      /* summed device time (CUDA events on the stream(s) the phase ran on) */
 } relpos_phase_stat;
 
 /* Starts bracketing every phase the library enqueues with CUDA events
