@@ -291,7 +291,12 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
 #pragma unroll 1
     for (int it = 0; it < nkt; ++it) {
       const int j0 = it * kT;
-      const int cls = tile_class(qt, it, N, nkv, p.causal, p.E_lo, p.E_hi);
+      // class of this half's 64 keys: the two halves of a tile on the edge of
+      // the band often differ (one BAND, one CONST).  Bias-only variants keep
+      // the tile's class (their band is wider than a half for the maps here,
+      // and the extra live values make that variant spill).
+      const int cls = (AQ || AK) ? half_class(qt, it, hc, true, N, nkv, p.causal, p.E_lo, p.E_hi)
+                                 : tile_class(qt, it, N, nkv, p.causal, p.E_lo, p.E_hi);
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
       const int stage = it % kStages;
       const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
@@ -708,7 +713,9 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
 #pragma unroll 1
     for (int it = 0; it < nq; ++it) {
       const int qi = qt0 + it, qb = qi * kT;
-      const int cls = tile_class(qi, kt, N, nkv, p.causal, p.E_lo, p.E_hi);
+      // class of this half's 64 queries (bias-only variants: the tile's class)
+      const int cls = (AQ || AK) ? half_class(qi, kt, hc, false, N, nkv, p.causal, p.E_lo, p.E_hi)
+                                 : tile_class(qi, kt, N, nkv, p.causal, p.E_lo, p.E_hi);
       const bool is_const = cls == RELPOS_TILE_CONST_LO || cls == RELPOS_TILE_CONST_HI;
       const int stage = it % kStages;
       const float* vec = reinterpret_cast<const float*>(sg + kOffQD + (uint32_t)stage * kStageBytes + 2 * kTileBytes);

@@ -145,14 +145,39 @@ RP_HD long long head_elems(const Plan& p, int key_side) {
 // ---------------------------------------------------------------------------
 // Tile plan: the two comparisons of a tile's offset range with (E_lo, E_hi).
 // ---------------------------------------------------------------------------
-RP_HD int tile_class(int qi, int kj, int N, int nkv, int causal, int E_lo, int E_hi) {
-  const int i0 = qi * kTile, i1 = imin(i0 + kTile, N) - 1;
-  const int j0 = kj * kTile, j1 = imin(j0 + kTile, N) - 1;
+// Class of the cells with queries [i0, i1] and keys [j0, j1] (both ranges
+// inside [0, N)): the same two comparisons as for a whole tile.
+RP_HD int block_class(int i0, int i1, int j0, int j1, int nkv, int causal, int E_lo, int E_hi) {
   if (j0 >= nkv || (causal && j0 > i1)) return RELPOS_TILE_MASKED;
   const int j1v = imin(j1, nkv - 1);
   if (j1v - i0 <= E_lo) return RELPOS_TILE_CONST_LO;
   if (j0 - i1 >= E_hi) return RELPOS_TILE_CONST_HI;
   return RELPOS_TILE_BAND;
+}
+
+RP_HD int tile_class(int qi, int kj, int N, int nkv, int causal, int E_lo, int E_hi) {
+  const int i0 = qi * kTile, i1 = imin(i0 + kTile, N) - 1;
+  const int j0 = kj * kTile, j1 = imin(j0 + kTile, N) - 1;
+  return block_class(i0, i1, j0, j1, nkv, causal, E_lo, E_hi);
+}
+
+// Class of the 64-column half h of tile (qi, kj) as the backward's compute
+// warps see it: the half's columns are keys (key_cols) or queries; a half
+// whose cells are all masked counts as CONST_LO (its values are masked to 0).
+RP_HD int half_class(int qi, int kj, int h, bool key_cols, int N, int nkv, int causal, int E_lo, int E_hi) {
+  int i0 = qi * kTile, i1 = imin(i0 + kTile, N) - 1;
+  int j0 = kj * kTile, j1 = imin(j0 + kTile, N) - 1;
+  if (key_cols) {
+    j0 += 64 * h;
+    j1 = imin(j1, j0 + 63);
+    if (j0 > j1) return RELPOS_TILE_CONST_LO;
+  } else {
+    i0 += 64 * h;
+    i1 = imin(i1, i0 + 63);
+    if (i0 > i1) return RELPOS_TILE_CONST_LO;
+  }
+  const int c = block_class(i0, i1, j0, j1, nkv, causal, E_lo, E_hi);
+  return c == RELPOS_TILE_MASKED ? RELPOS_TILE_CONST_LO : c;
 }
 
 // Segments of query tile qi: key tiles [0, lo_end) are CONST_LO, [lo_end,
