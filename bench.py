@@ -230,6 +230,65 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """--sweep: the sequence-length sweep of the four mechanisms at 16384 tokens
+    per batch (B = 16384 / N), one JSON line per (mechanism, N): forward and
+    backward device time (CUDA events, L2 flushed before every step) and
+    useful TFLOP/s."""
+    import torch
+    import exact_relative_position_b200 as rp
+    from synth import SWEEP_LENGTHS, SWEEP_MECHANISMS, sweep_workload
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    mechs = args.sweep_mechanisms.split(",") if args.sweep_mechanisms else list(SWEEP_MECHANISMS)
+    lengths = [int(x) for x in args.sweep_lengths.split(",")] if args.sweep_lengths else list(SWEEP_LENGTHS)
+    for mech in mechs:
+        for N in lengths:
+            w = sweep_workload(mech, N)
+            m = rp.RelPosMap(w.map_kind, w.clip, w.num_buckets, w.max_distance, w.bidirectional)
+            elo, ehi = rp.expanded_bounds(m, w.N)
+            fwd_flops, bwd_flops = useful_flops(w, ehi - elo + 1)
+            d = lambda t: None if t is None else t.to(dev).contiguous()
+            q, k, v, do, aq, ak, b = (d(getattr(w, n)) for n in ("q", "k", "v", "do", "aq", "ak", "b"))
+            o = torch.empty_like(q)
+            lse = torch.empty(q.shape[:3], device=dev, dtype=torch.float32)
+            grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                     None if aq is None else torch.empty(aq.shape, device=dev, dtype=torch.float32),
+                     None if ak is None else torch.empty(ak.shape, device=dev, dtype=torch.float32),
+                     None if b is None else torch.empty(b.shape, device=dev, dtype=torch.float32))
+            fws, bws = rp.workspace_size(q, aq, ak, b, w.tau, m)
+            ws = torch.empty(max(fws, bws), device=dev, dtype=torch.uint8)
+            steps = args.sweep_steps
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+            for s in range(args.warmup + steps):
+                flush.zero_()
+                if s >= args.warmup:
+                    ev[s - args.warmup][0].record()
+                rp.relpos_attn_fwd(q, k, v, aq, ak, b, tau=w.tau, map=m, workspace=ws, o=o, lse=lse)
+                if s >= args.warmup:
+                    ev[s - args.warmup][1].record()
+                rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, tau=w.tau, map=m, workspace=ws, grads=grads,
+                                   reuse_forward=True)
+                if s >= args.warmup:
+                    ev[s - args.warmup][2].record()
+            torch.cuda.synchronize()
+            if rp.check_workspace(ws) != 0:
+                raise RuntimeError(f"{w.name}: device status not clean")
+            fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+            bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+            print(json.dumps({
+                "sweep": mech, "N": N, "B": w.B, "H": w.H, "d": w.d, "dtype": "fp16", "steps": steps,
+                "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+                "fwd_frac_of_peak": fwd_flops / (fwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "bwd_frac_of_peak": bwd_flops / (bwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "workspace_bytes": int(ws.numel()), "l2": "flushed before every step"}), flush=True)
+            del q, k, v, do, aq, ak, b, o, lse, grads, ws
+            torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -239,6 +298,11 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="sequence-length sweep of the four mechanisms at 16384 tokens per batch (one JSON line each)")
+    ap.add_argument("--sweep-mechanisms", default="", help="comma list (default: all four)")
+    ap.add_argument("--sweep-lengths", default="", help="comma list of N (default: 128 ... 8192)")
+    ap.add_argument("--sweep-steps", type=int, default=10)
     ap.add_argument("--ncu", action="store_true",
                     help="one forward + backward only (for an ncu capture of each kernel's first launch)")
     args = ap.parse_args()
@@ -249,6 +313,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
 
     import torch

@@ -112,6 +112,31 @@ CONFIGS = {
 }
 
 
+# The pages' sequence-length sweep: the four mechanisms at a fixed budget of
+# 16384 tokens per batch (B = 16384 / N) for N = 128 ... 8192, 12 heads,
+# head dim 64, fp16, bidirectional (no mask).
+SWEEP_TOKENS = 16384
+SWEEP_LENGTHS = (128, 256, 512, 1024, 2048, 4096, 8192)
+SWEEP_MECHANISMS = {
+    "shaw_clip256": dict(map_kind="truncated", clip=256, terms=("aQ", "aK"), tau=1 / 8),
+    "txl_identity": dict(map_kind="identity", terms=("aQ", "b"), per_head_tables=True, tau=1 / 8, txl=True),
+    "deberta_log256": dict(map_kind="log", num_buckets=256, max_distance=512, terms=("aQ", "aK"),
+                           per_head_tables=True, tau=1 / math.sqrt(3 * 64)),
+    "t5_bucket32": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=1, terms=("b",), tau=1.0,
+                        b_std=0.5),
+}
+
+
+def sweep_workload(mechanism: str, N: int, seed: int = 0, tokens: int = SWEEP_TOKENS, H: int = 12,
+                   **overrides) -> "Workload":
+    """One point of the sequence-length sweep: `mechanism` at length N with
+    B = tokens / N (rounded down, at least 1)."""
+    spec = dict(SWEEP_MECHANISMS[mechanism])
+    spec.update(name=f"{mechanism}_n{N}", B=max(1, tokens // N), H=H, N=N, d=64, dtype=torch.float16)
+    spec.update(overrides)
+    return make_workload(spec, seed=seed)
+
+
 def _normal(gen, shape, std):
     return torch.randn(shape, generator=gen, dtype=torch.float32) * std
 
