@@ -258,7 +258,7 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   L->dzk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
   L->dqacc = aq ? take(sizeof(float) * BH * N * 64) : 0;
   L->dkacc = ak ? take(sizeof(float) * BH * N * 64) : 0;
-  const int nE = (p->Rexp + 127) / 128;   // expanded-row blocks of the table-gradient kernel
+  const int nE = (p->Rexp + 255) / 256;   // expanded-row blocks of the table-gradient kernel
   const long long items = a->table_per_head ? (long long)a->B * p->nT : (long long)BH * p->nT;
   auto pick = [](long long want, long long items_) {
     long long s = std::max(1LL, want);
@@ -266,7 +266,7 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
     s = std::min(s, 256LL);
     return (int)std::max(1LL, s);
   };
-  L->nsq = pick(296LL / ((long long)nE * L->Hq), items);
+  L->nsq = pick(148LL / ((long long)nE * L->Hq), items);   // one table-gradient CTA per SM
   L->nsk = L->nsq;
   L->nsb = pick(592LL / ((long long)((p->Rexp + 255) / 256) * a->H), (long long)a->B * p->nT);
   L->daqp = aq ? take(sizeof(float) * (size_t)L->nsq * L->Hq * p->Rexp * 64) : 0;

@@ -260,15 +260,19 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
 // ------------------------------------------------------------------ table partials
 // part[s][hq][c0 + m][:] = sum over the split's (batch, head, group) items, in
 // order, of dZ_g[rows, c0 + m - e0] X[rows, :]   (tf32 tensor cores)
-// Block (e-block of 128 expanded rows, table, split).  The split's positions
-// are streamed in chunks of 32 rows of (dZ, X) through a 4-stage cp.async
+// Block (e-block of 256 expanded rows, table, split).  The split's positions
+// are streamed in chunks of 32 rows of (dZ, X) through a 3-stage cp.async
 // ring that runs across item boundaries; items whose group stores none of the
-// block's columns are skipped.  Warp w owns expanded rows 16w .. 16w + 15.
+// block's columns are skipped.  Warp w owns expanded rows 32w .. 32w + 31 (two
+// m16 tiles), so every X fragment feeds two MMAs.  dZ is copied in 16-byte
+// pieces when the item's first column lines up with the block (the common
+// case: e0 = 0 for every group of a map whose groups reach all offsets), else
+// in 4-byte pieces.
 namespace tp {
-constexpr int kEB = 128;       // expanded rows per block
+constexpr int kEB = 256;       // expanded rows per block
 constexpr int kRC = 32;        // positions per chunk
-constexpr int kStages = 4;
-constexpr int kZP = 136;       // floats per row of a dZ chunk [32][128]: conflict-free transposed fragment reads
+constexpr int kStages = 3;
+constexpr int kZP = 264;       // floats per row of a dZ chunk [32][256]: conflict-free transposed fragment reads
 constexpr int kXP = 72;        // elements per row of an X chunk [32][64]
 template <typename T>
 constexpr uint32_t stage_bytes() { return (uint32_t)kRC * kZP * 4u + (uint32_t)(kRC * kXP * sizeof(T)); }
@@ -333,15 +337,29 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
     const T* Xg = X + ((size_t)bh * p.N + r0) * 64;
     const uint32_t zs = sbase + (uint32_t)(q % tp::kStages) * kSB;
     const uint32_t xs = zs + (uint32_t)tp::kRC * tp::kZP * 4u;
-    // dZ rows rc .. rc + 31, expanded columns c0 .. c0 + 127 (4-byte copies:
-    // the group's first column e0 has no alignment)
+    // dZ rows rc .. rc + 31, expanded columns c0 .. c0 + 255 (local column lc = c - e0)
+    if (((c0 - gi.e0) & 3) == 0) {
+      // 16-byte pieces: lc is a multiple of 4 and the row stride S too; the
+      // columns [W, S) are stored zeros
 #pragma unroll 4
-    for (int u = 0; u < tp::kRC * tp::kEB / 256; ++u) {
-      const int idx = u * 256 + tid;
-      const int r = idx >> 7, c = idx & 127;
-      const int lc = c0 + c - gi.e0;
-      const bool ok = cur.rc + r < nrows && lc >= 0 && lc < gi.W;
-      cp_async4(zs + (uint32_t)(r * tp::kZP + c) * 4u, ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg, ok ? 4 : 0);
+      for (int u = 0; u < tp::kRC * tp::kEB / 4 / 256; ++u) {
+        const int idx = u * 256 + tid;
+        const int r = idx >> 6, c = (idx & 63) * 4;
+        const int lc = c0 + c - gi.e0;
+        const bool ok = cur.rc + r < nrows && lc >= 0 && lc < gi.S;
+        cp_async16(zs + (uint32_t)(r * tp::kZP + c) * 4u, ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg,
+                   ok ? 16 : 0);
+      }
+    } else {
+#pragma unroll 4
+      for (int u = 0; u < tp::kRC * tp::kEB / 256; ++u) {
+        const int idx = u * 256 + tid;
+        const int r = idx >> 8, c = idx & 255;
+        const int lc = c0 + c - gi.e0;
+        const bool ok = cur.rc + r < nrows && lc >= 0 && lc < gi.W;
+        cp_async4(zs + (uint32_t)(r * tp::kZP + c) * 4u, ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg,
+                  ok ? 4 : 0);
+      }
     }
     {
       const int r = tid >> 3, pc = tid & 7;
@@ -356,10 +374,12 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
       skip();
     }
   };
-  const int g8 = lane >> 2, tq = lane & 3, eb = warp * 16;
-  float acc[8][4];
+  const int g8 = lane >> 2, tq = lane & 3, eb = warp * 32;
+  float acc[2][8][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[mt][i][0] = acc[mt][i][1] = acc[mt][i][2] = acc[mt][i][3] = 0.f;
 #pragma unroll
   for (int q = 0; q < tp::kStages - 1; ++q) {
     if (q < nchunks) load(q);
@@ -376,28 +396,37 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
 #pragma unroll
     for (int ks = 0; ks < tp::kRC / 8; ++ks) {
       // A = dZ^T: rows = expanded offsets, columns = positions
-      const uint32_t a0 = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + eb + g8]);
-      const uint32_t a1 = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + eb + g8 + 8]);
-      const uint32_t a2 = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + eb + g8]);
-      const uint32_t a3 = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + eb + g8 + 8]);
+      uint32_t a[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int m0 = eb + 16 * mt + g8;
+        a[mt][0] = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + m0]);
+        a[mt][1] = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + m0 + 8]);
+        a[mt][2] = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + m0]);
+        a[mt][3] = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + m0 + 8]);
+      }
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const uint32_t b0 = __float_as_uint(DT<T>::to_f(Xs[(ks * 8 + tq) * tp::kXP + nt * 8 + g8]));
         const uint32_t b1 = __float_as_uint(DT<T>::to_f(Xs[(ks * 8 + tq + 4) * tp::kXP + nt * 8 + g8]));
-        mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
       }
     }
   }
   cp_async_wait<0>();
   float* P = part + ((size_t)s * Hq + hq) * (size_t)p.Rexp * 64;
 #pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    const int e = c0 + eb + g8 + 8 * hf;
-    if (e >= p.Rexp) continue;
+  for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int d = nt * 8 + 2 * tq;
-      *reinterpret_cast<float2*>(P + (size_t)e * 64 + d) = make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+    for (int hf = 0; hf < 2; ++hf) {
+      const int e = c0 + eb + 16 * mt + g8 + 8 * hf;
+      if (e >= p.Rexp) continue;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int d = nt * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(P + (size_t)e * 64 + d) = make_float2(acc[mt][nt][2 * hf], acc[mt][nt][2 * hf + 1]);
+      }
     }
   }
 }
