@@ -1,0 +1,70 @@
+"""Model-level adapters over `relpos_attention`.
+
+Transformer-XL's relative attention written in the unified score of the paper
+digest ("Fast and Exact Relative-Position Attention via Structure-Aware
+Kernels", Eq. (1); the Transformer-XL workload of its experimental setup): for
+head h,
+
+    score_ij = tau [ (q_i + u_h) . k_j  +  (q_i + v_h) . W_r^h R_(j - i) ]
+
+with R the fixed sinusoid table over offsets and W_r^h the layer's relation
+projection.  In the unified form this is
+
+    q' = q + u,   aQ_h = R W_r^h (identity map, one row per offset),
+    b_h[r] = (v_h - u_h) . aQ_h[r],
+
+so the kernel sees q'.k + q'.aQ + b.  The re-parameterisation is plain PyTorch,
+so autograd carries the kernel's gradients (dq, daQ, db) on to u, v and W_r.
+Offsets follow the library's convention delta = j - i (Transformer-XL writes
+R_(i - j): the same table with its rows reversed).
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import RelPosMap, relpos_attention
+
+
+def sinusoid_table(N: int, dim: int, device=None) -> torch.Tensor:
+    """[2N - 1, dim] float32: row r is offset r - (N - 1), columns
+    [sin(delta w_m) | cos(delta w_m)] with w_m = 10000^(-2m / dim)."""
+    off = torch.arange(-(N - 1), N, dtype=torch.float64, device=device)
+    m = torch.arange(dim // 2, dtype=torch.float64, device=device)
+    omega = torch.pow(10000.0, -2.0 * m / dim)
+    ang = off[:, None] * omega[None, :]
+    return torch.cat([torch.sin(ang), torch.cos(ang)], dim=1).float()
+
+
+class TransformerXLRelPos(torch.nn.Module):
+    """One Transformer-XL relative attention layer over given q, k, v.
+
+    Parameters: W_r [H, d_model, d_head] (relation projection per head), u, v
+    [H, d_head] (the content and position biases).  forward(q, k, v) with
+    q, k, v [B, H, N, d_head] fp16/bf16 on the GPU returns O [B, H, N, d_head].
+    """
+
+    def __init__(self, n_heads: int, d_head: int = 64, d_model: int | None = None, causal: bool = True,
+                 tau: float | None = None, init_std: float = 0.02):
+        super().__init__()
+        self.n_heads, self.d_head = n_heads, d_head
+        self.d_model = d_model or n_heads * d_head
+        self.causal = causal
+        self.tau = tau if tau is not None else 1.0 / math.sqrt(d_head)
+        self.W_r = torch.nn.Parameter(torch.randn(n_heads, self.d_model, d_head) * init_std)
+        self.u = torch.nn.Parameter(torch.randn(n_heads, d_head) * init_std)
+        self.v = torch.nn.Parameter(torch.randn(n_heads, d_head) * init_std)
+
+    def unified_inputs(self, q: torch.Tensor):
+        """q' = q + u, aQ [H, 2N - 1, d] (in q's dtype) and b [H, 2N - 1] fp32."""
+        N = q.shape[2]
+        R = sinusoid_table(N, self.d_model, device=q.device)
+        aq32 = torch.einsum("rc,hcd->hrd", R, self.W_r.float())
+        b = torch.einsum("hd,hrd->hr", (self.v - self.u).float(), aq32)
+        qp = q + self.u[None, :, None, :].to(q.dtype)
+        return qp, aq32.to(q.dtype).contiguous(), b.contiguous()
+
+    def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
+        qp, aq, b = self.unified_inputs(q)
+        return relpos_attention(qp, k, v, aq, None, b, tau=self.tau, map=RelPosMap("identity"), causal=self.causal)
