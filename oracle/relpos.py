@@ -267,6 +267,55 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
+# ----------------------------------------------------------------------------
+# Attention dropout (the scope table's next row f3; not on the pages, the
+# standard attention-dropout semantics): O = (P o M / (1 - p)) V with P the
+# softmax of S (so LSE is that of S), M_ij in {0, 1}.  The mask is drawn by
+# the counter-based generator Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+# "Parallel random numbers: as easy as 1, 2, 3", SC 2011), restated here from
+# that definition: ten rounds of
+#     (hi0, lo0) = M0 * x0,  (hi1, lo1) = M1 * x2   (32 x 32 -> 64-bit products)
+#     x = (hi1 ^ x1 ^ k0, lo1, hi0 ^ x3 ^ k1, lo0)
+# with the key bumped by (W0, W1) before every round after the first.
+# Cell (bh, i, j): counter (j >> 1, i >> 1, bh, offset), key (seed low 32
+# bits, seed high 32 bits); output word 2 (i & 1) + (j & 1) as w; kept when
+# (w >> 8) 2^-24 >= p.
+# ----------------------------------------------------------------------------
+
+PHILOX_M0, PHILOX_M1 = 0xD2511F53, 0xCD9E8D57
+PHILOX_W0, PHILOX_W1 = 0x9E3779B9, 0xBB67AE85
+
+
+def philox4x32_10(ctr, key):
+    """ctr: 4 arrays (or ints) of uint32, key: 2 of them (broadcast together).
+    Returns the 4 output words as uint64 arrays holding 32-bit values."""
+    mask = np.uint64(0xFFFFFFFF)
+    x = [np.asarray(c, dtype=np.uint64) & mask for c in ctr]
+    k0, k1 = (np.asarray(c, dtype=np.uint64) & mask for c in key)
+    for r in range(10):
+        if r > 0:
+            k0 = (k0 + np.uint64(PHILOX_W0)) & mask
+            k1 = (k1 + np.uint64(PHILOX_W1)) & mask
+        p0 = np.uint64(PHILOX_M0) * x[0]
+        p1 = np.uint64(PHILOX_M1) * x[2]
+        hi0, lo0 = p0 >> np.uint64(32), p0 & mask
+        hi1, lo1 = p1 >> np.uint64(32), p1 & mask
+        x = [hi1 ^ x[1] ^ k0, lo1, hi0 ^ x[3] ^ k1, lo0]
+    return x
+
+
+def dropout_keep(bh, rows, N, p, seed, offset):
+    """Kept cells [len(rows), N] (bool) of slice bh = b * H + h."""
+    i = np.asarray(rows, dtype=np.uint64)[:, None]
+    j = np.arange(N, dtype=np.uint64)[None, :]
+    w = philox4x32_10((j >> np.uint64(1), i >> np.uint64(1), np.uint64(bh), np.uint64(offset & 0xFFFFFFFF)),
+                      (np.uint64(seed & 0xFFFFFFFF), np.uint64((seed >> 32) & 0xFFFFFFFF)))
+    sel = (i & np.uint64(1)) * np.uint64(2) + (j & np.uint64(1))
+    word = np.choose(sel.astype(np.int64) + np.zeros(w[0].shape, dtype=np.int64), w)
+    u = (word >> np.uint64(8)).astype(np.float64) * 2.0 ** -24
+    return u >= p
+
+
 def head_scores(q, k, aq, ak, bvec, tau, phi, allowed):
     """S for query rows q [n, d] against all keys k [N, d] (Eq. (1) via Eq. (2)/(3)).
 
@@ -297,21 +346,27 @@ def head_softmax(S):
     return P, lse
 
 
-def head_forward(q, k, v, aq, ak, bvec, tau, phi, allowed):
+def head_forward(q, k, v, aq, ak, bvec, tau, phi, allowed, keep=None, p=0.0):
+    """O, LSE, P of one slice; with `keep` (bool [n, N]) O uses P o keep / (1 - p)."""
     S = head_scores(q, k, aq, ak, bvec, tau, phi, allowed)
     P, lse = head_softmax(S)
-    return P @ v, lse, P
+    Pv = P if keep is None else np.where(keep, P / (1.0 - p), 0.0)
+    return Pv @ v, lse, P
 
 
-def head_backward(q, k, v, do, aq, ak, bvec, tau, phi, allowed, R):
+def head_backward(q, k, v, do, aq, ak, bvec, tau, phi, allowed, R, keep=None, p=0.0):
     """Gradients of one full (b, h) slice for the upstream gradient dO.
 
     Returns dict: dq, dk, dv, dzq [N,R], dzk [N,R], daq [R,d], dak [R,d], db [R],
-    plus o, lse."""
+    plus o, lse.  With dropout (`keep`), O = (P o M s) V, s = 1 / (1 - p):
+    dV = (P o M s)^T dO, dS = P o (M s o dO V^T - D), D_i = sum_c dO_ic O_ic."""
     N, d = q.shape
-    O, lse, P = head_forward(q, k, v, aq, ak, bvec, tau, phi, allowed)
-    dV = P.T @ do
+    O, lse, P = head_forward(q, k, v, aq, ak, bvec, tau, phi, allowed, keep, p)
+    Ms = None if keep is None else np.where(keep, 1.0 / (1.0 - p), 0.0)
+    dV = (P if Ms is None else P * Ms).T @ do
     dP = do @ v.T
+    if Ms is not None:
+        dP = dP * Ms
     D = np.sum(do * O, axis=1, keepdims=True)
     dS = P * (dP - D)                                   # gradient w.r.t. S (incl. tau)
     rows = np.repeat(np.arange(N), N)
@@ -346,11 +401,12 @@ def _table(t, h):
     return t[h] if t.ndim == 3 else t
 
 
-def forward(q, k, v, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None, rows=None):
+def forward(q, k, v, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None, rows=None,
+            dropout_p=0.0, dropout_seed=0, dropout_offset=0):
     """O [B,H,n,d] and LSE [B,H,n] for the query rows `rows` (default all).
 
     q, k, v: [B,H,N,d]; aq, ak: [R,d] (shared) or [H,R,d] (per head) or None;
-    b: [H,R] or None; key_len: [B] or None."""
+    b: [H,R] or None; key_len: [B] or None; dropout as in dropout_keep."""
     q, k, v, aq, ak, b = (_f64(x) for x in (q, k, v, aq, ak, b))
     B, H, N, d = q.shape
     rows = np.arange(N) if rows is None else np.asarray(rows)
@@ -361,13 +417,16 @@ def forward(q, k, v, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None, row
     for bi in range(B):
         allowed = allowed_matrix(N, causal, None if kl is None else kl[bi], rows)
         for h in range(H):
+            keep = None if dropout_p == 0 else dropout_keep(bi * H + h, rows, N, dropout_p, dropout_seed,
+                                                             dropout_offset)
             o, lse, _ = head_forward(q[bi, h, rows], k[bi, h], v[bi, h], _table(aq, h),
-                                     _table(ak, h), None if b is None else b[h], tau, phi, allowed)
+                                     _table(ak, h), None if b is None else b[h], tau, phi, allowed, keep, dropout_p)
             O[bi, h], L[bi, h] = o, lse
     return O, L
 
 
-def backward(q, k, v, do, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None):
+def backward(q, k, v, do, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None,
+             dropout_p=0.0, dropout_seed=0, dropout_offset=0):
     """All outputs and gradients of the layer for upstream gradient dO.
 
     Shared tables ([R,d]) get gradients summed over batch then heads in
@@ -386,8 +445,10 @@ def backward(q, k, v, do, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None
     for h in range(H):
         for bi in range(B):
             allowed = allowed_matrix(N, causal, None if kl is None else kl[bi])
+            keep = None if dropout_p == 0 else dropout_keep(bi * H + h, np.arange(N), N, dropout_p, dropout_seed,
+                                                             dropout_offset)
             g = head_backward(q[bi, h], k[bi, h], v[bi, h], do[bi, h], _table(aq, h),
-                              _table(ak, h), None if b is None else b[h], tau, phi, allowed, R)
+                              _table(ak, h), None if b is None else b[h], tau, phi, allowed, R, keep, dropout_p)
             for n in ("o", "dq", "dk", "dv", "lse"):
                 res[n][bi, h] = g[n]
             if aq is not None:

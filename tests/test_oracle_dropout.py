@@ -1,0 +1,102 @@
+"""Pins of the oracle's attention dropout (scope-table next row f3).
+
+The Philox4x32-10 generator against its published known-answer vectors
+(tests/golden/philox4x32_10_kat.json); the keep rate; the p = 0 case against
+the dropout-free oracle; and the dropout backward against central finite
+differences of sum(dO o O) with the mask held fixed (the mask depends only on
+(seed, offset, b, h, i, j), never on the inputs)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle as orc
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def test_philox_known_answer_vectors():
+    with open(os.path.join(HERE, "golden", "philox4x32_10_kat.json")) as f:
+        kat = json.load(f)
+    for v in kat["vectors"]:
+        ctr = [int(x, 16) for x in v["ctr"]]
+        key = [int(x, 16) for x in v["key"]]
+        out = orc.philox4x32_10(ctr, key)
+        assert [int(o) for o in out] == [int(x, 16) for x in v["out"]]
+
+
+def test_philox_vectorised_matches_scalar():
+    rng = np.random.default_rng(0)
+    ctr = rng.integers(0, 2 ** 32, size=(4, 50), dtype=np.uint64)
+    key = rng.integers(0, 2 ** 32, size=(2, 50), dtype=np.uint64)
+    vec = orc.philox4x32_10(list(ctr), list(key))
+    for t in range(50):
+        sc = orc.philox4x32_10([int(c[t]) for c in ctr], [int(k[t]) for k in key])
+        assert [int(w[t]) for w in vec] == [int(x) for x in sc]
+
+
+@pytest.mark.parametrize("p", [0.1, 0.5, 0.9])
+def test_keep_rate(p):
+    keep = orc.dropout_keep(5, np.arange(512), 512, p, seed=0x1234_5678_9ABC_DEF0, offset=77)
+    n = keep.size
+    sd = np.sqrt(p * (1 - p) / n)
+    assert abs(keep.mean() - (1 - p)) < 6 * sd
+
+
+def test_mask_rows_are_independent_of_the_row_subset():
+    full = orc.dropout_keep(3, np.arange(40), 40, 0.3, seed=9, offset=4)
+    rows = np.array([0, 7, 8, 33])
+    assert np.array_equal(orc.dropout_keep(3, rows, 40, 0.3, seed=9, offset=4), full[rows])
+    # another slice, seed or offset gives another mask
+    assert not np.array_equal(orc.dropout_keep(4, np.arange(40), 40, 0.3, 9, 4), full)
+    assert not np.array_equal(orc.dropout_keep(3, np.arange(40), 40, 0.3, 10, 4), full)
+    assert not np.array_equal(orc.dropout_keep(3, np.arange(40), 40, 0.3, 9, 5), full)
+
+
+def _case():
+    N, d, H, B = 9, 3, 2, 2
+    m = orc.MapDesc("truncated", clip=2)
+    R = orc.table_rows(m, N)
+    rng = np.random.default_rng(7)
+    x = dict(q=rng.standard_normal((B, H, N, d)), k=rng.standard_normal((B, H, N, d)),
+             v=rng.standard_normal((B, H, N, d)), aq=rng.standard_normal((R, d)) * 0.5,
+             ak=rng.standard_normal((R, d)) * 0.5, b=rng.standard_normal((H, R)))
+    return m, x, rng.standard_normal((B, H, N, d)), 0.45
+
+
+def test_zero_rate_equals_no_dropout():
+    m, x, do, tau = _case()
+    a = orc.backward(x["q"], x["k"], x["v"], do, x["aq"], x["ak"], x["b"], tau, m, causal=True)
+    b = orc.backward(x["q"], x["k"], x["v"], do, x["aq"], x["ak"], x["b"], tau, m, causal=True,
+                     dropout_p=0.0, dropout_seed=5, dropout_offset=1)
+    for n in ("o", "lse", "dq", "dk", "dv", "daq", "dak", "db"):
+        assert np.array_equal(a[n], b[n])
+
+
+@pytest.mark.parametrize("p,causal", [(0.3, False), (0.6, True)])
+def test_dropout_gradients_central_differences(p, causal):
+    m, x, do, tau = _case()
+    kw = dict(causal=causal, dropout_p=p, dropout_seed=0xABCDEF0123, dropout_offset=3)
+
+    def loss(xx):
+        O, _ = orc.forward(xx["q"], xx["k"], xx["v"], xx["aq"], xx["ak"], xx["b"], tau, m, **kw)
+        return float(np.sum(O * do))
+
+    g = orc.backward(x["q"], x["k"], x["v"], do, x["aq"], x["ak"], x["b"], tau, m, **kw)
+    # the forward inside backward() agrees with forward()
+    O, L = orc.forward(x["q"], x["k"], x["v"], x["aq"], x["ak"], x["b"], tau, m, **kw)
+    assert np.allclose(g["o"], O, rtol=0, atol=1e-13) and np.allclose(g["lse"], L, rtol=0, atol=1e-13)
+    names = {"q": "dq", "k": "dk", "v": "dv", "aq": "daq", "ak": "dak", "b": "db"}
+    eps = 1e-6
+    rng = np.random.default_rng(3)
+    for n, gn in names.items():
+        flat = x[n].reshape(-1)
+        for t in rng.choice(flat.size, size=min(flat.size, 30), replace=False):
+            xp = {kk: vv.copy() for kk, vv in x.items()}
+            xm = {kk: vv.copy() for kk, vv in x.items()}
+            xp[n].reshape(-1)[t] += eps
+            xm[n].reshape(-1)[t] -= eps
+            fd = (loss(xp) - loss(xm)) / (2 * eps)
+            an = g[gn].reshape(-1)[t]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (n, t, fd, an)
