@@ -298,6 +298,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="attention dropout rate for a measurement of its cost (default 0: none)")
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length sweep of the four mechanisms at 16384 tokens per batch (one JSON line each)")
     ap.add_argument("--sweep-mechanisms", default="", help="comma list (default: all four)")
@@ -348,12 +350,15 @@ def main():
     flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)   # 256 MiB > 126 MB L2
     kw = dict(tau=w.tau, map=m, causal=w.causal, key_len=kl)
 
+    dkw = dict(dropout_p=args.dropout, dropout_seed=0x5EED, dropout_offset=0)
+
     def fwd():
-        rp.relpos_attn_fwd(q, k, v, aq, ak, b, out_f32=out_f32, workspace=ws, o=o, lse=lse, **kw)
+        rp.relpos_attn_fwd(q, k, v, aq, ak, b, out_f32=out_f32, workspace=ws, o=o, lse=lse, **kw, **dkw)
 
     def bwd():
         # the backward reads the forward's tables and projections from `ws`
-        rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, workspace=ws, grads=grads, reuse_forward=True, **kw)
+        rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, workspace=ws, grads=grads, reuse_forward=True, **kw,
+                           **dkw)
 
     if args.ncu:
         fwd()
@@ -452,6 +457,7 @@ def main():
             "dtype": "fp16" if w.dtype == torch.float16 else "bf16", "data": "synthetic",
             "config": {"workload": args.workload, **{k_: v_ for k_, v_ in w.describe().items() if k_ != "workload"},
                        "R_exp": R_exp, "l2": "flushed (256 MiB write) before every step",
+                       "dropout": args.dropout,
                        "parallelism": f"replicas x{world}"},
             "passes": {
                 "fwd_ms": t_fwd / args.steps, "bwd_ms": t_bwd / args.steps,

@@ -35,7 +35,8 @@ class relpos_fwd_args(ctypes.Structure):
                 ("map", relpos_map_desc), ("mask", ctypes.c_int32), ("table_per_head", ctypes.c_int32),
                 ("key_len", ctypes.c_void_p), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("aq", ctypes.c_void_p), ("ak", ctypes.c_void_p),
-                ("b", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+                ("b", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("dropout_p", ctypes.c_float), ("dropout_offset", ctypes.c_uint32), ("dropout_seed", ctypes.c_uint64)]
 
 
 class relpos_bwd_args(ctypes.Structure):
@@ -151,7 +152,8 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise RelPosError(f"unsupported dtype {dt}")
 
 
-def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o=None, lse=None):
+def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o=None, lse=None,
+              dropout=(0.0, 0, 0)):
     B, H, N, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda or not t.is_contiguous() or t.shape != q.shape or t.dtype != q.dtype:
@@ -177,6 +179,7 @@ def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o
     a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
     a.aq, a.ak, a.b = _ptr(aq), _ptr(ak), _ptr(b)
     a.o, a.lse = _ptr(o), _ptr(lse)
+    a.dropout_p, a.dropout_seed, a.dropout_offset = float(dropout[0]), int(dropout[1]), int(dropout[2])
     return a
 
 
@@ -192,8 +195,11 @@ def _stream(dev) -> int:
 
 
 def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap, causal: bool = False,
-                    key_len=None, out_f32: bool = False, workspace=None, o=None, lse=None):
-    """Forward through the C ABI.  Returns (O, LSE); O is float32 when out_f32."""
+                    key_len=None, out_f32: bool = False, workspace=None, o=None, lse=None,
+                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
+    """Forward through the C ABI.  Returns (O, LSE); O is float32 when out_f32.
+    Attention dropout with rate dropout_p uses the Philox mask of (seed, offset);
+    the backward needs the same three values."""
     B, H, N, d = q.shape
     if o is None:
         o = torch.empty(q.shape, device=q.device, dtype=torch.float32 if out_f32 else q.dtype)
@@ -201,7 +207,8 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
     if key_len is not None:
         key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
-    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse)
+    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse,
+                  (dropout_p, dropout_seed, dropout_offset))
     f, bw = ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
     if workspace is None or workspace.numel() < f.value:
@@ -212,7 +219,8 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
 
 
 def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap,
-                    causal: bool = False, key_len=None, workspace=None, grads=None, reuse_forward: bool = False):
+                    causal: bool = False, key_len=None, workspace=None, grads=None, reuse_forward: bool = False,
+                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
     """Backward through the C ABI.  Returns (dq, dk, dv, daq, dak, db).
 
     reuse_forward: `workspace` is the one the forward with these same arguments
@@ -223,7 +231,8 @@ def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: flo
     out_f32 = o.dtype == torch.float32
     if not dout.is_contiguous() or dout.dtype != q.dtype or dout.shape != q.shape:
         raise RelPosError("dout must be contiguous, shaped and typed like q")
-    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse)
+    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse,
+                  (dropout_p, dropout_seed, dropout_offset))
     g = relpos_bwd_args()
     g.fwd = a
     if grads is None:

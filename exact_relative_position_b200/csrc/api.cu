@@ -227,6 +227,13 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   p->causal = (a->mask & RELPOS_MASK_CAUSAL) != 0;
   p->padding = (a->mask & RELPOS_MASK_KEY_PADDING) != 0;
   p->tau = a->tau;
+  if (!(a->dropout_p >= 0.f && a->dropout_p < 1.f)) return RELPOS_ERR_INVALID_ARG;
+  p->dropout = a->dropout_p > 0.f;
+  p->drop_thresh = (uint32_t)ceil((double)a->dropout_p * 16777216.0);
+  p->drop_scale = p->dropout ? 1.f / (1.f - a->dropout_p) : 1.f;
+  p->seed_lo = (uint32_t)(a->dropout_seed & 0xFFFFFFFFull);
+  p->seed_hi = (uint32_t)(a->dropout_seed >> 32);
+  p->drop_offset = a->dropout_offset;
   const bool aq = a->aq != nullptr, ak = a->ak != nullptr, bb = a->b != nullptr;
   const long long zq_head = head_elems(*p, 0), zk_head = head_elems(*p, 1);
   p->zq_head = (aq || bb) ? zq_head : 0;

@@ -109,7 +109,7 @@ constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kStages, kBa
               kBarDsReady = kBarDpFree + 1, kBarDsFree = kBarDsReady + 2, kBarDrain = kBarDsFree + 2;
 }  // namespace qp
 
-template <typename T, bool AQ, bool AK, bool BIAS, bool DZQ, bool DQ32>
+template <typename T, bool AQ, bool AK, bool BIAS, bool DZQ, bool DQ32, bool DROP>
 __global__ void __launch_bounds__(qp::kThreads, 1)
     dq_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -366,6 +366,15 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(kBarDpFree));     // dP(t + 1) may now be written
+        if (DROP) {
+          // dropout: dS = P o (M / (1 - p) o dP - D)
+#pragma unroll
+          for (int w = 0; w < 32; ++w) {
+            const uint32_t kb = keep_key_pair(p, bh, i, j0 + cb + 2 * w);
+            dp[2 * w] = __float_as_uint((kb & 1u) ? __uint_as_float(dp[2 * w]) * p.drop_scale : 0.f);
+            dp[2 * w + 1] = __float_as_uint((kb & 2u) ? __uint_as_float(dp[2 * w + 1]) * p.drop_scale : 0.f);
+          }
+        }
         if (!DZQ || is_const) {
           float ssum[2] = {0.f, 0.f};
 #pragma unroll
@@ -522,7 +531,7 @@ constexpr int kBarKV = 0, kBarQsFull = 1, kBarQsEmpty = kBarQsFull + kStages, kB
               kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
 }  // namespace kp
 
-template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32>
+template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32, bool DROP>
 __global__ void __launch_bounds__(kp::kThreads, 1)
     dkdv_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -786,10 +795,24 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
       }
+      // dropout: keep bits of this half's 64 queries for this key (bit c of km)
+      uint32_t km[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+      if (DROP) {
+        km[0] = km[1] = 0u;
+#pragma unroll
+        for (int w = 0; w < 32; ++w) km[w >> 4] |= keep_query_pair(p, bh, qb + cb + 2 * w, j) << (2 * (w & 15));
+      }
+      auto kept = [&](int c) { return ((km[c >> 5] >> (c & 31)) & 1u) != 0u; };
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
+        for (int u = 0; u < 32; ++u) {
+          if (DROP)   // dV sees P^T o M / (1 - p)
+            pk[u] = DT<T>::pack(kept(2 * u) ? x[2 * u] * p.drop_scale : 0.f,
+                                kept(2 * u + 1) ? x[2 * u + 1] * p.drop_scale : 0.f);
+          else
+            pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
+        }
         tmem_st32(tmem + t_lane + kTmP + 32 * hc, pk);
         tmem_wait_st();
       }
@@ -808,6 +831,11 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(kBarDpFree));   // dP(t + 1) may now be written
+        if (DROP) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            dp[c] = __float_as_uint(kept(c) ? __uint_as_float(dp[c]) * p.drop_scale : 0.f);
+        }
         if (!DZK || is_const) {
           float ssum[2] = {0.f, 0.f};
 #pragma unroll
@@ -984,8 +1012,10 @@ cudaError_t dq_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   const dim3 grid(p.nT, p.B * p.H);
 #define RP_DQ(A, K_, B_)                                                                                       \
   if (aq == A && ak == K_ && bb == B_)                                                                         \
-    return launch4(dq_sm100_kernel<T, A, K_, B_, (A || B_), A>, grid, qp::kThreads, qp::kSmemBytes, p, t, m.q, \
-                   m.k, m.v, m.dout, s);
+    return p.dropout ? launch4(dq_sm100_kernel<T, A, K_, B_, (A || B_), A, true>, grid, qp::kThreads,          \
+                               qp::kSmemBytes, p, t, m.q, m.k, m.v, m.dout, s)                                 \
+                     : launch4(dq_sm100_kernel<T, A, K_, B_, (A || B_), A, false>, grid, qp::kThreads,         \
+                               qp::kSmemBytes, p, t, m.q, m.k, m.v, m.dout, s);
   RP_DQ(false, false, false) RP_DQ(true, false, false) RP_DQ(false, true, false) RP_DQ(true, true, false)
   RP_DQ(false, false, true) RP_DQ(true, false, true) RP_DQ(false, true, true) RP_DQ(true, true, true)
 #undef RP_DQ
@@ -1000,8 +1030,10 @@ cudaError_t dk_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   const dim3 grid(p.nT, p.B * p.H);
 #define RP_DK(A, K_, B_)                                                                                         \
   if (aq == A && ak == K_ && bb == B_)                                                                           \
-    return launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_>, grid, kp::kThreads, kp::kSmemBytes, p, t, m.q, m.k, \
-                   m.v, m.dout, s);
+    return p.dropout ? launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, true>, grid, kp::kThreads, kp::kSmemBytes, \
+                               p, t, m.q, m.k, m.v, m.dout, s)                                                   \
+                     : launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, false>, grid, kp::kThreads, kp::kSmemBytes, \
+                               p, t, m.q, m.k, m.v, m.dout, s);
   RP_DK(false, false, false) RP_DK(true, false, false) RP_DK(false, true, false) RP_DK(true, true, false)
   RP_DK(false, false, true) RP_DK(true, false, true) RP_DK(false, true, true) RP_DK(true, true, true)
 #undef RP_DK

@@ -97,7 +97,7 @@ template <typename T> struct RowStore {
   }
 };
 
-template <typename T, typename OutT, bool AQ, bool AK, bool BIAS>
+template <typename T, typename OutT, bool AQ, bool AK, bool BIAS, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
@@ -386,9 +386,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 e = make_float2(fast_exp2(z.x), fast_exp2(z.y));
         pk[w] = DT<T>::pack(e.x, e.y);
         // bf16 keeps 8 bits: sum what PV really uses; fp16's rounding is small
-        // enough to sum the fp32 values and spare the conversions
+        // enough to sum the fp32 values and spare the conversions.  The row sum
+        // (hence LSE) is that of the undropped P.
         if (DT<T>::kCoarse) ps[w & 1] += DT<T>::pair_sum(pk[w]);
         else ps2[w & 1] = fadd2(ps2[w & 1], e);
+        if (DROP) {
+          // PV sees P o M / (1 - p)
+          const uint32_t kb = keep_key_pair(p, bh, i, j0 + 2 * w);
+          pk[w] = DT<T>::pack((kb & 1u) ? e.x * p.drop_scale : 0.f, (kb & 2u) ? e.y * p.drop_scale : 0.f);
+        }
       }
       l_run += DT<T>::kCoarse ? ps[0] + ps[1] : (ps2[0].x + ps2[1].x) + (ps2[0].y + ps2[1].y);
       if (!pfree_seen) {
@@ -469,15 +475,23 @@ template <typename T, typename OutT>
 cudaError_t launch_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   const int mask = (t.aq_exp ? 1 : 0) | (t.ak_exp ? 2 : 0) | (t.b_exp ? 4 : 0);
   void (*kern)(const Plan, const Tensors, const CUtensorMap, const CUtensorMap, const CUtensorMap) = nullptr;
-  switch (mask) {
-    case 0: kern = fwd_sm100_kernel<T, OutT, false, false, false>; break;
-    case 1: kern = fwd_sm100_kernel<T, OutT, true, false, false>; break;
-    case 2: kern = fwd_sm100_kernel<T, OutT, false, true, false>; break;
-    case 3: kern = fwd_sm100_kernel<T, OutT, true, true, false>; break;
-    case 4: kern = fwd_sm100_kernel<T, OutT, false, false, true>; break;
-    case 5: kern = fwd_sm100_kernel<T, OutT, true, false, true>; break;
-    case 6: kern = fwd_sm100_kernel<T, OutT, false, true, true>; break;
-    default: kern = fwd_sm100_kernel<T, OutT, true, true, true>; break;
+  switch (mask + (p.dropout ? 8 : 0)) {
+    case 0: kern = fwd_sm100_kernel<T, OutT, false, false, false, false>; break;
+    case 1: kern = fwd_sm100_kernel<T, OutT, true, false, false, false>; break;
+    case 2: kern = fwd_sm100_kernel<T, OutT, false, true, false, false>; break;
+    case 3: kern = fwd_sm100_kernel<T, OutT, true, true, false, false>; break;
+    case 4: kern = fwd_sm100_kernel<T, OutT, false, false, true, false>; break;
+    case 5: kern = fwd_sm100_kernel<T, OutT, true, false, true, false>; break;
+    case 6: kern = fwd_sm100_kernel<T, OutT, false, true, true, false>; break;
+    case 7: kern = fwd_sm100_kernel<T, OutT, true, true, true, false>; break;
+    case 8: kern = fwd_sm100_kernel<T, OutT, false, false, false, true>; break;
+    case 9: kern = fwd_sm100_kernel<T, OutT, true, false, false, true>; break;
+    case 10: kern = fwd_sm100_kernel<T, OutT, false, true, false, true>; break;
+    case 11: kern = fwd_sm100_kernel<T, OutT, true, true, false, true>; break;
+    case 12: kern = fwd_sm100_kernel<T, OutT, false, false, true, true>; break;
+    case 13: kern = fwd_sm100_kernel<T, OutT, true, false, true, true>; break;
+    case 14: kern = fwd_sm100_kernel<T, OutT, false, true, true, true>; break;
+    default: kern = fwd_sm100_kernel<T, OutT, true, true, true, true>; break;
   }
   CUtensorMap mq, mk, mv;
   const int BH = p.B * p.H;

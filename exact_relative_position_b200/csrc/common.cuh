@@ -101,6 +101,10 @@ struct Plan {
   const GroupInfo* gq;          // device [nT]
   const GroupInfo* gk;          // device [nT]
   const int* key_len;           // device [B] or null
+  // attention dropout (0 = off): keep cell when (Philox word >> 8) >= drop_thresh
+  int dropout;
+  uint32_t drop_thresh, seed_lo, seed_hi, drop_offset;
+  float drop_scale;             // 1 / (1 - p)
 };
 
 // Reachable expanded columns of query group g (key_side = 0) or key group g
@@ -228,5 +232,55 @@ template <> struct DT<__nv_bfloat16> {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------------------
+// Attention dropout mask.  Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC 2011), restated from its
+// definition: ten rounds of (hi0, lo0) = M0 x0, (hi1, lo1) = M1 x2 (32 x 32 ->
+// 64-bit), x = (hi1 ^ x1 ^ k0, lo1, hi0 ^ x3 ^ k1, lo0), the key bumped by
+// (W0, W1) before every round after the first.  Cell (bh, i, j) uses counter
+// (j >> 1, i >> 1, bh, offset) and key (seed_lo, seed_hi) and takes output word
+// 2 (i & 1) + (j & 1): one generator call serves a 2 x 2 block, i.e. a pair of
+// keys of one query row and a pair of queries of one key row alike.
+// ---------------------------------------------------------------------------
+#ifdef __CUDACC__
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
+                                               uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, x0), lo0 = 0xD2511F53u * x0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, x2), lo1 = 0xCD9E8D57u * x2;
+    x0 = hi1 ^ x1 ^ k0;
+    x1 = lo1;
+    x2 = hi0 ^ x3 ^ k1;
+    x3 = lo0;
+  }
+  return make_uint4(x0, x1, x2, x3);
+}
+
+__device__ __forceinline__ uint32_t philox_word(const uint4& w, int idx) {
+  return idx == 0 ? w.x : idx == 1 ? w.y : idx == 2 ? w.z : w.w;
+}
+
+// Keep bits of cells (i, j) [bit 0] and (i, j + 1) [bit 1] of slice bh, j even.
+__device__ __forceinline__ uint32_t keep_key_pair(const Plan& p, int bh, int i, int j) {
+  const uint4 w = philox4x32_10((uint32_t)j >> 1, (uint32_t)i >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
+  const int base = 2 * (i & 1);
+  return ((philox_word(w, base) >> 8) >= p.drop_thresh ? 1u : 0u) |
+         ((philox_word(w, base + 1) >> 8) >= p.drop_thresh ? 2u : 0u);
+}
+
+// Keep bits of cells (i, j) [bit 0] and (i + 1, j) [bit 1] of slice bh, i even.
+__device__ __forceinline__ uint32_t keep_query_pair(const Plan& p, int bh, int i, int j) {
+  const uint4 w = philox4x32_10((uint32_t)j >> 1, (uint32_t)i >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
+  const int jb = j & 1;
+  return ((philox_word(w, jb) >> 8) >= p.drop_thresh ? 1u : 0u) |
+         ((philox_word(w, 2 + jb) >> 8) >= p.drop_thresh ? 2u : 0u);
+}
+#endif
 
 }  // namespace relpos

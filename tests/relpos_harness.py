@@ -31,25 +31,28 @@ def to_dev(w, device="cuda"):
     return dict(q=d(w.q), k=d(w.k), v=d(w.v), do=d(w.do), aq=d(w.aq), ak=d(w.ak), b=d(w.b), key_len=d(w.key_len))
 
 
-def run_library(w, backward=True, out_f32=False, dev=None):
+def run_library(w, backward=True, out_f32=False, dev=None, dropout=(0.0, 0, 0)):
     dev = dev or to_dev(w)
+    dkw = dict(dropout_p=dropout[0], dropout_seed=dropout[1], dropout_offset=dropout[2])
     o, lse = rp.relpos_attn_fwd(dev["q"], dev["k"], dev["v"], dev["aq"], dev["ak"], dev["b"], tau=w.tau,
-                                map=lmap(w), causal=w.causal, key_len=dev["key_len"], out_f32=out_f32)
+                                map=lmap(w), causal=w.causal, key_len=dev["key_len"], out_f32=out_f32, **dkw)
     res = dict(o=o, lse=lse)
     if backward:
         dq, dk, dv, daq, dak, db = rp.relpos_attn_bwd(dev["do"], dev["q"], dev["k"], dev["v"], o, lse, dev["aq"],
                                                       dev["ak"], dev["b"], tau=w.tau, map=lmap(w), causal=w.causal,
-                                                      key_len=dev["key_len"])
+                                                      key_len=dev["key_len"], **dkw)
         res.update(dq=dq, dk=dk, dv=dv, daq=daq, dak=dak, db=db)
     torch.cuda.synchronize()
     return {k: (None if v is None else v.detach().double().cpu().numpy()) for k, v in res.items()}
 
 
-def run_oracle(w, backward=True):
+def run_oracle(w, backward=True, dropout=(0.0, 0, 0)):
     kl = None if w.key_len is None else w.key_len.numpy()
+    # the library receives the rate as float32: the oracle takes that value
+    dkw = dict(dropout_p=float(np.float32(dropout[0])), dropout_seed=dropout[1], dropout_offset=dropout[2])
     if backward:
-        return orc.backward(w.q, w.k, w.v, w.do, w.aq, w.ak, w.b, w.tau, omap(w), causal=w.causal, key_len=kl)
-    O, L = orc.forward(w.q, w.k, w.v, w.aq, w.ak, w.b, w.tau, omap(w), causal=w.causal, key_len=kl)
+        return orc.backward(w.q, w.k, w.v, w.do, w.aq, w.ak, w.b, w.tau, omap(w), causal=w.causal, key_len=kl, **dkw)
+    O, L = orc.forward(w.q, w.k, w.v, w.aq, w.ak, w.b, w.tau, omap(w), causal=w.causal, key_len=kl, **dkw)
     return dict(o=O, lse=L)
 
 
