@@ -368,9 +368,11 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         mbar_arrive(bar(kBarDpFree));     // dP(t + 1) may now be written
         if (DROP) {
           // dropout: dS = P o (M / (1 - p) o dP - D)
+          uint32_t km[2];
+          keep_mask64(p, bh, i, j0 + cb, true, km);
 #pragma unroll
           for (int w = 0; w < 32; ++w) {
-            const uint32_t kb = keep_key_pair(p, bh, i, j0 + cb + 2 * w);
+            const uint32_t kb = (km[w >> 4] >> (2 * (w & 15))) & 3u;
             dp[2 * w] = __float_as_uint((kb & 1u) ? __uint_as_float(dp[2 * w]) * p.drop_scale : 0.f);
             dp[2 * w + 1] = __float_as_uint((kb & 2u) ? __uint_as_float(dp[2 * w + 1]) * p.drop_scale : 0.f);
           }
@@ -797,11 +799,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       }
       // dropout: keep bits of this half's 64 queries for this key (bit c of km)
       uint32_t km[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
-      if (DROP) {
-        km[0] = km[1] = 0u;
-#pragma unroll
-        for (int w = 0; w < 32; ++w) km[w >> 4] |= keep_query_pair(p, bh, qb + cb + 2 * w, j) << (2 * (w & 15));
-      }
+      if (DROP) keep_mask64(p, bh, j, qb + cb, false, km);
       auto kept = [&](int c) { return ((km[c >> 5] >> (c & 31)) & 1u) != 0u; };
       {
         uint32_t pk[32];

@@ -380,6 +380,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float ps[2] = {0.f, 0.f};
       uint32_t pk[64];
+      uint32_t km[4] = {0u, 0u, 0u, 0u};   // dropout keep bits of the 128 keys
+      if (DROP) {
+        keep_mask64(p, bh, i, j0, true, *reinterpret_cast<uint32_t(*)[2]>(km));
+        keep_mask64(p, bh, i, j0 + 64, true, *reinterpret_cast<uint32_t(*)[2]>(km + 2));
+      }
 #pragma unroll
       for (int w = 0; w < 64; ++w) {
         const float2 z = ffma2(make_float2(x[2 * w], x[2 * w + 1]), xs2, ms2);
@@ -392,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else ps2[w & 1] = fadd2(ps2[w & 1], e);
         if (DROP) {
           // PV sees P o M / (1 - p)
-          const uint32_t kb = keep_key_pair(p, bh, i, j0 + 2 * w);
+          const uint32_t kb = (km[w >> 4] >> (2 * (w & 15))) & 3u;
           pk[w] = DT<T>::pack((kb & 1u) ? e.x * p.drop_scale : 0.f, (kb & 2u) ? e.y * p.drop_scale : 0.f);
         }
       }

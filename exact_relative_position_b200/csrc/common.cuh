@@ -281,6 +281,42 @@ __device__ __forceinline__ uint32_t keep_query_pair(const Plan& p, int bh, int i
   return ((philox_word(w, jb) >> 8) >= p.drop_thresh ? 1u : 0u) |
          ((philox_word(w, 2 + jb) >> 8) >= p.drop_thresh ? 2u : 0u);
 }
+// Keep bits of 64 consecutive columns c0 .. c0 + 63 (c0 even) for this lane's
+// row, where lane l and lane l ^ 1 own rows 2k and 2k + 1 (row parity = lane
+// parity; the whole warp calls this).  Rows are queries with key columns
+// (row_is_query) or keys with query columns.  Each lane draws every other
+// 2 x 2 block and passes its partner the two words of the partner's row, so a
+// lane makes 16 generator calls for its 64 cells.  Bit c of km[c >> 5] keeps
+// column c0 + c.
+__device__ __forceinline__ void keep_mask64(const Plan& p, int bh, int row, int c0, bool row_is_query,
+                                            uint32_t (&km)[2]) {
+  const int par = row & 1;
+  km[0] = km[1] = 0u;
+#pragma unroll
+  for (int w2 = 0; w2 < 16; ++w2) {
+    const int wm = 2 * w2 + par;              // block this lane draws: columns c0 + 2 wm, + 1
+    const uint32_t col = (uint32_t)(c0 + 2 * wm);
+    const uint4 r = row_is_query
+                        ? philox4x32_10(col >> 1, (uint32_t)row >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi)
+                        : philox4x32_10((uint32_t)row >> 1, col >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
+    // block words: x (i even, j even), y (i even, j odd), z (i odd, j even), w (i odd, j odd);
+    // a row's two cells of the block, in column order, and the partner row's
+    uint32_t m0, m1, o0, o1;
+    if (row_is_query) {        // row = i, columns j
+      m0 = par ? r.z : r.x; m1 = par ? r.w : r.y;
+      o0 = par ? r.x : r.z; o1 = par ? r.y : r.w;
+    } else {                   // row = j, columns i
+      m0 = par ? r.y : r.x; m1 = par ? r.w : r.z;
+      o0 = par ? r.x : r.y; o1 = par ? r.z : r.w;
+    }
+    const uint32_t g0 = __shfl_xor_sync(0xFFFFFFFFu, o0, 1), g1 = __shfl_xor_sync(0xFFFFFFFFu, o1, 1);
+    const int wp = 2 * w2 + (par ^ 1);         // block the partner drew for this row
+    const uint32_t bm = ((m0 >> 8) >= p.drop_thresh ? 1u : 0u) | ((m1 >> 8) >= p.drop_thresh ? 2u : 0u);
+    const uint32_t bp = ((g0 >> 8) >= p.drop_thresh ? 1u : 0u) | ((g1 >> 8) >= p.drop_thresh ? 2u : 0u);
+    km[wm >> 4] |= bm << (2 * (wm & 15));
+    km[wp >> 4] |= bp << (2 * (wp & 15));
+  }
+}
 #endif
 
 }  // namespace relpos
