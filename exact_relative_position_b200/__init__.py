@@ -10,7 +10,7 @@ memory and streams only.
 from ._binding import (  # noqa: F401
     RelPosError, RelPosMap, check_workspace, debug_phi, debug_phi_device, debug_tile_plan, debug_tile_plan_device,
     expanded_bounds, kernel_launches, lib, profile_start, profile_stop, relpos_attn_bwd, relpos_attn_fwd,
-    table_rows, workspace_size,
+    sum_partials, table_rows, workspace_size,
 )
 
 import torch

@@ -54,7 +54,7 @@ EXPORTS = ["relpos_table_rows", "relpos_expanded_bounds", "relpos_workspace_size
            "relpos_attn_bwd", "relpos_status_string", "relpos_last_cuda_error", "relpos_debug_phi",
            "relpos_debug_phi_device", "relpos_debug_tile_plan", "relpos_debug_tile_plan_device",
            "relpos_profile_start", "relpos_profile_stop", "relpos_kernel_launches", "relpos_attn_fwd_noalloc",
-           "relpos_check_workspace"]
+           "relpos_check_workspace", "relpos_sum_partials"]
 
 
 def load_library(path: str = LIBPATH) -> ctypes.CDLL:
@@ -82,6 +82,7 @@ def load_library(path: str = LIBPATH) -> ctypes.CDLL:
     sig["relpos_kernel_launches"] = []
     sig["relpos_attn_fwd_noalloc"] = [P(relpos_fwd_args), ctypes.c_void_p]
     sig["relpos_check_workspace"] = [ctypes.c_void_p, ctypes.c_void_p, P(ctypes.c_int32)]
+    sig["relpos_sum_partials"] = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -333,3 +334,19 @@ def check_workspace(workspace) -> int:
     _check(lib().relpos_check_workspace(workspace.data_ptr(), _stream(workspace.device), ctypes.byref(st)),
            "relpos_check_workspace")
     return st.value
+
+
+def sum_partials(partials: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """relpos_sum_partials: partials [world, n] fp32 CUDA (contiguous) -> [n], the
+    rows added in ascending order.  out may be partials[0] or a separate [n] buffer."""
+    if partials.device.type != "cuda" or partials.dtype != torch.float32 or partials.dim() != 2 \
+            or not partials.is_contiguous():
+        raise ValueError("partials must be a contiguous [world, n] float32 CUDA tensor")
+    world, n = partials.shape
+    if out is None:
+        out = torch.empty(n, device=partials.device, dtype=torch.float32)
+    if out.device != partials.device or out.dtype != torch.float32 or out.numel() != n or not out.is_contiguous():
+        raise ValueError("out must be a contiguous float32 tensor of n entries on the partials' device")
+    _check(lib().relpos_sum_partials(partials.data_ptr(), world, n, out.data_ptr(), _stream(partials.device)),
+           "relpos_sum_partials")
+    return out

@@ -549,6 +549,40 @@ RELPOS_EXPORT int relpos_profile_stop(relpos_phase_stat* stats, int32_t max_stat
 
 RELPOS_EXPORT int64_t relpos_kernel_launches(void) { return g_kernel_launches.load(); }
 
+// ---------------------------------------------------------------- data-parallel exchange
+namespace relpos {
+namespace {
+// out[i] = ((p[0][i] + p[1][i]) + p[2][i]) + ... : one thread per entry, rows
+// added in ascending order, so the bits do not depend on the launch shape.
+// out may be row 0 of p (each entry is read before it is written).
+__global__ void sum_partials_kernel(const float* p, int world, long long n, float* out) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    float acc = p[i];
+    for (int r = 1; r < world; ++r) acc = __fadd_rn(acc, p[(long long)r * n + i]);
+    out[i] = acc;
+  }
+}
+}  // namespace
+}  // namespace relpos
+
+RELPOS_EXPORT int relpos_sum_partials(const float* partials, int32_t world, int64_t n, float* out,
+                                      relpos_stream_t stream) {
+  using namespace relpos;
+  if (world < 1 || n < 0) return RELPOS_ERR_INVALID_ARG;
+  if (n == 0) return RELPOS_OK;
+  if (!partials || !out || (reinterpret_cast<uintptr_t>(partials) & 3) || (reinterpret_cast<uintptr_t>(out) & 3))
+    return RELPOS_ERR_INVALID_ARG;
+  // out is row 0 or lies outside rows 1 .. world - 1
+  const float* rows_end = partials + (long long)world * n;
+  if (out != partials && out + n > partials && out < rows_end) return RELPOS_ERR_INVALID_ARG;
+  const long long blocks = (n + 255) / 256;
+  const int grid = (int)(blocks < 148 * 8 ? blocks : 148 * 8);
+  sum_partials_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(partials, world, n, out);
+  note_launch(1);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RELPOS_OK : cuda_fail(e);
+}
+
 RELPOS_EXPORT int relpos_debug_phi(const relpos_map_desc* map, int32_t N, int32_t* phi_host) {
   if (!map || !phi_host || N < 1 || N > 46340) return RELPOS_ERR_INVALID_ARG;
   const int st = check_map(map);

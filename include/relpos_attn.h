@@ -234,6 +234,24 @@ int relpos_profile_stop(relpos_phase_stat* stats, int32_t max_stats, int32_t* n_
 /* Number of kernels this library has launched in this process so far. */
 int64_t relpos_kernel_launches(void);
 
+/* --- data-parallel exchange -------------------------------------------- */
+
+/* Ascending-rank sum of per-rank partial table gradients.
+ * The gradient of a table shared across the batch is a sum over every cell
+ * that reads it (digest: Eq. (4)), so when the batch is split over ranks each
+ * rank's relpos_attn_bwd leaves the partial sum of its own batch elements in
+ * daq / dak / db.  After an all-gather puts the partials in rank order, this
+ * call adds them in that order, out[i] = ((p[0][i] + p[1][i]) + p[2][i]) + ...,
+ * in fp32 with round-to-nearest adds, so every rank obtains the same bits.
+ *  partials: device fp32 [world][n] (row r = rank r's partial, rows contiguous),
+ *            4-byte aligned.  Not written unless out is its row 0.
+ *  out:      device fp32 [n]; either partials itself (row 0) or a range that
+ *            overlaps none of the rows.
+ *  world >= 1; n >= 0 (n = 0: returns RELPOS_OK without a launch).
+ *  Asynchronous on stream.  Errors: INVALID_ARG (world < 1, n < 0, null or
+ *  misaligned pointer, overlapping out), CUDA. */
+int relpos_sum_partials(const float* partials, int32_t world, int64_t n, float* out, relpos_stream_t stream);
+
 /* --- parity exports (used by the tests) --------------------------------- */
 
 /* phi(i, j) for all N x N cells computed on the host. phi_host: host [N*N] int32. */
