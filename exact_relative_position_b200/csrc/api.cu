@@ -84,29 +84,34 @@ struct PairTimer {
   }
 };
 
-// A second stream per device, created once (non-blocking, never destroyed).
-// A fork records an event on the caller's stream and makes the side stream
-// wait for it; join does the reverse, so work issued on the side stream in
-// between is ordered before anything the caller issues afterwards (also under
-// stream capture).  If the side stream or the events cannot be created the
-// fork degrades to the caller's stream alone.
-cudaStream_t side_stream() {
+// Extra streams per device, created once (non-blocking, never destroyed):
+// 0 carries the K-parallel backward pass, 1 and 2 the relation-gradient row
+// updates of the query and the key side.  A fork records an event on the
+// caller's stream and makes the side stream wait for it; join does the
+// reverse, so work issued on the side stream in between is ordered before
+// anything the caller issues afterwards (also under stream capture).  If the
+// side stream or the events cannot be created the fork degrades to the
+// caller's stream alone.
+constexpr int kSideStreams = 3;
+cudaStream_t side_stream(int which) {
   static std::mutex mu;
-  static cudaStream_t streams[64] = {};
+  static cudaStream_t streams[64][kSideStreams] = {};
   int dev = 0;
+  if (which < 0 || which >= kSideStreams) return nullptr;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
-  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+  cudaStream_t& st = streams[dev][which];
+  if (!st && cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) {
     cudaGetLastError();
-    streams[dev] = nullptr;
+    st = nullptr;
   }
-  return streams[dev];
+  return st;
 }
 
 class Fork {
  public:
-  explicit Fork(cudaStream_t s) : s_(s), side_(s) {
-    cudaStream_t s2 = side_stream();
+  explicit Fork(cudaStream_t s, int which = 0) : s_(s), side_(s) {
+    cudaStream_t s2 = side_stream(which);
     if (!s2 || cudaEventCreateWithFlags(&fork_, cudaEventDisableTiming) != cudaSuccess) return;
     if (cudaEventCreateWithFlags(&join_, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventRecord(fork_, s) != cudaSuccess || cudaStreamWaitEvent(s2, fork_, 0) != cudaSuccess) {
@@ -465,8 +470,17 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   e2 = run_phase(PH_DKDV, s2, [&] { return launch_bwd_dkdv(p, t, s2); });
   pair.end_second(s2);
   pair.commit(2);
-  if (terms && e == cudaSuccess) e = run_phase(PH_RELGRAD, s, [&] { return launch_relgrad(p, t, 0, s); });
-  if (a->ak && e2 == cudaSuccess) e2 = run_phase(PH_RELGRAD, s2, [&] { return launch_relgrad(p, t, 1, s2); });
+  // each side's dQ / dK row update runs beside its table-gradient kernels
+  auto relgrad = [&](int side, cudaStream_t st) {
+    return run_phase(PH_RELGRAD, st, [&] {
+      Fork aux(st, 1 + side);
+      const cudaError_t el = launch_relgrad(p, t, side, st, aux.side());
+      const cudaError_t ea = aux.join();
+      return el != cudaSuccess ? el : ea;
+    });
+  };
+  if (terms && e == cudaSuccess) e = relgrad(0, s);
+  if (a->ak && e2 == cudaSuccess) e2 = relgrad(1, s2);
   const cudaError_t ej = fork.join();
   if (e != cudaSuccess) return cuda_fail(e);
   if (e2 != cudaSuccess) return cuda_fail(e2);

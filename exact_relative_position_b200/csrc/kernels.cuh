@@ -64,8 +64,10 @@ cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dkdv(const Plan& p, const Tensors& t, cudaStream_t s);
 // side 0: query-side relation gradients (dQ += dZ^Q aQ_exp, daQ, db);
-// side 1: key side (dK += dZ^K aK_exp, daK)
-cudaError_t launch_relgrad(const Plan& p, const Tensors& t, int side, cudaStream_t s);
+// side 1: key side (dK += dZ^K aK_exp, daK).  The dQ / dK row update goes to
+// rows_stream and the table gradients to s (the two share no outputs); the
+// caller orders rows_stream after s's earlier work and joins it back.
+cudaError_t launch_relgrad(const Plan& p, const Tensors& t, int side, cudaStream_t s, cudaStream_t rows_stream);
 cudaError_t launch_debug_phi(const relpos_map_desc& map, int N, int* out, cudaStream_t s);
 cudaError_t launch_debug_tile_plan(int B, int N, int causal, const int* key_len, int E_lo, int E_hi,
                                    int* classes, int* segs, cudaStream_t s);

@@ -604,7 +604,7 @@ cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s) {
 
 // side 0: the query side (aQ rows, aQ table, bias); side 1: the key side (aK).
 template <typename T>
-static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cudaStream_t s) {
+static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cudaStream_t s, cudaStream_t sr) {
   const int Hq = t.table_per_head ? p.H : 1;
   const int nE = (p.Rexp + tp::kEB - 1) / tp::kEB;
   constexpr uint32_t kRowsSmem = rg::kStages * rg::stage_bytes<T>();
@@ -614,7 +614,7 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cuda
     e = cudaFuncSetAttribute(table_part_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPartSmem);
   if (e != cudaSuccess) return e;
   if (side == 0 && t.aq_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
                                                                         t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
     { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
                                                                            t.table_per_head, t.nsplit_q, t.daq_part); note_launch(1); }
@@ -622,7 +622,7 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cuda
                                                                      t.fold_lo, t.fold_hi, t.daq); note_launch(1); }
   }
   if (side == 1 && t.ak_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
                                                                         t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
     { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
                                                                            t.table_per_head, t.nsplit_k, t.dak_part); note_launch(1); }
@@ -637,8 +637,9 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cuda
   return cudaGetLastError();
 }
 
-cudaError_t launch_relgrad(const Plan& p, const Tensors& t, int side, cudaStream_t s) {
-  return t.is_bf16 ? relgrad_typed<__nv_bfloat16>(p, t, side, s) : relgrad_typed<__half>(p, t, side, s);
+cudaError_t launch_relgrad(const Plan& p, const Tensors& t, int side, cudaStream_t s, cudaStream_t rows_stream) {
+  return t.is_bf16 ? relgrad_typed<__nv_bfloat16>(p, t, side, s, rows_stream)
+                   : relgrad_typed<__half>(p, t, side, s, rows_stream);
 }
 
 cudaError_t launch_debug_phi(const relpos_map_desc& map, int N, int* out, cudaStream_t s) {

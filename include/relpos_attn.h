@@ -211,7 +211,9 @@ int relpos_attn_fwd_noalloc(const relpos_fwd_args* a, relpos_stream_t stream);
  * "bwd_attention".  The backward runs its Q-parallel pass (then the query-side
  * relation gradients) on the caller's stream and its K-parallel pass (then the
  * key side) concurrently on a second stream, so "bwd_dkdv" and the key-side
- * "relation_grads" are measured on that stream and overlap other phases;
+ * "relation_grads" are measured on that stream and overlap other phases.
+ * Each side's dQ / dK row update runs on a further stream of its own, joined
+ * back inside its "relation_grads" phase;
  * "bwd_attention" spans both passes, from the start of the first to the end
  * of the later one. */
 typedef struct {
