@@ -92,12 +92,15 @@ struct PairTimer {
 // anything the caller issues afterwards (also under stream capture).  If the
 // side stream or the events cannot be created the fork degrades to the
 // caller's stream alone.
+// A thread that sets single-stream mode gets no side stream: its forks
+// degrade to the caller's stream and create no streams or events.
 constexpr int kSideStreams = 3;
+thread_local bool g_single_stream = false;
 cudaStream_t side_stream(int which) {
   static std::mutex mu;
   static cudaStream_t streams[64][kSideStreams] = {};
   int dev = 0;
-  if (which < 0 || which >= kSideStreams) return nullptr;
+  if (g_single_stream || which < 0 || which >= kSideStreams) return nullptr;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
   cudaStream_t& st = streams[dev][which];
@@ -349,10 +352,13 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
   });
   if (e != cudaSuccess) return cuda_fail(e);
   if (a->aq || a->ak) {
+    // Z^Q on the caller's stream, Z^K and its saturated columns beside it
     e = run_phase(PH_PROJ, s, [&] {
-      cudaError_t e1 = launch_projection(p, t, s);
-      if (e1 == cudaSuccess && a->ak) e1 = launch_saturated_columns(p, t, s);
-      return e1;
+      Fork aux(s, 1);
+      cudaError_t e1 = launch_projection(p, t, s, aux.side());
+      if (e1 == cudaSuccess && a->ak) e1 = launch_saturated_columns(p, t, aux.side());
+      const cudaError_t ej = aux.join();
+      return e1 != cudaSuccess ? e1 : ej;
     });
     if (e != cudaSuccess) return cuda_fail(e);
   }
@@ -360,6 +366,10 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
 }
 
 }  // namespace
+
+namespace relpos {
+void set_single_stream(bool on) { g_single_stream = on; }
+}  // namespace relpos
 
 RELPOS_EXPORT int relpos_table_rows(const relpos_map_desc* map, int32_t N, int32_t* R_out) {
   if (!map || !R_out || N < 1 || N > kMaxN) return RELPOS_ERR_INVALID_ARG;

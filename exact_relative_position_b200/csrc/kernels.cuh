@@ -42,6 +42,9 @@ struct Tensors {
 };
 
 // Records e as this thread's last CUDA error and returns RELPOS_ERR_CUDA.
+// Thread-local: while on, the library issues everything on the caller's stream
+// (no side streams or events are created).
+void set_single_stream(bool on);
 int cuda_status(cudaError_t e);
 
 // Counts kernel launches (process-wide, reported by relpos_kernel_launches).
@@ -52,7 +55,7 @@ cudaError_t launch_build_tables(const Plan& p, const relpos_map_desc& map, Group
                                 void* aq_exp, void* ak_exp, const float* b, float* b_exp, int is_bf16,
                                 int expand_tables, cudaStream_t s);
 cudaError_t launch_fold_ranges(const Plan& p, const int* phi_exp, int R, int* fold_lo, int* fold_hi, cudaStream_t s);
-cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s);
+cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s, cudaStream_t key_stream);
 cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t s);
 

@@ -55,5 +55,9 @@ RELPOS_EXPORT int relpos_attn_fwd_noalloc(const relpos_fwd_args* a, relpos_strea
   void* ws = nullptr;
   const int e = scratch_for_current_device(&ws);
   if (e) return relpos::cuda_status((cudaError_t)e);
-  return relpos_attn_fwd(a, ws, kScratchBytes, stream);
+  // the caller's stream only: forks would create events (and a stream on first use)
+  relpos::set_single_stream(true);
+  const int st2 = relpos_attn_fwd(a, ws, kScratchBytes, stream);
+  relpos::set_single_stream(false);
+  return st2;
 }

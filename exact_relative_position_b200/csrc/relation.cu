@@ -562,7 +562,7 @@ cudaError_t launch_fold_ranges(const Plan& p, const int* phi_exp, int R, int* fo
 }
 
 template <typename T>
-static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
+static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_t s, cudaStream_t sk) {
   cudaError_t e = cudaFuncSetAttribute(projection_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kProjSmem);
   if (e != cudaSuccess) return e;
   // widest group decides the chunk count; narrower groups exit early
@@ -576,7 +576,7 @@ static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_
   }
   if (t.zk && t.ak_exp) {
     dim3 grid((wk + 63) / 64, p.nT, p.B * p.H);
-    { projection_kernel<T><<<grid, 256, kProjSmem, s>>>(p, 1, (const T*)t.k, (const T*)t.ak_exp,
+    { projection_kernel<T><<<grid, 256, kProjSmem, sk>>>(p, 1, (const T*)t.k, (const T*)t.ak_exp,
                                                       t.table_per_head ? t.ak_hs : 0, t.zk, p.zk_head); note_launch(1); }
   }
   return cudaGetLastError();
@@ -598,8 +598,8 @@ cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s) {
-  return t.is_bf16 ? projection_typed<__nv_bfloat16>(p, t, s) : projection_typed<__half>(p, t, s);
+cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s, cudaStream_t key_stream) {
+  return t.is_bf16 ? projection_typed<__nv_bfloat16>(p, t, s, key_stream) : projection_typed<__half>(p, t, s, key_stream);
 }
 
 // side 0: the query side (aQ rows, aQ table, bias); side 1: the key side (aK).
