@@ -262,15 +262,39 @@ def run_sweep(args):
             ws = torch.empty(max(fws, bws), device=dev, dtype=torch.uint8)
             steps = args.sweep_steps
             ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+
+            def fwd():
+                rp.relpos_attn_fwd(q, k, v, aq, ak, b, tau=w.tau, map=m, workspace=ws, o=o, lse=lse)
+
+            def bwd():
+                rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, tau=w.tau, map=m, workspace=ws, grads=grads,
+                                   reuse_forward=True)
+
+            graphs = []
+            if args.graph:
+                # one eager pass on a side stream, then each pass captured once;
+                # a replay re-runs every kernel of the pass on the same buffers
+                side = torch.cuda.Stream(dev)
+                side.wait_stream(torch.cuda.current_stream(dev))
+                with torch.cuda.stream(side):
+                    fwd()
+                    bwd()
+                torch.cuda.current_stream(dev).wait_stream(side)
+                torch.cuda.synchronize()
+                graphs = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+                with torch.cuda.graph(graphs[0]):
+                    fwd()
+                with torch.cuda.graph(graphs[1]):
+                    bwd()
+                fwd, bwd = graphs[0].replay, graphs[1].replay
             for s in range(args.warmup + steps):
                 flush.zero_()
                 if s >= args.warmup:
                     ev[s - args.warmup][0].record()
-                rp.relpos_attn_fwd(q, k, v, aq, ak, b, tau=w.tau, map=m, workspace=ws, o=o, lse=lse)
+                fwd()
                 if s >= args.warmup:
                     ev[s - args.warmup][1].record()
-                rp.relpos_attn_bwd(do, q, k, v, o, lse, aq, ak, b, tau=w.tau, map=m, workspace=ws, grads=grads,
-                                   reuse_forward=True)
+                bwd()
                 if s >= args.warmup:
                     ev[s - args.warmup][2].record()
             torch.cuda.synchronize()
@@ -284,7 +308,9 @@ def run_sweep(args):
                 "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
                 "fwd_frac_of_peak": fwd_flops / (fwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                 "bwd_frac_of_peak": bwd_flops / (bwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-                "workspace_bytes": int(ws.numel()), "l2": "flushed before every step"}), flush=True)
+                "workspace_bytes": int(ws.numel()), "l2": "flushed before every step",
+                "launch": "cuda graph replay" if args.graph else "eager calls"}), flush=True)
+            del graphs, fwd, bwd
             del q, k, v, do, aq, ak, b, o, lse, grads, ws
             torch.cuda.empty_cache()
 
@@ -305,6 +331,9 @@ def main():
     ap.add_argument("--sweep-mechanisms", default="", help="comma list (default: all four)")
     ap.add_argument("--sweep-lengths", default="", help="comma list of N (default: 128 ... 8192)")
     ap.add_argument("--sweep-steps", type=int, default=10)
+    ap.add_argument("--graph", action="store_true",
+                    help="with --sweep: capture each point's forward and backward once as CUDA graphs and time "
+                         "their replays (the short-N points are launch-bound when called eagerly)")
     ap.add_argument("--ncu", action="store_true",
                     help="one forward + backward only (for an ncu capture of each kernel's first launch)")
     args = ap.parse_args()
