@@ -34,6 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "shaw_clip64_n8192"
+METRIC = "useful TFLOP/s of one rel-pos attention layer (fwd+bwd), 8K x 12h x d64 fp16"
 
 
 def useful_flops(w, R_exp):
@@ -220,11 +221,12 @@ def run_reference(args, rank, world):
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     sample = (f"fp64 oracle forward+backward of one block of {block} query rows of head 0 against all {w.N} keys "
               f"per step")
-    line = {"impl": "reference", "metric": "useful TFLOP/s of one rel-pos attention layer (fwd+bwd)",
+    line = {"impl": "reference", "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, **{k_: v_ for k_, v_ in w.describe().items() if k_ != "workload"}},
+            "config": {"workload": WORKLOAD, **{k_: v_ for k_, v_ in w.describe().items() if k_ != "workload"},
+                       "R_exp": R_exp, "dropout": 0.0, "parallelism": "host oracle on rank 0"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -518,7 +520,7 @@ def main():
         ms = t_step / args.steps
         value = step_flops / (ms * 1e-3) / 1e12
         line = {
-            "metric": "useful TFLOP/s of one rel-pos attention layer (fwd+bwd), 8K x 12h x d64 fp16",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp16" if w.dtype == torch.float16 else "bf16", "data": "synthetic",
