@@ -48,11 +48,17 @@ def useful_flops(w, R_exp):
 
 
 def kernel_flops(w):
-    """Tensor-core FLOPs each attention kernel's algorithm performs per launch."""
+    """Per launch of each attention phase: (algorithmic, executed) tensor FLOPs.
+
+    Algorithmic is the useful work of the FlashAttention convention: forward
+    QK^T and PV (4 B H N^2 d), backward the five GEMMs S, dP, dV, dK and dQ
+    (10 B H N^2 d); causal halves both.  Executed adds what the two-pass
+    backward recomputes: each pass forms S and dP itself (7 GEMMs)."""
     cf = 0.5 if w.causal else 1.0
     base = 2.0 * w.B * w.H * w.N * w.N * w.d * cf    # one N x N x d GEMM
     # the two backward passes run concurrently (two streams): timed together
-    return {"fwd_attention": 2 * base, "bwd_attention": 7 * base}
+    return ({"fwd_attention": 2 * base, "bwd_attention": 5 * base},
+            {"fwd_attention": 2 * base, "bwd_attention": 7 * base})
 
 
 def load_peaks():
@@ -503,7 +509,7 @@ def main():
 
     if rank == 0:
         peaks = load_peaks()
-        kf = kernel_flops(w)
+        kf, kx = kernel_flops(w)
         cand = {ph: v for ph, v in phases.items() if ph in kf}
         dom = max(cand, key=lambda ph: cand[ph][2]) if cand else None
         roof = None
@@ -515,7 +521,13 @@ def main():
             roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": tr,
                     "peak_source": f"{peaks['source']} dense bf16 (burst); fp16 has the same nominal rate",
-                    "avg_launch_ms": avg_ms, "algorithmic_flops_per_launch": kf[dom]}
+                    "avg_launch_ms": avg_ms, "algorithmic_flops_per_launch": kf[dom],
+                    "executed_flops_per_launch": kx[dom],
+                    "executed_tflops": kx[dom] / (avg_ms * 1e-3) / 1e12,
+                    "phases": {ph: {"avg_launch_ms": cand[ph][2] / max(cand[ph][0], 1),
+                                    "achieved_tflops": kf[ph] / (cand[ph][2] / max(cand[ph][0], 1) * 1e-3) / 1e12,
+                                    "frac": kf[ph] / (cand[ph][2] / max(cand[ph][0], 1) * 1e-3) / 1e12
+                                            / peaks["bf16_tflops"]} for ph in cand}}
         step_flops = (fwd_flops + bwd_flops) * world
         ms = t_step / args.steps
         value = step_flops / (ms * 1e-3) / 1e12

@@ -45,6 +45,18 @@ class relpos_bwd_args(ctypes.Structure):
                 ("dak", ctypes.c_void_p), ("db", ctypes.c_void_p), ("reuse_forward_workspace", ctypes.c_int32)]
 
 
+class relpos_group_info(ctypes.Structure):
+    _fields_ = [("e0", ctypes.c_int32), ("W", ctypes.c_int32), ("S", ctypes.c_int32), ("pad", ctypes.c_int32),
+                ("base", ctypes.c_int64)]
+
+
+class relpos_projection_layout(ctypes.Structure):
+    _fields_ = [("E_lo", ctypes.c_int32), ("E_hi", ctypes.c_int32), ("R_exp", ctypes.c_int32),
+                ("nT", ctypes.c_int32), ("grouped", ctypes.c_int32), ("pad", ctypes.c_int32),
+                ("zq_offset", ctypes.c_int64), ("zk_offset", ctypes.c_int64), ("zq_head", ctypes.c_int64),
+                ("zk_head", ctypes.c_int64), ("gq_offset", ctypes.c_int64), ("gk_offset", ctypes.c_int64)]
+
+
 class relpos_phase_stat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("calls", ctypes.c_int32), ("kernels", ctypes.c_int32),
                 ("total_ms", ctypes.c_float)]
@@ -54,7 +66,8 @@ EXPORTS = ["relpos_table_rows", "relpos_expanded_bounds", "relpos_workspace_size
            "relpos_attn_bwd", "relpos_status_string", "relpos_last_cuda_error", "relpos_debug_phi",
            "relpos_debug_phi_device", "relpos_debug_tile_plan", "relpos_debug_tile_plan_device",
            "relpos_profile_start", "relpos_profile_stop", "relpos_kernel_launches", "relpos_attn_fwd_noalloc",
-           "relpos_check_workspace", "relpos_sum_partials"]
+           "relpos_check_workspace", "relpos_sum_partials", "relpos_check_noalloc", "relpos_debug_projection",
+           "relpos_set_wait_limit_ns"]
 
 
 def load_library(path: str = LIBPATH) -> ctypes.CDLL:
@@ -83,6 +96,10 @@ def load_library(path: str = LIBPATH) -> ctypes.CDLL:
     sig["relpos_attn_fwd_noalloc"] = [P(relpos_fwd_args), ctypes.c_void_p]
     sig["relpos_check_workspace"] = [ctypes.c_void_p, ctypes.c_void_p, P(ctypes.c_int32)]
     sig["relpos_sum_partials"] = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    sig["relpos_check_noalloc"] = [ctypes.c_void_p, P(ctypes.c_int32)]
+    sig["relpos_debug_projection"] = [P(relpos_fwd_args), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                      P(relpos_projection_layout)]
+    sig["relpos_set_wait_limit_ns"] = [ctypes.c_uint64]
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -325,6 +342,47 @@ def relpos_attn_fwd_noalloc(q, k, v, aq=None, ak=None, b=None, *, tau: float, ma
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse)
     _check(lib().relpos_attn_fwd_noalloc(ctypes.byref(a), _stream(q.device)), "relpos_attn_fwd_noalloc")
     return o, lse
+
+
+def check_noalloc(device=None) -> int:
+    """Synchronises the current stream and returns the device status word of the
+    last relpos_attn_fwd_noalloc on this device (0 = ok); raises RelPosError on a
+    timeout."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_int32()
+    _check(lib().relpos_check_noalloc(_stream(dev), ctypes.byref(st)), "relpos_check_noalloc")
+    return st.value
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Limit of the fused kernels' bounded waits for later launches (0 = the
+    default 2 s).  Only for tests of the timeout path."""
+    _check(lib().relpos_set_wait_limit_ns(int(ns)), "relpos_set_wait_limit_ns")
+
+
+def debug_projection(q, k, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap, causal: bool = False,
+                     key_len=None):
+    """relpos_debug_projection: runs the table expansion and the projections only.
+
+    Returns (layout, workspace, groups_q, groups_k): the layout record, the
+    workspace tensor holding Z^Q / Z^K at the recorded offsets, and the group
+    records of each side as [nT, 4] int32 (e0, W, S, pad) plus [nT] int64 bases."""
+    if key_len is not None:
+        key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
+    a = _fwd_args(q, k, q, aq, ak, b, tau, map, causal, key_len, False)
+    f, bw = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
+    ws = torch.zeros(max(f.value, 256), device=q.device, dtype=torch.uint8)
+    lay = relpos_projection_layout()
+    _check(lib().relpos_debug_projection(ctypes.byref(a), ws.data_ptr(), ws.numel(), _stream(q.device),
+                                         ctypes.byref(lay)), "relpos_debug_projection")
+
+    def groups(off):
+        raw = ws[off:off + 24 * lay.nT].cpu()
+        ints = raw.view(torch.int32).reshape(lay.nT, 6)
+        return ints[:, :4].clone(), raw.view(torch.int64).reshape(lay.nT, 3)[:, 2].clone()
+
+    return lay, ws, groups(lay.gq_offset), groups(lay.gk_offset)
 
 
 def check_workspace(workspace) -> int:

@@ -8,6 +8,7 @@
 // Backward (two-pass backward, Eq. (4)):
 //   tables -> projection -> D -> Q-parallel pass (dQ, dZ^Q) -> K-parallel pass
 //   (dK, dV, dZ^K) -> relation GEMMs, split sums and bucket fold.
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -17,6 +18,7 @@
 #include <vector>
 
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 #define RELPOS_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -151,6 +153,10 @@ int cuda_fail(cudaError_t e) {
 
 constexpr int kMaxN = 1 << 22;
 
+// Limit of the fused kernels' bounded waits for launches planned from now on
+// (0: the built-in 2 s).  Process-wide; only tests lower it.
+std::atomic<unsigned long long> g_wait_limit_ns{0};
+
 int check_map(const relpos_map_desc* m) {
   if (!m) return RELPOS_ERR_INVALID_ARG;
   switch (m->kind) {
@@ -242,6 +248,10 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   p->seed_lo = (uint32_t)(a->dropout_seed & 0xFFFFFFFFull);
   p->seed_hi = (uint32_t)(a->dropout_seed >> 32);
   p->drop_offset = a->dropout_offset;
+  {
+    const unsigned long long lim = g_wait_limit_ns.load();
+    p->wait_ns = lim ? lim : (unsigned long long)sm100::kTimeoutNs;
+  }
   const bool aq = a->aq != nullptr, ak = a->ak != nullptr, bb = a->b != nullptr;
   const long long zq_head = head_elems(*p, 0), zk_head = head_elems(*p, 1);
   p->zq_head = (aq || bb) ? zq_head : 0;
@@ -498,6 +508,47 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   return RELPOS_OK;
 }
 
+static_assert(sizeof(relpos_group_info) == sizeof(GroupInfo), "relpos_group_info mirrors GroupInfo");
+static_assert(offsetof(relpos_group_info, base) == offsetof(GroupInfo, base), "relpos_group_info mirrors GroupInfo");
+
+RELPOS_EXPORT int relpos_debug_projection(const relpos_fwd_args* a, void* workspace, size_t ws_bytes,
+                                          relpos_stream_t stream, relpos_projection_layout* layout) {
+  Plan p;
+  Layout L;
+  int st = make_plan(a, &p, &L);
+  if (st) return st;
+  if (!layout || !a->q || !a->k) return RELPOS_ERR_INVALID_ARG;
+  if ((a->mask & RELPOS_MASK_KEY_PADDING) && !a->key_len) return RELPOS_ERR_INVALID_ARG;
+  const void* al[] = {a->q, a->k, a->aq, a->ak};
+  for (const void* x : al)
+    if (x && !aligned16(x)) return RELPOS_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < L.fwd_end || (reinterpret_cast<uintptr_t>(workspace) & 255)) return RELPOS_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Tensors t;
+  st = prepare(a, p, L, static_cast<uint8_t*>(workspace), t, s);
+  if (st) return st;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  layout->E_lo = p.E_lo;
+  layout->E_hi = p.E_hi;
+  layout->R_exp = p.Rexp;
+  layout->nT = p.nT;
+  layout->grouped = p.grouped;
+  layout->pad = 0;
+  layout->zq_offset = a->aq ? (int64_t)L.zq : -1;
+  layout->zk_offset = a->ak ? (int64_t)L.zk : -1;
+  layout->zq_head = a->aq ? p.zq_head : 0;
+  layout->zk_head = a->ak ? p.zk_head : 0;
+  layout->gq_offset = (int64_t)L.gq;
+  layout->gk_offset = (int64_t)L.gk;
+  return RELPOS_OK;
+}
+
+RELPOS_EXPORT int relpos_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store((unsigned long long)ns);
+  return RELPOS_OK;
+}
+
 RELPOS_EXPORT const char* relpos_status_string(int status) {
   switch (status) {
     case RELPOS_OK: return "ok";
@@ -640,7 +691,7 @@ RELPOS_EXPORT int relpos_debug_tile_plan(const relpos_map_desc* map, int32_t B, 
   const int nT = (N + kTile - 1) / kTile;
   const int causal = (mask & RELPOS_MASK_CAUSAL) != 0;
   for (int b = 0; b < B; ++b) {
-    const int nkv = (mask & RELPOS_MASK_KEY_PADDING) ? key_len_host[b] : N;
+    const int nkv = (mask & RELPOS_MASK_KEY_PADDING) ? iclamp(key_len_host[b], 0, N) : N;
     for (int qi = 0; qi < nT; ++qi) {
       for (int kj = 0; kj < nT; ++kj)
         classes_host[((size_t)b * nT + qi) * nT + kj] = tile_class(qi, kj, N, nkv, causal, lo, hi);

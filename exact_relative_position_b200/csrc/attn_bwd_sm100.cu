@@ -15,12 +15,12 @@
 //                gradient by offset in the same single-writer way.
 // No gradient entry has two writers: no atomics, fixed summation order.
 //
-// Pipelining (both passes): the score GEMM of tile t+2 and the dP GEMM of
-// tile t+1 are issued while the compute warps work on tile t, with two score
-// buffers and one dP buffer in tensor memory.  Compute threads own one row of
-// the tile (its tensor-memory lane) and write the 16-bit P / dS operands of
-// the next GEMMs into 128-byte-swizzled shared-memory tiles.  Every mbarrier
-// wait is bounded (see sm100.cuh).
+// Pipelining (both passes): the score and dP GEMMs of tile t+1 are issued as
+// soon as the compute warps have read tile t's S and dP out of tensor memory.
+// Two compute warps share each row of the tile (its tensor-memory lane), one
+// per 64-column half, and write the 16-bit P / dS operands of the next GEMMs
+// back into tensor memory, where the TS-form GEMMs read them as their A
+// operand.  Every mbarrier wait is bounded (see sm100.cuh).
 #include <cudaTypedefs.h>
 
 #include "band.cuh"
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
   const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, q0 = qt * kT;
   const int npad = p.nT * kT;
-  const int nkv = p.padding ? p.key_len[b] : N;
+  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
   int kend = nkv;
   if (p.causal) kend = imin(kend, imin(q0 + kT, N));
   const int nkt = kend > 0 ? (kend + kT - 1) / kT : 0;
@@ -174,10 +174,11 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
         tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
         tma_load_3d(sb + kOffDO, &tmDO, bar(kBarQ), 0, q0, bh);
+        int issued = 0;
   #pragma unroll 1
         for (int it = 0; it < nkt; ++it) {
           const int s = it % kStages;
-          if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+          if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag, p.wait_ns)) break;
           const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
           mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
           tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kT, bh);
@@ -187,7 +188,12 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
             bulk_load(dst + 2 * kTileBytes, src, kT * 4, bar(kBarKvFull + s));
             bulk_load(dst + 2 * kTileBytes + kT * 4, src + npad, kT * 4, bar(kBarKvFull + s));
           }
+          issued = it + 1;
         }
+        // no load may still be landing when the CTA exits (see the forward)
+        mbar_drain(bar(kBarQ), 0);
+        for (int it = imax(0, issued - kStages); it < issued; ++it)
+          mbar_drain(bar(kBarKvFull + it % kStages), (it / kStages) & 1);
       }
     } else if (warp == 1) {
       if (lane == 0 && nkt > 0) {
@@ -220,7 +226,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
   #pragma unroll 1
           for (int kk = 0; kk < 8; ++kk) mma_ts(tmem + kTmDQ, a + 8 * kk, kd + 128 * kk, id_dq, (acc || kk > 0) ? 1u : 0u);
         };
-        bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
+        bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.wait_ns) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag, p.wait_ns);
         if (ok) {
           tc_fence_after();
           issue_s(0);
@@ -232,26 +238,27 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         for (int it = 0; it < nkt && ok; ++it) {
           const int s = it % kStages, s1 = (it + 1) % kStages;
           if (it + 1 < nkt) {
-            ok = mbar_wait(bar(kBarKvFull + s1), ((it + 1) / kStages) & 1, abort_flag) &&
-                 mbar_wait(bar(kBarSFree), it & 1, abort_flag);
+            ok = mbar_wait(bar(kBarKvFull + s1), ((it + 1) / kStages) & 1, abort_flag, p.wait_ns) &&
+                 mbar_wait(bar(kBarSFree), it & 1, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
             issue_s(s1);
             mma_commit(bar(kBarSFull));
-            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
             issue_dp(s1);
             mma_commit(bar(kBarDpFull));
           }
-          ok = mbar_wait(bar(kBarDsReady + (it & 1)), (it >> 1) & 1, abort_flag);
+          ok = mbar_wait(bar(kBarDsReady + (it & 1)), (it >> 1) & 1, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_dq(s, it & 1, it > 0);
           mma_commit(bar(kBarDsFree + (it & 1)));
           mma_commit(bar(kBarKvEmpty + s));
         }
-        if (!ok) {
+        {
+          // drain (bounded): no MMA may still run when tensor memory is freed
           mma_commit(bar(kBarDrain));
           const uint64_t t0 = globaltimer();
           while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
@@ -301,8 +308,8 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       const int stage = it % kStages;
       const float* cv = reinterpret_cast<const float*>(sg + kOffKV + (uint32_t)stage * kStageBytes + 2 * kTileBytes) +
                         (cls == RELPOS_TILE_CONST_LO ? 0 : kT) + cb;
-      const bool got_s = mbar_wait(bar(kBarSFull), it & 1, abort_flag) &&
-                         (!(AK && is_const) || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
+      const bool got_s = mbar_wait(bar(kBarSFull), it & 1, abort_flag, p.wait_ns) &&
+                         (!(AK && is_const) || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag, p.wait_ns));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       float x[64];
@@ -355,7 +362,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       }
       // dS = P (dP - D) for this thread's 64 keys; written as the 16-bit A
       // operand of dQ += dS K
-      const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag);
+      const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag, p.wait_ns);
       if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
       tc_fence_after();
       {
@@ -408,7 +415,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       }
       // dS buffer (t & 1) is free once dQ(t - 2) has read it
       if (it > 1) {
-        const bool got = mbar_wait(bar(kBarDsFree + (it & 1)), ((it >> 1) - 1) & 1, abort_flag);
+        const bool got = mbar_wait(bar(kBarDsFree + (it & 1)), ((it >> 1) - 1) & 1, abort_flag, p.wait_ns);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
       }
@@ -461,7 +468,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
 #pragma unroll
     for (int c = 0; c < 32; ++c) dq[c] = 0.f;
     // the last dQ GEMM's commit covers every earlier one
-    const bool got_q = nkt > 0 && ok && mbar_wait(bar(kBarDsFree + ((nkt - 1) & 1)), ((nkt - 1) >> 1) & 1, abort_flag);
+    const bool got_q = nkt > 0 && ok && mbar_wait(bar(kBarDsFree + ((nkt - 1) & 1)), ((nkt - 1) >> 1) & 1, abort_flag, p.wait_ns);
     if (__all_sync(0xffffffffu, got_q)) {
       tc_fence_after();
       uint32_t u[32];
@@ -551,7 +558,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
   const int kt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, k0 = kt * kT;
   const int npad = p.nT * kT;
-  const int nkv = p.padding ? p.key_len[b] : N;
+  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
   const int qt0 = p.causal ? kt : 0;            // queries i >= j only under the causal mask
   const int nq = k0 < nkv ? p.nT - qt0 : 0;
 
@@ -597,10 +604,11 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         mbar_expect_tx(bar(kBarKV), 2 * kTileBytes);
         tma_load_3d(sb + kOffK, &tmK, bar(kBarKV), 0, k0, bh);
         tma_load_3d(sb + kOffV, &tmV, bar(kBarKV), 0, k0, bh);
+        int issued = 0;
   #pragma unroll 1
         for (int it = 0; it < nq; ++it) {
           const int s = it % kStages;
-          if (it >= kStages && !mbar_wait(bar(kBarQsEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+          if (it >= kStages && !mbar_wait(bar(kBarQsEmpty + s), ((it / kStages) - 1) & 1, abort_flag, p.wait_ns)) break;
           const int qb = (qt0 + it) * kT;
           const uint32_t dst = sb + kOffQD + (uint32_t)s * kStageBytes;
           const uint32_t fb = bar(kBarQsFull + s);
@@ -615,7 +623,12 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
             bulk_load(dst + 2 * kTileBytes + 2 * kT * 4, src, kT * 4, fb);
             bulk_load(dst + 2 * kTileBytes + 3 * kT * 4, src + npad, kT * 4, fb);
           }
+          issued = it + 1;
         }
+        // no load may still be landing when the CTA exits (see the forward)
+        mbar_drain(bar(kBarKV), 0);
+        for (int it = imax(0, issued - kStages); it < issued; ++it)
+          mbar_drain(bar(kBarQsFull + it % kStages), (it / kStages) & 1);
       }
     } else if (warp == 1) {
       if (lane == 0 && nq > 0) {
@@ -646,7 +659,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
   #pragma unroll 1
           for (int kk = 0; kk < 8; ++kk) mma_ts(d, a + 8 * kk, bmn + 128 * kk, id_g, (acc || kk > 0) ? 1u : 0u);
         };
-        bool ok = mbar_wait(bar(kBarKV), 0, abort_flag) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag);
+        bool ok = mbar_wait(bar(kBarKV), 0, abort_flag, p.wait_ns) && mbar_wait(bar(kBarQsFull + 0), 0, abort_flag, p.wait_ns);
         if (ok) {
           tc_fence_after();
           issue_s(0);
@@ -660,33 +673,34 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         for (int it = 0; it < nq && ok; ++it) {
           const int s = it % kStages, s1 = (it + 1) % kStages;
           if (it + 1 < nq) {
-            ok = mbar_wait(bar(kBarQsFull + s1), ((it + 1) / kStages) & 1, abort_flag) &&
-                 mbar_wait(bar(kBarSFree), it & 1, abort_flag);
+            ok = mbar_wait(bar(kBarQsFull + s1), ((it + 1) / kStages) & 1, abort_flag, p.wait_ns) &&
+                 mbar_wait(bar(kBarSFree), it & 1, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
             issue_s(s1);
             mma_commit(bar(kBarSFull));
           }
-          ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag);
+          ok = mbar_wait(bar(kBarPReady), it & 1, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_g(tmem + kTmDV, tmem + kTmP, ddomn0 + (uint64_t)s * kStage16, it > 0);
           mma_commit(bar(kBarPFree));
           if (it + 1 < nq) {
-            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag);
+            ok = mbar_wait(bar(kBarDpFree), it & 1, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
             issue_dp(s1);
             mma_commit(bar(kBarDpFull));
           }
-          ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag);
+          ok = mbar_wait(bar(kBarDsReady), it & 1, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_g(tmem + kTmDK, tmem + kTmDS, dqmn0 + (uint64_t)s * kStage16, it > 0);
           mma_commit(bar(kBarDsFree));
           mma_commit(bar(kBarQsEmpty + s));
         }
-        if (!ok) {
+        {
+          // drain (bounded): no MMA may still run when tensor memory is freed
           mma_commit(bar(kBarDrain));
           const uint64_t t0 = globaltimer();
           while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
@@ -734,8 +748,8 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       const float* dvec = vec + kT + cb;
       const float* cvq = vec + (cls == RELPOS_TILE_CONST_LO ? 2 * kT : 3 * kT) + cb;
       // the stage's own barrier makes its TMA-written vectors visible to these threads
-      const bool got_s = mbar_wait(bar(kBarSFull), it & 1, abort_flag) &&
-                         mbar_wait(bar(kBarQsFull + stage), (it / kStages) & 1, abort_flag);
+      const bool got_s = mbar_wait(bar(kBarSFull), it & 1, abort_flag, p.wait_ns) &&
+                         mbar_wait(bar(kBarQsFull + stage), (it / kStages) & 1, abort_flag, p.wait_ns);
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       float x[64];
@@ -793,7 +807,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       }
       // P^T, two queries per column, once dV(t - 1) has read P^T(t - 1)
       if (it > 0) {
-        const bool got = mbar_wait(bar(kBarPFree), (it - 1) & 1, abort_flag);
+        const bool got = mbar_wait(bar(kBarPFree), (it - 1) & 1, abort_flag, p.wait_ns);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
       }
@@ -818,7 +832,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       mbar_arrive(bar(kBarPReady));
       // dS^T = P^T (dP^T - D_i): the A operand of dK += dS^T Q, and the
       // key-side relation gradient of this key row
-      const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag);
+      const bool got_dp = mbar_wait(bar(kBarDpFull), it & 1, abort_flag, p.wait_ns);
       if (!__all_sync(0xffffffffu, got_dp)) { ok = false; break; }
       tc_fence_after();
       {
@@ -877,7 +891,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       }
       // dS^T, two queries per column, once dK(t - 1) has read dS^T(t - 1)
       if (it > 0) {
-        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag);
+        const bool got = mbar_wait(bar(kBarDsFree), (it - 1) & 1, abort_flag, p.wait_ns);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
       }
@@ -928,7 +942,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     float dv[32], dk[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) dv[c] = dk[c] = 0.f;
-    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDsFree), (nq - 1) & 1, abort_flag);
+    const bool got_o = nq > 0 && ok && mbar_wait(bar(kBarDsFree), (nq - 1) & 1, abort_flag, p.wait_ns);
     if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
       uint32_t u[32];

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, q0 = blockIdx.x * (2 * kBQ);
-  const int nkv = p.padding ? p.key_len[b] : N;
+  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
   int kend = nkv;
   if (p.causal) kend = imin(kend, imin(q0 + 2 * kBQ, N));
   const int nkt = kend > 0 ? (kend + kBK - 1) / kBK : 0;
@@ -155,10 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
       tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
       tma_load_3d(sb + kOffQ + kTileBytes, &tmQ, bar(kBarQ), 0, q0 + kBQ, bh);
+      int issued = 0;
 #pragma unroll 1
       for (int it = 0; it < nkt; ++it) {
         const int s = it % kStages;
-        if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag)) break;
+        if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag, p.wait_ns)) break;
         const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
         mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
         tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kBK, bh);
@@ -168,7 +169,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(dst + 2 * kTileBytes, src, kBK * 4, bar(kBarKvFull + s));
           bulk_load(dst + 2 * kTileBytes + kBK * 4, src + (size_t)p.nT * kBK, kBK * 4, bar(kBarKvFull + s));
         }
+        issued = it + 1;
       }
+      // every load issued has landed before the CTA can exit (after an abort
+      // the consumers may never have waited for them); each stage's last fill
+      // is the latest phase of its barrier
+      mbar_drain(bar(kBarQ), 0);
+      for (int it = imax(0, issued - kStages); it < issued; ++it)
+        mbar_drain(bar(kBarKvFull + it % kStages), (it / kStages) & 1);
     } else if (warp == 1 && lane == 0 && nkt > 0) {
       // ---------------------------------------------------------- MMA issuer
       // order per key tile t: S_0(t+1), S_1(t+1) as soon as S_g(t) has been
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int kk = 0; kk < 8; ++kk) mma_ts(d, pt + 8 * kk, v + 128 * kk, id_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag);
+      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.wait_ns) && mbar_wait(bar(kBarKvFull + 0), 0, abort_flag, p.wait_ns);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
@@ -210,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % kStages;
           if (it + 1 < nkt) {
             const int sn = (it + 1) % kStages;
-            ok = mbar_wait(bar(kBarKvFull + sn), ((it + 1) / kStages) & 1, abort_flag);
+            ok = mbar_wait(bar(kBarKvFull + sn), ((it + 1) / kStages) & 1, abort_flag, p.wait_ns);
             for (int g = 0; g < 2 && ok; ++g) {
-              ok = mbar_wait(bar(kBarSFree + g), it & 1, abort_flag);
+              ok = mbar_wait(bar(kBarSFree + g), it & 1, abort_flag, p.wait_ns);
               if (!ok) break;
               tc_fence_after();
               issue_qk(g, sn);
@@ -220,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           for (int g = 0; g < 2 && ok; ++g) {
-            ok = mbar_wait(bar(kBarPReady + g), it & 1, abort_flag);
+            ok = mbar_wait(bar(kBarPReady + g), it & 1, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
             issue_pv(g, s, it > 0);
@@ -229,8 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) mma_commit(bar(kBarKvEmpty + s));
         }
       }
-      if (!ok) {
-        // drain: wait (bounded, ignoring the abort flag) until issued MMAs are done
+      {
+        // drain: wait (bounded, ignoring the abort flag) until every issued MMA is
+        // done, also when only the compute warps gave up, so that tensor memory is
+        // never freed under a running MMA
         mma_commit(bar(kBarDrain));
         const uint64_t t0 = globaltimer();
         while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kTimeoutNs) {
@@ -284,8 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every decision before a tcgen05.ld/st (warp-collective) is warp-uniform;
       // S ready implies the stage's TMA data landed, and waiting on the stage's
       // own barrier as well makes its saturated columns visible to these threads
-      const bool got_s = mbar_wait(bar(kBarSFull + g), it & 1, abort_flag) &&
-                         (!AK || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag));
+      const bool got_s = mbar_wait(bar(kBarSFull + g), it & 1, abort_flag, p.wait_ns) &&
+                         (!AK || mbar_wait(bar(kBarKvFull + stage), (it / kStages) & 1, abort_flag, p.wait_ns));
       if (!__all_sync(0xffffffffu, got_s)) { ok = false; break; }
       tc_fence_after();
       float x[128];
@@ -354,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = grow ? fast_exp2(m_run - m_new) : 1.f;
       bool pfree_seen = it == 0;
       if (it > 0 && __any_sync(0xffffffffu, grow)) {
-        const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
+        const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag, p.wait_ns);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         pfree_seen = true;
         tc_fence_after();
@@ -403,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l_run += DT<T>::kCoarse ? ps[0] + ps[1] : (ps2[0].x + ps2[1].x) + (ps2[0].y + ps2[1].y);
       if (!pfree_seen) {
-        const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag);
+        const bool got = mbar_wait(bar(kBarPFree + g), (it - 1) & 1, abort_flag, p.wait_ns);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
       }
@@ -417,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float ov[64];
 #pragma unroll
     for (int c = 0; c < 64; ++c) ov[c] = 0.f;
-    const bool got_o = nkt > 0 && ok && mbar_wait(bar(kBarPFree + g), (nkt - 1) & 1, abort_flag);
+    const bool got_o = nkt > 0 && ok && mbar_wait(bar(kBarPFree + g), (nkt - 1) & 1, abort_flag, p.wait_ns);
     if (__all_sync(0xffffffffu, got_o)) {
       tc_fence_after();
       uint32_t u[64];

@@ -105,6 +105,9 @@ struct Plan {
   int dropout;
   uint32_t drop_thresh, seed_lo, seed_hi, drop_offset;
   float drop_scale;             // 1 / (1 - p)
+  // limit of every bounded mbarrier wait in the fused kernels (ns); the host
+  // lowers it only to exercise the timeout path
+  unsigned long long wait_ns;
 };
 
 // Reachable expanded columns of query group g (key_side = 0) or key group g

@@ -10,7 +10,12 @@
 // device image, so the call itself never allocates.
 //
 // The array is kScratchBytes (32 MiB) of global memory on every GPU that
-// loads this library, held until the process exits.
+// loads this library, held until the process exits.  It lives in this file's
+// own module, which CUDA loads lazily by default: the first call on a device
+// (its cudaGetSymbolAddress) loads the module and commits the 32 MiB, and the
+// first launch of each kernel loads that kernel's module.  A caller that must
+// not allocate later makes one small call on each device early, before a pool
+// claims the memory, or runs with CUDA_MODULE_LOADING=EAGER.
 #include <mutex>
 
 #include "kernels.cuh"
@@ -60,4 +65,12 @@ RELPOS_EXPORT int relpos_attn_fwd_noalloc(const relpos_fwd_args* a, relpos_strea
   const int st2 = relpos_attn_fwd(a, ws, kScratchBytes, stream);
   relpos::set_single_stream(false);
   return st2;
+}
+
+RELPOS_EXPORT int relpos_check_noalloc(relpos_stream_t stream, int32_t* device_status) {
+  void* ws = nullptr;
+  const int e = scratch_for_current_device(&ws);
+  if (e) return relpos::cuda_status((cudaError_t)e);
+  // the status word sits at the start of the forward's workspace layout
+  return relpos_check_workspace(ws, stream, device_status);
 }

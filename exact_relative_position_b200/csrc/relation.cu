@@ -524,7 +524,7 @@ __global__ void debug_plan_kernel(const int B, const int N, const int causal, co
   const int kj = (int)(idx % nT);
   const int qi = (int)((idx / nT) % nT);
   const int b = (int)(idx / ((long long)nT * nT));
-  const int nkv = key_len ? key_len[b] : N;
+  const int nkv = key_len ? iclamp(key_len[b], 0, N) : N;
   classes[idx] = tile_class(qi, kj, N, nkv, causal, E_lo, E_hi);
   if (kj == 0) {
     int sg[4];

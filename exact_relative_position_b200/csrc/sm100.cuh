@@ -46,18 +46,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for phase `parity` of `bar`.  Gives up (returns false) when another
-// role of the CTA has already flagged *abort, or after kTimeoutNs, in which
-// case it sets *abort itself.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// role of the CTA has already flagged *abort, or after `limit_ns` (the plan's
+// wait limit, kTimeoutNs unless the host lowered it), in which case it sets
+// *abort itself.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       return false;
     }
+  }
+}
+
+// Drain after an abort: waits, bounded by kTimeoutNs and ignoring the abort
+// flag, until phase `parity` of `bar` has completed.  The producer calls it for
+// every load it has issued, so that no TMA write into shared memory is still
+// in flight when the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kTimeoutNs) {
   }
 }
 

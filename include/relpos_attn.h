@@ -100,7 +100,9 @@ typedef struct {
   relpos_map_desc map;
   int32_t mask;              /* relpos_mask_flags */
   int32_t table_per_head;    /* 0: aq/ak are [R,d] shared by all heads; 1: [H,R,d] */
-  const int32_t* key_len;    /* device [B], each in [0, N]; required iff mask has KEY_PADDING */
+  const int32_t* key_len;    /* device [B]; required iff mask has KEY_PADDING.  Keys j >= key_len[b]
+                                are masked; a value below 0 counts as 0 and one above N as N
+                                (the kernels clamp it, so no length can make them read past N) */
   const void* q;             /* device [B,H,N,d] dtype */
   const void* k;             /* device [B,H,N,d] dtype */
   const void* v;             /* device [B,H,N,d] dtype */
@@ -141,26 +143,34 @@ typedef struct {
                                 garbage: the library cannot tell. */
 } relpos_bwd_args;
 
-/* Number of rows R of a relation table for `map` at sequence length N (host only).
+/* Number of rows R of a relation table for `map` at sequence length N (host only):
+ * the table sizes of the four mechanisms of the digest's experimental setup
+ * (truncated 2 clip + 1, identity 2N - 1, T5 num_buckets, DeBERTa 2 num_buckets).
  * Errors: INVALID_ARG for null pointers or N < 1, UNSUPPORTED for an unknown kind. */
 int relpos_table_rows(const relpos_map_desc* map, int32_t N, int32_t* R_out);
 
-/* Saturation bounds of the expanded truncated map (host only, digest "constant
- * tiles and the saturated region"): every reachable offset <= *e_lo maps to one
- * row, every offset >= *e_hi to one row; the expanded table has one row per
- * offset in [*e_lo, *e_hi]. */
+/* Saturation bounds of the expanded truncated map (host only; digest, "constant
+ * tiles and the saturated region": bucketed maps are expanded by copying each
+ * bucket row once per offset it covers): every reachable offset <= *e_lo maps
+ * to one row, every offset >= *e_hi to one row; the expanded table has one row
+ * per offset in [*e_lo, *e_hi].  Errors: INVALID_ARG, UNSUPPORTED as above. */
 int relpos_expanded_bounds(const relpos_map_desc* map, int32_t N, int32_t* e_lo, int32_t* e_hi);
 
 /* Workspace bytes needed by relpos_attn_fwd / relpos_attn_bwd for these
  * arguments (pointers are not read; only sizes, map, mask and which of
- * aq/ak/b are non-NULL).  The workspace holds the projections Z^Q/Z^K
- * (O(B H N R_reach), never N x N for non-identity maps), the expanded
- * tables, and in backward the offset-sharded gradients. */
+ * aq/ak/b are non-NULL).  The workspace holds the projections Z^Q/Z^K over
+ * each 128-row group's reachable columns (digest, "grouped reachable range":
+ * about N + G - 1 columns per group for the identity map, all R_exp columns
+ * when one group covers the table; never N x N for the other maps), the
+ * expanded tables, and in backward the offset-sharded gradients of Eq. (4).
+ * Errors: INVALID_ARG, UNSUPPORTED. */
 int relpos_workspace_size(const relpos_fwd_args* a, size_t* fwd_bytes, size_t* bwd_bytes);
 
-/* Forward: writes a->o and a->lse.  workspace: device, >= fwd_bytes, 256-byte
- * aligned, contents on entry ignored.  Errors: INVALID_ARG, UNSUPPORTED,
- * WORKSPACE, CUDA. */
+/* Forward (digest, pipeline section: grouped projections, then the
+ * FlashAttention-style query-tile / key-tile loop with the relation terms
+ * added on chip and an online softmax): writes a->o and a->lse.
+ * workspace: device, >= fwd_bytes, 256-byte aligned, contents on entry
+ * ignored.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 int relpos_attn_fwd(const relpos_fwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream);
 
 /* Backward (digest: two-pass backward, Eq. (4)): from dO and the forward's O
@@ -170,17 +180,20 @@ int relpos_attn_fwd(const relpos_fwd_args* a, void* workspace, size_t ws_bytes, 
 int relpos_attn_bwd(const relpos_bwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream);
 
 /* Device-side status of the last call that used `workspace` (synchronous:
- * waits for `stream`).  The fused kernels bound every wait on an mbarrier;
+ * waits for `stream`).  No counterpart on the pages: the library's own
+ * failure report.  The fused kernels bound every wait on an mbarrier;
  * when one expires the kernel stops its pipeline, frees its tensor memory,
  * returns, and leaves a non-zero status word at the start of the workspace
  * (its outputs are then invalid).  Returns RELPOS_OK, RELPOS_ERR_TIMEOUT
  * (*device_status = 1), or RELPOS_ERR_CUDA.  device_status: host, may be NULL. */
 int relpos_check_workspace(const void* workspace, relpos_stream_t stream, int32_t* device_status);
 
-/* Human-readable text of a relpos_status (static storage). */
+/* Human-readable text of a relpos_status (static storage).  No counterpart on
+ * the pages (error reporting of this interface). */
 const char* relpos_status_string(int status);
 
-/* The last cudaError_t seen by this thread inside the library (0 = none). */
+/* The last cudaError_t seen by this thread inside the library (0 = none).  No
+ * counterpart on the pages (error reporting of this interface). */
 int relpos_last_cuda_error(void);
 
 /* Forward without a caller workspace (no counterpart in the paper; an
@@ -188,20 +201,32 @@ int relpos_last_cuda_error(void);
  * while a memory pool or another runtime owns the whole device and forbids
  * outside allocations, or an enqueue step that must not allocate).
  *
- * Same arguments, outputs and errors as relpos_attn_fwd, but the workspace is
- * a fixed 32 MiB array inside the library's device image.  Every GPU that
- * loads the library holds that array until the process exits.  The call
- * itself calls no cudaMalloc / cudaFree or any allocating routine.
+ * Same arguments and outputs as relpos_attn_fwd, but the workspace is a fixed
+ * 32 MiB array inside the library's device image.  Every GPU on which the
+ * library has made its first such call holds that array until the process
+ * exits.  Apart from that first call (below), a call calls no cudaMalloc /
+ * cudaFree or any allocating routine.
  *  - Shapes whose forward workspace (relpos_workspace_size's fwd_bytes)
  *    exceeds 32 MiB are rejected with RELPOS_ERR_WORKSPACE before any launch.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    outside any stream capture.
+ *    outside any stream capture.  CUDA loads modules lazily by default, so
+ *    that first call also loads the array's module (committing the 32 MiB)
+ *    and each kernel's first launch loads its module: make one small call on
+ *    every device before a pool claims the device's memory, or run with
+ *    CUDA_MODULE_LOADING=EAGER.
  *  - All calls share the one array and it keeps the previous call's contents;
  *    the forward reads nothing from it that the same call has not written.
  *    Calls whose work overlaps on the GPU (different streams, or several
- *    host threads) race on the array: serialise them. */
+ *    host threads) race on the array: serialise them.
+ *  - A kernel whose bounded wait expired is reported by relpos_check_noalloc
+ *    (the status word lives in the array), until the next call clears it. */
 int relpos_attn_fwd_noalloc(const relpos_fwd_args* a, relpos_stream_t stream);
+
+/* Device status of the last relpos_attn_fwd_noalloc on the current device
+ * (synchronous: waits for `stream`); results as relpos_check_workspace.  No
+ * counterpart in the paper (failure report of the no-allocation forward). */
+int relpos_check_noalloc(relpos_stream_t stream, int32_t* device_status);
 
 /* --- measurement ---------------------------------------------------------- */
 
@@ -255,6 +280,44 @@ int64_t relpos_kernel_launches(void);
 int relpos_sum_partials(const float* partials, int32_t world, int64_t n, float* out, relpos_stream_t stream);
 
 /* --- parity exports (used by the tests) --------------------------------- */
+
+/* Storage of one 128-row projection group (digest, "grouped reachable range",
+ * Eq. (3)): its rows hold the expanded columns [e0, e0 + W) (expanded column
+ * e is offset E_lo + e) with a row stride of S floats, starting `base` floats
+ * into a (batch, head) slice.  Columns [W, S) of a row are padding. */
+typedef struct {
+  int32_t e0, W, S, pad;
+  int64_t base;
+} relpos_group_info;
+
+/* Where relpos_debug_projection left the projections in the workspace. */
+typedef struct {
+  int32_t E_lo, E_hi, R_exp;   /* expanded offset range [E_lo, E_hi], R_exp = E_hi - E_lo + 1 */
+  int32_t nT;                  /* groups (= 128-row tiles) per (batch, head) */
+  int32_t grouped;             /* 1: per-group reachable columns; 0: every group stores all R_exp */
+  int32_t pad;
+  int64_t zq_offset, zk_offset;   /* byte offsets of Z^Q / Z^K (float32) in the workspace; -1 if absent */
+  int64_t zq_head, zk_head;       /* floats per (batch, head) slice of Z^Q / Z^K */
+  int64_t gq_offset, gk_offset;   /* byte offsets of the query / key groups' relpos_group_info [nT] */
+} relpos_projection_layout;
+
+/* Runs the forward's table expansion and projections only (digest, Eq. (2)/(3)
+ * over each group's reachable range) and leaves Z^Q = Q aQ_exp^T and
+ * Z^K = K aK_exp^T in `workspace`: for row i of (b, h), g = i / 128, group
+ * record gi, and expanded column e in [gi.e0, gi.e0 + gi.W), Z^Q[b, h, i, e]
+ * is the float at byte zq_offset + 4 (((b H + h) zq_head) + gi.base +
+ * (i % 128) gi.S + e - gi.e0); Z^K likewise with the key groups.  Arguments
+ * as relpos_attn_fwd (o, lse, v are not read).  Synchronous.  Errors:
+ * INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+int relpos_debug_projection(const relpos_fwd_args* a, void* workspace, size_t ws_bytes, relpos_stream_t stream,
+                            relpos_projection_layout* layout);
+
+/* Limit, in nanoseconds, of every bounded wait in the fused kernels launched
+ * after this call (process-wide; 0 restores the default of 2 s).  Exists so
+ * that tests can make a wait run out on purpose and check that the kernels
+ * stop cleanly and report RELPOS_ERR_TIMEOUT.  No counterpart on the pages
+ * (failure detection of this library). */
+int relpos_set_wait_limit_ns(uint64_t ns);
 
 /* phi(i, j) for all N x N cells computed on the host. phi_host: host [N*N] int32. */
 int relpos_debug_phi(const relpos_map_desc* map, int32_t N, int32_t* phi_host);

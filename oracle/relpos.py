@@ -179,12 +179,6 @@ def expanded_bounds(m: MapDesc, N: int):
     return int(deltas[lo]), int(deltas[hi])
 
 
-def expanded_row_map(m: MapDesc, N: int):
-    """For each expanded row e (offset E_lo + e), the original table row phi."""
-    elo, ehi = expanded_bounds(m, N)
-    return phi_of_delta(m, np.arange(elo, ehi + 1, dtype=np.int64), N)
-
-
 def tile_plan_brute(m: MapDesc, N: int, T: int, causal: bool, key_len=None, B: int = 1):
     """Tile classes by inspecting every cell of every tile.
 
@@ -561,15 +555,33 @@ def head_block_step(q, k, v, do, aq, ak, bvec, tau, m: MapDesc, causal, key_len_
     ri = np.repeat(np.arange(n), N)
     cj = np.tile(np.arange(N), n)
     fp = phi.reshape(-1)
-    dzq = tau * np.bincount(ri * R + fp, weights=dS.reshape(-1), minlength=n * R).reshape(n, R)
-    dzk = tau * np.bincount(cj * R + fp, weights=dS.reshape(-1), minlength=N * R).reshape(N, R)
     out = dict(o=O, lse=lse, dv=P.T @ do[rows], dq=tau * (dS @ k), dk=tau * (dS.T @ q[rows]))
+    # each relation gradient only when its term is present (the key-side one is
+    # N x R per block: 4 GB for the identity map at N = 16384)
     if aq is not None:
+        dzq = tau * np.bincount(ri * R + fp, weights=dS.reshape(-1), minlength=n * R).reshape(n, R)
         out["dq"] = out["dq"] + dzq @ aq
         out["daq"] = dzq.T @ q[rows]
     if ak is not None:
+        dzk = tau * np.bincount(cj * R + fp, weights=dS.reshape(-1), minlength=N * R).reshape(N, R)
         out["dak"] = dzk.T @ k
         out["dk_rel"] = dzk @ ak
     if bvec is not None:
         out["db"] = tau * np.bincount(fp, weights=dS.reshape(-1), minlength=R)
     return out
+
+
+def head_table_grads(q, k, v, do, aq, ak, bvec, tau, m: MapDesc, causal, key_len_b, block=512):
+    """Table gradients daq, dak, db of one (b, h) slice (those whose term is
+    present), as the sum of head_block_step's contributions over consecutive
+    blocks of query rows: the Eq. (4) sums taken over all query rows without
+    holding an N x N matrix."""
+    N = q.shape[0]
+    acc = {}
+    for r0 in range(0, N, block):
+        part = head_block_step(q, k, v, do, aq, ak, bvec, tau, m, causal, key_len_b,
+                               np.arange(r0, min(N, r0 + block)))
+        for name in ("daq", "dak", "db"):
+            if name in part:
+                acc[name] = part[name] if name not in acc else acc[name] + part[name]
+    return acc

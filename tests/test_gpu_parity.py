@@ -141,3 +141,18 @@ def test_large_scores_exercise_lazy_rescale(dtype):
         assert relf(got["o"], want["o"]) <= TOL_O_RELF
         assert maxabs(got["o"], want["o"]) <= 3.5e-2
     check_backward(got, want)
+
+
+@pytest.mark.parametrize("key_len", [[300 + 200, -1], [-7, 299]])
+def test_out_of_range_key_lengths_clamp(key_len):
+    """Key lengths outside [0, N] act as their clamped values: the kernels clamp
+    them, and the oracle's mask (keys j >= key_len are masked) needs no clamp.
+    A length of -1 masks every key of that batch element (O = 0, LSE = -inf);
+    N + 200 masks none.  Forward, backward and the device tile plan."""
+    w = small_workload(N=300, B=2, H=2, terms=("aQ", "aK", "b"), key_len=key_len, **MAPS["log"])
+    got, want = run_library(w), run_oracle(w)
+    check_forward(got, want, "clamped key_len")
+    check_backward(got, want, "clamped key_len")
+    cls, seg = rp.debug_tile_plan_device(lmap(w), 2, 300, key_len=key_len)
+    want_cls, want_seg = orc.tile_plan_rule(omap(w), 300, 128, False, key_len=key_len, B=2)
+    assert np.array_equal(cls.cpu().numpy(), want_cls) and np.array_equal(seg.cpu().numpy(), want_seg)

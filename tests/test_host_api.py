@@ -136,6 +136,21 @@ def test_validation_rejects_before_launch(lib):
     g.db = 1 << 20
     assert lib.relpos_attn_bwd(ctypes.byref(g), 1 << 20, 1 << 34, None) == -1
     assert lib.relpos_status_string(-3).decode().startswith("workspace")
+    # debug projection: missing layout record, then a workspace that is too small
+    lay = bd.relpos_projection_layout()
+    assert lib.relpos_debug_projection(ctypes.byref(_args()), 1 << 20, 1 << 30, None, None) == -1
+    assert lib.relpos_debug_projection(ctypes.byref(_args()), 1 << 20, 16, None, ctypes.byref(lay)) == -3
+
+
+@pytest.mark.parametrize("key_len", [[8192 + 200, -1], [-5, 100000], [0, 8191]])
+def test_tile_plan_clamps_out_of_range_key_lengths(lib, key_len):
+    """A key length outside [0, N] masks as its clamped value would (the oracle's
+    mask j >= key_len needs no clamp): the host plan equals the oracle's rule."""
+    m, lm = _maps("truncated", dict(clip=64))
+    N = 8192
+    cls, seg = bd.debug_tile_plan(lm, 2, N, causal=False, key_len=key_len)
+    want_cls, want_seg = orc.tile_plan_rule(m, N, 128, False, key_len=key_len, B=2)
+    assert np.array_equal(cls.numpy(), want_cls) and np.array_equal(seg.numpy(), want_seg)
 
 
 @pytest.mark.parametrize("kind,clip,N,B,H", [("truncated", 64, 8192, 1, 12), ("t5", 0, 8192, 1, 12),

@@ -456,3 +456,27 @@ def test_row_blocks_sum_to_full_backward():
     np.testing.assert_allclose(acc["daq"], full["daq"], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(acc["dak"], full["dak"], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(acc["db"], full["db"], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind,terms,causal,kl", [
+    ("identity", ("aq", "b"), True, None), ("truncated", ("aq", "ak"), False, 23),
+    ("t5", ("b",), False, None), ("log", ("aq", "ak", "b"), True, 17)])
+def test_row_block_table_grads_equal_full_backward(kind, terms, causal, kl):
+    """The row-block sums behind the config-size table-gradient checks equal the
+    full-matrix backward (itself pinned by central differences), for every term
+    subset, with causal and key-padding masks."""
+    N, d = 29, 4
+    kw = {"truncated": dict(clip=5), "identity": {}, "t5": dict(num_buckets=8, max_distance=20, bidirectional=1),
+          "log": dict(num_buckets=8, max_distance=24)}[kind]
+    m = orc.MapDesc(kind, **kw)
+    R = orc.table_rows(m, N)
+    q, k, v, do = (_rand((N, d), s) for s in range(4))
+    aq = _rand((R, d), 5, 0.5) if "aq" in terms else None
+    ak = _rand((R, d), 6, 0.5) if "ak" in terms else None
+    b = _rand((R,), 7) if "b" in terms else None
+    phi = orc.phi_matrix(m, N)
+    full = orc.head_backward(q, k, v, do, aq, ak, b, 0.3, phi, orc.allowed_matrix(N, causal, kl), R)
+    got = orc.head_table_grads(q, k, v, do, aq, ak, b, 0.3, m, causal, kl, block=6)
+    assert set(got) == {n for n, t in (("daq", aq), ("dak", ak), ("db", b)) if t is not None}
+    for n in got:
+        np.testing.assert_allclose(got[n], full[n], rtol=1e-10, atol=1e-12)
