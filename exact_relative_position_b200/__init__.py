@@ -8,9 +8,9 @@ library behind the C ABI in include/relpos_attn.h.  PyTorch supplies device
 memory and streams only.
 """
 from ._binding import (  # noqa: F401
-    RelPosError, RelPosMap, check_workspace, debug_phi, debug_phi_device, debug_tile_plan, debug_tile_plan_device,
-    expanded_bounds, kernel_launches, lib, profile_start, profile_stop, relpos_attn_bwd, relpos_attn_fwd,
-    sum_partials, table_rows, workspace_size,
+    RelPosError, RelPosMap, check_noalloc, check_workspace, debug_phi, debug_phi_device, debug_projection,
+    debug_tile_plan, debug_tile_plan_device, expanded_bounds, kernel_launches, lib, profile_start, profile_stop,
+    relpos_attn_bwd, relpos_attn_fwd, set_wait_limit_ns, sum_partials, table_rows, workspace_size,
 )
 
 import torch
