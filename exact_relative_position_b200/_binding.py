@@ -19,6 +19,7 @@ RELPOS_OK = 0
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "workspace", -4: "cuda error", -5: "timeout"}
 MAP_KINDS = {"truncated": 0, "identity": 1, "t5": 2, "log": 3}
 MASK_CAUSAL, MASK_KEY_PADDING = 1, 2
+PROJECTION_MODES = {"retained": 0, "recompute": 1}
 F16, BF16, F32 = 0, 1, 2
 TILE = 128
 TILE_MASKED, TILE_CONST_LO, TILE_BAND, TILE_CONST_HI = 0, 1, 2, 3
@@ -36,7 +37,8 @@ class relpos_fwd_args(ctypes.Structure):
                 ("key_len", ctypes.c_void_p), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("aq", ctypes.c_void_p), ("ak", ctypes.c_void_p),
                 ("b", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
-                ("dropout_p", ctypes.c_float), ("dropout_offset", ctypes.c_uint32), ("dropout_seed", ctypes.c_uint64)]
+                ("dropout_p", ctypes.c_float), ("dropout_offset", ctypes.c_uint32), ("dropout_seed", ctypes.c_uint64),
+                ("projection", ctypes.c_int32)]
 
 
 class relpos_bwd_args(ctypes.Structure):
@@ -171,7 +173,7 @@ def _dtype_code(dt: torch.dtype) -> int:
 
 
 def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o=None, lse=None,
-              dropout=(0.0, 0, 0)):
+              dropout=(0.0, 0, 0), projection="retained"):
     B, H, N, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda or not t.is_contiguous() or t.shape != q.shape or t.dtype != q.dtype:
@@ -198,11 +200,15 @@ def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o
     a.aq, a.ak, a.b = _ptr(aq), _ptr(ak), _ptr(b)
     a.o, a.lse = _ptr(o), _ptr(lse)
     a.dropout_p, a.dropout_seed, a.dropout_offset = float(dropout[0]), int(dropout[1]), int(dropout[2])
+    if projection not in PROJECTION_MODES:
+        raise RelPosError(f"projection must be one of {sorted(PROJECTION_MODES)}")
+    a.projection = PROJECTION_MODES[projection]
     return a
 
 
-def workspace_size(q, aq, ak, b, tau, m: RelPosMap, causal=False, key_len=None, out_f32=False):
-    a = _fwd_args(q, q, q, aq, ak, b, tau, m, causal, key_len, out_f32)
+def workspace_size(q, aq, ak, b, tau, m: RelPosMap, causal=False, key_len=None, out_f32=False,
+                   projection="retained"):
+    a = _fwd_args(q, q, q, aq, ak, b, tau, m, causal, key_len, out_f32, projection=projection)
     f, bw = ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
     return f.value, bw.value
@@ -214,10 +220,12 @@ def _stream(dev) -> int:
 
 def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap, causal: bool = False,
                     key_len=None, out_f32: bool = False, workspace=None, o=None, lse=None,
-                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
+                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0,
+                    projection: str = "retained"):
     """Forward through the C ABI.  Returns (O, LSE); O is float32 when out_f32.
     Attention dropout with rate dropout_p uses the Philox mask of (seed, offset);
-    the backward needs the same three values."""
+    the backward needs the same three values.  projection="recompute" projects
+    q.aQ inside every tile instead of storing Z^Q (linear forward memory)."""
     B, H, N, d = q.shape
     if o is None:
         o = torch.empty(q.shape, device=q.device, dtype=torch.float32 if out_f32 else q.dtype)
@@ -226,7 +234,7 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
     if key_len is not None:
         key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse,
-                  (dropout_p, dropout_seed, dropout_offset))
+                  (dropout_p, dropout_seed, dropout_offset), projection)
     f, bw = ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
     if workspace is None or workspace.numel() < f.value:
@@ -238,7 +246,8 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
 
 def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap,
                     causal: bool = False, key_len=None, workspace=None, grads=None, reuse_forward: bool = False,
-                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
+                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0,
+                    projection: str = "retained"):
     """Backward through the C ABI.  Returns (dq, dk, dv, daq, dak, db).
 
     reuse_forward: `workspace` is the one the forward with these same arguments
@@ -250,7 +259,7 @@ def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: flo
     if not dout.is_contiguous() or dout.dtype != q.dtype or dout.shape != q.shape:
         raise RelPosError("dout must be contiguous, shaped and typed like q")
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse,
-                  (dropout_p, dropout_seed, dropout_offset))
+                  (dropout_p, dropout_seed, dropout_offset), projection)
     g = relpos_bwd_args()
     g.fwd = a
     if grads is None:
@@ -329,7 +338,7 @@ NOALLOC_MAX_WORKSPACE = 32 << 20
 
 
 def relpos_attn_fwd_noalloc(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap, causal: bool = False,
-                            key_len=None, out_f32: bool = False, o=None, lse=None):
+                            key_len=None, out_f32: bool = False, o=None, lse=None, projection: str = "retained"):
     """Forward through relpos_attn_fwd_noalloc: the library's fixed 32 MiB scratch
     array replaces the workspace, so the call needs no device allocation for it."""
     B, H, N, d = q.shape
@@ -339,7 +348,7 @@ def relpos_attn_fwd_noalloc(q, k, v, aq=None, ak=None, b=None, *, tau: float, ma
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
     if key_len is not None:
         key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
-    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse)
+    a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse, projection=projection)
     _check(lib().relpos_attn_fwd_noalloc(ctypes.byref(a), _stream(q.device)), "relpos_attn_fwd_noalloc")
     return o, lse
 

@@ -46,11 +46,14 @@ class TransformerXLRelPos(torch.nn.Module):
     """
 
     def __init__(self, n_heads: int, d_head: int = 64, d_model: int | None = None, causal: bool = True,
-                 tau: float | None = None, init_std: float = 0.02):
+                 tau: float | None = None, init_std: float = 0.02, projection: str = "retained"):
         super().__init__()
         self.n_heads, self.d_head = n_heads, d_head
         self.d_model = d_model or n_heads * d_head
         self.causal = causal
+        # "recompute": the kernel projects q'.aQ inside every tile, so the
+        # forward never stores the quadratic identity-map projection
+        self.projection = projection
         self.tau = tau if tau is not None else 1.0 / math.sqrt(d_head)
         self.W_r = torch.nn.Parameter(torch.randn(n_heads, self.d_model, d_head) * init_std)
         self.u = torch.nn.Parameter(torch.randn(n_heads, d_head) * init_std)
@@ -67,4 +70,5 @@ class TransformerXLRelPos(torch.nn.Module):
 
     def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
         qp, aq, b = self.unified_inputs(q)
-        return relpos_attention(qp, k, v, aq, None, b, tau=self.tau, map=RelPosMap("identity"), causal=self.causal)
+        return relpos_attention(qp, k, v, aq, None, b, tau=self.tau, map=RelPosMap("identity"), causal=self.causal,
+                                projection=self.projection)

@@ -217,6 +217,7 @@ struct Layout {
   size_t status, zksat, gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
   size_t dsum, lse2, zqsat, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
   int R, Hq, expand, nsq, nsk, nsb;
+  int recompute;   // projection = RECOMPUTE: Z^Q lives in the backward-only part
 };
 
 int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
@@ -227,9 +228,14 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   if (a->B < 1 || a->H < 1 || a->N < 1 || a->N > kMaxN) return RELPOS_ERR_INVALID_ARG;
   if ((long long)a->B * a->H > 65535) return RELPOS_ERR_INVALID_ARG;
   if (a->mask & ~(RELPOS_MASK_CAUSAL | RELPOS_MASK_KEY_PADDING)) return RELPOS_ERR_UNSUPPORTED;
-  if (!(a->tau == a->tau) || a->tau > 3.0e38f || a->tau < -3.0e38f) return RELPOS_ERR_INVALID_ARG;
+  // tau > 0 and finite: the kernels fold tau into the base-2 exponent and take
+  // row maxima of the scaled scores, which assumes a positive scale
+  if (!(a->tau > 0.f) || a->tau > 3.0e38f) return RELPOS_ERR_INVALID_ARG;
   int st = check_map(&a->map);
   if (st) return st;
+  if (a->projection != RELPOS_PROJECTION_RETAINED && a->projection != RELPOS_PROJECTION_RECOMPUTE)
+    return RELPOS_ERR_INVALID_ARG;
+  if (a->projection == RELPOS_PROJECTION_RECOMPUTE && a->ak) return RELPOS_ERR_UNSUPPORTED;
   memset(p, 0, sizeof(*p));
   memset(L, 0, sizeof(*L));
   const int N = a->N;
@@ -259,6 +265,7 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   L->R = rows_of(a->map, N);
   L->Hq = a->table_per_head ? a->H : 1;
   L->expand = a->map.kind == RELPOS_MAP_BUCKET_T5 || a->map.kind == RELPOS_MAP_BUCKET_LOG;
+  L->recompute = a->projection == RELPOS_PROJECTION_RECOMPUTE;
   const size_t BH = (size_t)a->B * a->H;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = up256(off + bytes); return o; };
@@ -271,10 +278,12 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   L->bexp = bb ? take(sizeof(float) * a->H * p->Rexp) : 0;
   L->aqe = (aq && L->expand) ? take((size_t)2 * L->Hq * p->Rexp * 64) : 0;
   L->ake = (ak && L->expand) ? take((size_t)2 * L->Hq * p->Rexp * 64) : 0;
-  L->zq = aq ? take(sizeof(float) * BH * p->zq_head) : 0;
+  L->zq = (aq && !L->recompute) ? take(sizeof(float) * BH * p->zq_head) : 0;
   L->zk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
   L->zksat = ak ? take(sizeof(float) * BH * 2 * (size_t)p->nT * kTile) : 0;
   L->fwd_end = off;
+  // a recomputing forward stores no projection; its backward rebuilds Z^Q here
+  if (aq && L->recompute) L->zq = take(sizeof(float) * BH * p->zq_head);
   const size_t npad = (size_t)p->nT * kTile;
   L->dsum = take(sizeof(float) * BH * npad);
   L->lse2 = take(sizeof(float) * BH * npad);
@@ -317,7 +326,7 @@ int check_fwd_ptrs(const relpos_fwd_args* a) {
 // (the forward always builds; the backward skips it when the caller declares
 // the forward's state still in the workspace).
 int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Tensors& t, cudaStream_t s,
-            bool build = true) {
+            bool build = true, bool build_projection = true) {
   memset(&t, 0, sizeof(t));
   GroupInfo* gq = reinterpret_cast<GroupInfo*>(ws + L.gq);
   GroupInfo* gk = reinterpret_cast<GroupInfo*>(ws + L.gk);
@@ -355,13 +364,15 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
     t.zk = reinterpret_cast<float*>(ws + L.zk);
     t.zk_sat = reinterpret_cast<float*>(ws + L.zksat);
   }
-  if (!build) return RELPOS_OK;
-  cudaError_t e = run_phase(PH_TABLES, s, [&] {
-    return launch_build_tables(p, a->map, gq, gk, phi_exp, L.R, a->aq, a->ak, a->table_per_head, ws + L.aqe,
-                               ws + L.ake, a->b, const_cast<float*>(t.b_exp), t.is_bf16, L.expand, s);
-  });
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (a->aq || a->ak) {
+  cudaError_t e = cudaSuccess;
+  if (build) {
+    e = run_phase(PH_TABLES, s, [&] {
+      return launch_build_tables(p, a->map, gq, gk, phi_exp, L.R, a->aq, a->ak, a->table_per_head, ws + L.aqe,
+                                 ws + L.ake, a->b, const_cast<float*>(t.b_exp), t.is_bf16, L.expand, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (build_projection && (a->aq || a->ak)) {
     // Z^Q on the caller's stream, Z^K and its saturated columns beside it
     e = run_phase(PH_PROJ, s, [&] {
       Fork aux(s, 1);
@@ -417,9 +428,12 @@ RELPOS_EXPORT int relpos_attn_fwd(const relpos_fwd_args* a, void* workspace, siz
   if (!workspace || ws_bytes < L.fwd_end || (reinterpret_cast<uintptr_t>(workspace) & 255)) return RELPOS_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Tensors t;
-  st = prepare(a, p, L, static_cast<uint8_t*>(workspace), t, s);
+  // a recomputing forward builds the tables only; its kernel projects per tile
+  st = prepare(a, p, L, static_cast<uint8_t*>(workspace), t, s, true, !L.recompute);
   if (st) return st;
-  const cudaError_t e = run_phase(PH_FWD, s, [&] { return launch_forward(p, t, s); });
+  const cudaError_t e = run_phase(PH_FWD, s, [&] {
+    return L.recompute ? launch_forward_recompute(p, t, s) : launch_forward(p, t, s);
+  });
   if (e != cudaSuccess) return cuda_fail(e);
   return RELPOS_OK;
 }
@@ -443,7 +457,10 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (g->reuse_forward_workspace != 0 && g->reuse_forward_workspace != 1) return RELPOS_ERR_INVALID_ARG;
   Tensors t;
-  st = prepare(a, p, L, ws, t, s, /*build=*/g->reuse_forward_workspace == 0);
+  // reuse: the forward's tables (and, retained, its projections) are in the workspace;
+  // after a recomputing forward the projection is always rebuilt
+  st = prepare(a, p, L, ws, t, s, /*build=*/g->reuse_forward_workspace == 0,
+               /*build_projection=*/g->reuse_forward_workspace == 0 || L.recompute);
   if (st) return st;
   t.dout = g->dout;
   t.dsum = reinterpret_cast<float*>(ws + L.dsum);
@@ -511,8 +528,13 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
 static_assert(sizeof(relpos_group_info) == sizeof(GroupInfo), "relpos_group_info mirrors GroupInfo");
 static_assert(offsetof(relpos_group_info, base) == offsetof(GroupInfo, base), "relpos_group_info mirrors GroupInfo");
 
-RELPOS_EXPORT int relpos_debug_projection(const relpos_fwd_args* a, void* workspace, size_t ws_bytes,
+RELPOS_EXPORT int relpos_debug_projection(const relpos_fwd_args* a_in, void* workspace, size_t ws_bytes,
                                           relpos_stream_t stream, relpos_projection_layout* layout) {
+  if (!a_in) return RELPOS_ERR_INVALID_ARG;
+  // the stored projection is the retained mode's
+  relpos_fwd_args args = *a_in;
+  args.projection = RELPOS_PROJECTION_RETAINED;
+  const relpos_fwd_args* a = &args;
   Plan p;
   Layout L;
   int st = make_plan(a, &p, &L);

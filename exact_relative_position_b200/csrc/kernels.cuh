@@ -63,6 +63,8 @@ cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t 
 // swizzle, rows past N read as zero.
 bool make_rows_map(CUtensorMap* m, const void* base, int BH, int N, bool bf16);
 cudaError_t launch_forward(const Plan& p, const Tensors& t, cudaStream_t s);
+// Forward with Z^Q recomputed per tile (q.aQ and b terms only).
+cudaError_t launch_forward_recompute(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dq(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_bwd_dkdv(const Plan& p, const Tensors& t, cudaStream_t s);

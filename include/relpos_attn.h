@@ -96,7 +96,7 @@ typedef struct {
   int32_t B, H, N, d;        /* d must be 64 */
   int32_t dtype;             /* RELPOS_F16 or RELPOS_BF16: q, k, v, aq, ak (and dout, dq, dk, dv) */
   int32_t out_dtype;         /* O: same as dtype, or RELPOS_F32 */
-  float tau;                 /* score scale */
+  float tau;                 /* score scale, finite and > 0 (else INVALID_ARG) */
   relpos_map_desc map;
   int32_t mask;              /* relpos_mask_flags */
   int32_t table_per_head;    /* 0: aq/ak are [R,d] shared by all heads; 1: [H,R,d] */
@@ -122,7 +122,19 @@ typedef struct {
   float dropout_p;
   uint32_t dropout_offset;
   uint64_t dropout_seed;
+  /* Where the forward takes the query-side projection Z^Q from (digest,
+   * ablation "projection precompute" and limitations section):
+   * RELPOS_PROJECTION_RETAINED computes Z^Q over each group's reachable
+   * columns once and keeps it in the workspace (quadratic for the identity
+   * map); RELPOS_PROJECTION_RECOMPUTE recomputes it inside every tile on the
+   * tensor cores, so the forward workspace holds no projection at all (linear
+   * memory) at the price of more tensor work per tile.  RECOMPUTE supports
+   * the aq and b terms; with ak != NULL it returns UNSUPPORTED.  The backward
+   * of a RECOMPUTE forward rebuilds Z^Q in its own part of the workspace. */
+  int32_t projection;
 } relpos_fwd_args;
+
+typedef enum { RELPOS_PROJECTION_RETAINED = 0, RELPOS_PROJECTION_RECOMPUTE = 1 } relpos_projection_mode;
 
 typedef struct {
   relpos_fwd_args fwd;       /* the forward's inputs, plus its O and LSE (read) */
@@ -138,9 +150,10 @@ typedef struct {
                                 for these same forward arguments (expanded tables, group
                                 records, projections Z^Q / Z^K and their saturated columns);
                                 the backward then reads them instead of rebuilding them (the
-                                digest's retained projection).  0: rebuild them.  With 1 and
-                                a workspace that does not hold that state the gradients are
-                                garbage: the library cannot tell. */
+                                digest's retained projection; with projection = RECOMPUTE
+                                only the tables are reused and Z^Q is rebuilt).  0: rebuild
+                                them.  With 1 and a workspace that does not hold that state
+                                the gradients are garbage: the library cannot tell. */
 } relpos_bwd_args;
 
 /* Number of rows R of a relation table for `map` at sequence length N (host only):

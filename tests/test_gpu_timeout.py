@@ -18,8 +18,8 @@ from exact_relative_position_b200 import _binding as bd
 pytestmark = pytest.mark.gpu
 
 
-def _calls(w, dev, ws):
-    kw = dict(tau=w.tau, map=lmap(w), causal=w.causal, key_len=dev["key_len"])
+def _calls(w, dev, ws, projection="retained"):
+    kw = dict(tau=w.tau, map=lmap(w), causal=w.causal, key_len=dev["key_len"], projection=projection)
     o, lse = rp.relpos_attn_fwd(dev["q"], dev["k"], dev["v"], dev["aq"], dev["ak"], dev["b"], workspace=ws, **kw)
     fwd_status = _status(ws)
     grads = rp.relpos_attn_bwd(dev["do"], dev["q"], dev["k"], dev["v"], o, lse, dev["aq"], dev["ak"], dev["b"],
@@ -36,19 +36,20 @@ def _status(ws):
         return -5
 
 
-def test_wait_limit_expiry_reports_timeout_then_recovers():
-    w = make_workload("shaw_clip16_n256")
+@pytest.mark.parametrize("projection", ["retained", "recompute"])
+def test_wait_limit_expiry_reports_timeout_then_recovers(projection):
+    w = make_workload("shaw_clip16_n256")     # q.aQ only: both projection modes apply
     dev = to_dev(w)
-    f, b = rp.workspace_size(dev["q"], dev["aq"], dev["ak"], dev["b"], w.tau, lmap(w))
+    f, b = rp.workspace_size(dev["q"], dev["aq"], dev["ak"], dev["b"], w.tau, lmap(w), projection=projection)
     ws = torch.empty(max(f, b), device="cuda", dtype=torch.uint8)
     try:
         bd.set_wait_limit_ns(1)
-        _, _, _, fwd_status, bwd_status = _calls(w, dev, ws)
+        _, _, _, fwd_status, bwd_status = _calls(w, dev, ws, projection)
     finally:
         bd.set_wait_limit_ns(0)
     assert fwd_status == -5 and bwd_status == -5
     # same device, same workspace, default limit: clean status, correct results
-    o, lse, (dq, dk, dv, daq, dak, db), fwd_status, bwd_status = _calls(w, dev, ws)
+    o, lse, (dq, dk, dv, daq, dak, db), fwd_status, bwd_status = _calls(w, dev, ws, projection)
     assert fwd_status == 0 and bwd_status == 0
     f64 = lambda t: None if t is None else t.double().cpu().numpy()
     got = dict(o=f64(o), lse=f64(lse), dq=f64(dq), dk=f64(dk), dv=f64(dv), daq=f64(daq), dak=f64(dak), db=f64(db))

@@ -107,6 +107,10 @@ def test_validation_rejects_before_launch(lib):
     assert lib.relpos_workspace_size(ctypes.byref(_args(dtype=bd.F32)), ctypes.byref(f), ctypes.byref(b)) == -2
     assert lib.relpos_workspace_size(ctypes.byref(_args(N=0)), ctypes.byref(f), ctypes.byref(b)) == -1
     assert lib.relpos_workspace_size(ctypes.byref(_args(mask=8)), ctypes.byref(f), ctypes.byref(b)) == -2
+    for bad_tau in (0.0, -0.125, float("nan"), float("inf")):
+        a = _args()
+        a.tau = bad_tau
+        assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == -1, bad_tau
     assert lib.relpos_workspace_size(ctypes.byref(_args(kind="truncated", clip=-1)), ctypes.byref(f), ctypes.byref(b)) == -1
     a = _args()
     a.map.kind = 9
@@ -182,3 +186,26 @@ def test_identity_grouped_projection_reach(lib):
     G = 128
     zq = H * sum(G * (g * G + G) for g in range(N // G)) * 4
     assert zq <= f.value <= zq + (32 << 20)
+
+
+def test_recompute_projection_forward_workspace_is_linear(lib):
+    """Projection recomputed per tile: the forward workspace of the identity map
+    (the Transformer-XL layer, N = 16384, 8 heads, q.aQ and b) holds no
+    projection at all, O(B H N) instead of the retained O(B H N^2); the
+    backward, which rebuilds Z^Q, keeps its size.  The key-side term is not
+    available in this mode, and an unknown mode is rejected."""
+    N, B, H = 16384, 1, 8
+    a = _args(B=B, H=H, N=N, kind="identity", ak=False, mask=1, per_head=1)
+    f, b = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == 0
+    f_ret, b_ret = f.value, b.value
+    assert f_ret > B * H * N * N * 4 / 4          # retained: the quadratic Z^Q (causal: about half of N^2)
+    a.projection = 1
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == 0
+    assert f.value <= B * H * (2 * N - 1) * 4 + (4 << 20)   # expanded bias and group records only
+    assert b.value == b_ret
+    a.ak = 1 << 20
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == -2
+    a = _args()
+    a.projection = 2
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == -1
