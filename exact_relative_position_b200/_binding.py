@@ -17,7 +17,7 @@ from .build import LIBPATH
 
 RELPOS_OK = 0
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "workspace", -4: "cuda error", -5: "timeout"}
-MAP_KINDS = {"truncated": 0, "identity": 1, "t5": 2, "log": 3}
+MAP_KINDS = {"truncated": 0, "identity": 1, "t5": 2, "log": 3, "log_rev": 4}
 MASK_CAUSAL, MASK_KEY_PADDING = 1, 2
 PROJECTION_MODES = {"retained": 0, "recompute": 1}
 F16, BF16, F32 = 0, 1, 2

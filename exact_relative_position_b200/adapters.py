@@ -1,4 +1,4 @@
-"""Model-level adapters over `relpos_attention`.
+"""Model-level adapters over `relpos_attention`: Transformer-XL and DeBERTa.
 
 Transformer-XL's relative attention written in the unified score of the paper
 digest ("Fast and Exact Relative-Position Attention via Structure-Aware
@@ -72,3 +72,47 @@ class TransformerXLRelPos(torch.nn.Module):
         qp, aq, b = self.unified_inputs(q)
         return relpos_attention(qp, k, v, aq, None, b, tau=self.tau, map=RelPosMap("identity"), causal=self.causal,
                                 projection=self.projection)
+
+
+class DebertaRelPos(torch.nn.Module):
+    """DeBERTa's disentangled attention over given content q, k, v.
+
+    score_ij = tau [ q_i . k_j  +  q_i . (E W_kr)[row(i - j)]  +  k_j . (E W_qr)[row(i - j)] ]
+
+    with E the relative-position embeddings [2 span, d_model], W_kr / W_qr the
+    per-head position-key and position-query projections, tau = 1/sqrt(3 d),
+    and row(x) the DeBERTa log-bucket row of the query-minus-key position x
+    (content-to-position and position-to-content both land on it).  In the
+    unified score of the paper digest (Eq. (1)) this is aQ = E W_kr,
+    aK = E W_qr with the map 'log_rev' (the log row of -delta, delta = j - i),
+    one table pair per head.  Gradients reach E, W_kr and W_qr through
+    PyTorch's autograd around the kernel's daQ / daK.  forward(q, k, v,
+    key_len=None) with q, k, v [B, H, N, d_head] fp16/bf16 on the GPU returns
+    O [B, H, N, d_head]; key_len [B] masks padded keys.
+    """
+
+    def __init__(self, n_heads: int, d_head: int = 64, d_model: int | None = None, span: int = 256,
+                 max_position: int = 512, tau: float | None = None, init_std: float = 0.02):
+        super().__init__()
+        self.n_heads, self.d_head = n_heads, d_head
+        self.d_model = d_model or n_heads * d_head
+        self.span, self.max_position = span, max_position
+        self.tau = tau if tau is not None else 1.0 / math.sqrt(3 * d_head)
+        self.rel_embeddings = torch.nn.Parameter(torch.randn(2 * span, self.d_model) * init_std)
+        self.W_kr = torch.nn.Parameter(torch.randn(n_heads, self.d_model, d_head) * init_std)
+        self.W_qr = torch.nn.Parameter(torch.randn(n_heads, self.d_model, d_head) * init_std)
+
+    def rel_map(self) -> RelPosMap:
+        return RelPosMap("log_rev", num_buckets=self.span, max_distance=self.max_position)
+
+    def unified_inputs(self, dtype):
+        """aQ = E W_kr and aK = E W_qr, [H, 2 span, d] each, in the kernel's dtype."""
+        ct = torch.promote_types(self.rel_embeddings.dtype, torch.float32)   # at least fp32 for the products
+        E = self.rel_embeddings.to(ct)
+        aq = torch.einsum("rc,hcd->hrd", E, self.W_kr.to(ct)).to(dtype).contiguous()
+        ak = torch.einsum("rc,hcd->hrd", E, self.W_qr.to(ct)).to(dtype).contiguous()
+        return aq, ak
+
+    def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, key_len=None) -> torch.Tensor:
+        aq, ak = self.unified_inputs(q.dtype)
+        return relpos_attention(q, k, v, aq, ak, None, tau=self.tau, map=self.rel_map(), key_len=key_len)

@@ -170,7 +170,8 @@ int check_map(const relpos_map_desc* m) {
       if (m->max_distance <= h / 2) return RELPOS_ERR_INVALID_ARG;
       return RELPOS_OK;
     }
-    case RELPOS_MAP_BUCKET_LOG: {
+    case RELPOS_MAP_BUCKET_LOG:
+    case RELPOS_MAP_BUCKET_LOG_REVERSED: {
       if (m->num_buckets < 2 || m->num_buckets > 65536) return RELPOS_ERR_INVALID_ARG;
       if (m->max_distance - 1 <= m->num_buckets / 2) return RELPOS_ERR_INVALID_ARG;
       return RELPOS_OK;
@@ -264,7 +265,8 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   p->zk_head = ak ? zk_head : 0;
   L->R = rows_of(a->map, N);
   L->Hq = a->table_per_head ? a->H : 1;
-  L->expand = a->map.kind == RELPOS_MAP_BUCKET_T5 || a->map.kind == RELPOS_MAP_BUCKET_LOG;
+  L->expand = a->map.kind == RELPOS_MAP_BUCKET_T5 || a->map.kind == RELPOS_MAP_BUCKET_LOG ||
+              a->map.kind == RELPOS_MAP_BUCKET_LOG_REVERSED;
   L->recompute = a->projection == RELPOS_PROJECTION_RECOMPUTE;
   const size_t BH = (size_t)a->B * a->H;
   size_t off = 0;

@@ -74,6 +74,7 @@ RP_HD int phi_of(const relpos_map_desc& m, int N, int delta) {
     case RELPOS_MAP_TRUNCATED: return iclamp(delta, -m.clip, m.clip) + m.clip;
     case RELPOS_MAP_IDENTITY: return delta + N - 1;
     case RELPOS_MAP_BUCKET_T5: return phi_t5(delta, m.num_buckets, m.max_distance, m.bidirectional);
+    case RELPOS_MAP_BUCKET_LOG_REVERSED: return phi_log(-delta, m.num_buckets, m.max_distance);
     default: return phi_log(delta, m.num_buckets, m.max_distance);
   }
 }

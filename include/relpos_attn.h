@@ -60,8 +60,12 @@ typedef enum {
   RELPOS_MAP_TRUNCATED = 0,   /* phi = clamp(delta, -clip, clip) + clip; R = 2 clip + 1 */
   RELPOS_MAP_IDENTITY = 1,    /* phi = delta + N - 1; R = 2N - 1 */
   RELPOS_MAP_BUCKET_T5 = 2,   /* T5 buckets (num_buckets, max_distance, bidirectional); R = num_buckets */
-  RELPOS_MAP_BUCKET_LOG = 3   /* DeBERTa log buckets (num_buckets = span k, max_distance = max
+  RELPOS_MAP_BUCKET_LOG = 3,  /* DeBERTa log buckets (num_buckets = span k, max_distance = max
                                  position); R = 2 num_buckets */
+  RELPOS_MAP_BUCKET_LOG_REVERSED = 4
+                              /* the LOG row of the reversed offset -delta = i - j: the
+                                 query-minus-key position by which DeBERTa's c2p and p2c terms
+                                 both index their relation rows; R = 2 num_buckets */
 } relpos_map_kind;
 
 typedef struct {

@@ -43,8 +43,11 @@ MASKED, CONST_LO, BAND, CONST_HI = 0, 1, 2, 3
 @dataclass(frozen=True)
 class MapDesc:
     """Offset map phi: 'truncated' (clip), 'identity', 't5' (num_buckets,
-    max_distance, bidirectional) or 'log' (DeBERTa: num_buckets = bucket span,
-    max_distance = max position)."""
+    max_distance, bidirectional), 'log' (DeBERTa log buckets: num_buckets =
+    bucket span, max_distance = max position) or 'log_rev' (the 'log' row of
+    the reversed offset -delta = i - j, the query-minus-key position by which
+    DeBERTa's content-to-position and position-to-content terms both index
+    their relation rows)."""
     kind: str
     clip: int = 0
     num_buckets: int = 0
@@ -117,7 +120,7 @@ def table_rows(m: MapDesc, N: int) -> int:
         return 2 * N - 1
     if m.kind == "t5":
         return m.num_buckets
-    if m.kind == "log":
+    if m.kind in ("log", "log_rev"):
         return 2 * m.num_buckets
     raise ValueError(m.kind)
 
@@ -131,6 +134,8 @@ def phi_of_delta(m: MapDesc, delta, N: int):
         return t5_bucket(delta, m.num_buckets, m.max_distance, m.bidirectional)
     if m.kind == "log":
         return log_bucket(delta, m.num_buckets, m.max_distance)
+    if m.kind == "log_rev":
+        return log_bucket(-np.asarray(delta, dtype=np.int64), m.num_buckets, m.max_distance)
     raise ValueError(m.kind)
 
 

@@ -26,7 +26,7 @@ from typing import Optional
 
 import torch
 
-MAP_KINDS = ("truncated", "identity", "t5", "log")
+MAP_KINDS = ("truncated", "identity", "t5", "log", "log_rev")
 
 
 def table_rows(map_kind: str, N: int, clip: int = 0, num_buckets: int = 0) -> int:
@@ -37,7 +37,7 @@ def table_rows(map_kind: str, N: int, clip: int = 0, num_buckets: int = 0) -> in
         return 2 * N - 1
     if map_kind == "t5":
         return num_buckets
-    if map_kind == "log":
+    if map_kind in ("log", "log_rev"):
         return 2 * num_buckets
     raise ValueError(map_kind)
 

@@ -35,3 +35,28 @@ def test_unified_score_equals_transformer_xl_score():
                 unified = qp[0, h, i] @ k[0, h, j] + qp[0, h, i] @ rel[h, r] + b[h, r]
                 txl = (q[0, h, i] + layer.u[h]) @ k[0, h, j] + (q[0, h, i] + layer.v[h]) @ rel[h, r]
                 assert abs(float(unified - txl)) < 1e-12
+
+
+def test_deberta_unified_score_equals_disentangled_score():
+    """The DeBERTa adapter's tables in the unified score, q.k + q.aQ[phi] + k.aK[phi]
+    with phi = 'log_rev', equal DeBERTa's c2c + c2p + p2c in every cell, c2p and
+    p2c read at the log-bucket row of the query-minus-key position i - j."""
+    import oracle as orc
+    from exact_relative_position_b200.adapters import DebertaRelPos
+    torch.manual_seed(1)
+    H, N, d, span, md = 2, 23, 4, 4, 12
+    layer = DebertaRelPos(H, d, d_model=6, span=span, max_position=md, init_std=0.5).double()
+    q, k = torch.randn(1, H, N, d, dtype=torch.float64), torch.randn(1, H, N, d, dtype=torch.float64)
+    with torch.no_grad():
+        Kr = torch.einsum("rc,hcd->hrd", layer.rel_embeddings, layer.W_kr)
+        Qr = torch.einsum("rc,hcd->hrd", layer.rel_embeddings, layer.W_qr)
+        aq, ak = layer.unified_inputs(torch.float64)
+    m = layer.rel_map()
+    phi = orc.phi_matrix(orc.MapDesc(m.kind, num_buckets=m.num_buckets, max_distance=m.max_distance), N)
+    for h in range(H):
+        for i in range(N):
+            for j in range(N):
+                row = int(orc.log_bucket(i - j, span, md))
+                deberta = q[0, h, i] @ k[0, h, j] + q[0, h, i] @ Kr[h, row] + k[0, h, j] @ Qr[h, row]
+                unified = q[0, h, i] @ k[0, h, j] + q[0, h, i] @ aq[h, phi[i, j]] + k[0, h, j] @ ak[h, phi[i, j]]
+                assert abs(float(unified - deberta)) < 1e-12

@@ -23,6 +23,7 @@ MAPS = {
     "t5": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=1),
     "t5uni": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=0),
     "log": dict(map_kind="log", num_buckets=32, max_distance=128),
+    "log_rev": dict(map_kind="log_rev", num_buckets=32, max_distance=128),
 }
 
 
@@ -63,6 +64,8 @@ CASES = [
     ("t5uni", 300, ("b",), True, None, torch.float16, False),
     ("log", 300, ("aQ", "aK"), False, [300, 290], torch.float16, True),
     ("log", 777, ("aQ", "aK", "b"), False, None, torch.bfloat16, False),
+    ("log_rev", 600, ("aQ", "aK"), False, [600, 431], torch.float16, True),
+    ("log_rev", 300, ("aQ", "aK", "b"), True, None, torch.float16, False),
     ("trunc16", 200, (), False, None, torch.float16, False),
     ("trunc16", 200, ("aK",), True, None, torch.float16, False),
 ]

@@ -41,6 +41,7 @@ MAPS = [
     ("t5", dict(num_buckets=32, max_distance=128, bidirectional=1)),
     ("t5", dict(num_buckets=32, max_distance=128, bidirectional=0)),
     ("log", dict(num_buckets=256, max_distance=512)), ("log", dict(num_buckets=16, max_distance=64)),
+    ("log_rev", dict(num_buckets=256, max_distance=512)), ("log_rev", dict(num_buckets=16, max_distance=64)),
 ]
 
 

@@ -114,6 +114,53 @@ def test_log_bucket_saturation_and_coverage():
     assert orc.expanded_bounds(orc.MapDesc("log", num_buckets=256, max_distance=512), 2048) == (-512, 506)
 
 
+@pytest.mark.parametrize("nb,md", [(256, 512), (64, 512)])
+def test_log_rev_map_matches_high_precision(nb, md):
+    """'log_rev' is the DeBERTa bucket row of the query-minus-key position
+    i - j = -delta: the decimal evaluation of the log formula at -delta."""
+    deltas = np.arange(-4000, 4001)
+    got = orc.phi_of_delta(orc.MapDesc("log_rev", num_buckets=nb, max_distance=md), deltas, 5000)
+    want = np.array([_log_decimal(-int(x), nb, md) for x in deltas])
+    assert np.array_equal(got, want)
+
+
+def test_log_rev_saturation_closed_forms():
+    m = orc.MapDesc("log_rev", num_buckets=256, max_distance=512)
+    d = np.arange(-3000, 3001)
+    rows = orc.phi_of_delta(m, d, 3001)
+    assert np.all(np.diff(rows) <= 0)                   # monotone, decreasing in delta = j - i
+    # mirror of the 'log' map's closed forms: row 511 iff delta <= -506, row 0 iff delta >= 512
+    assert rows[d == -506][0] == 511 and rows[d == -505][0] == 510
+    assert rows[d == 512][0] == 0 and rows[d == 511][0] == 1
+    assert orc.expanded_bounds(m, 2048) == (-506, 512)
+    assert orc.table_rows(m, 2048) == 512
+
+
+def test_deberta_disentangled_score_is_unified_with_log_rev():
+    """DeBERTa's disentangled score, built the way its attention forms it --
+    c2p gathers q_i . K^r at the bucket row of the relative position i - j;
+    p2c gathers k . Q^r key-major at the row of the negated relative position
+    and is then transposed -- equals Eq. (1) with aQ = K^r, aK = Q^r and the
+    one map 'log_rev' (both terms land on the row of i - j)."""
+    N, d, nb, md = 37, 4, 8, 24
+    rng = np.random.default_rng(11)
+    q, k = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    Kr, Qr = rng.standard_normal((2 * nb, d)), rng.standard_normal((2 * nb, d))
+    tau = 1.0 / math.sqrt(3 * d)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    rel = i - j                                          # relative position, query minus key
+    c2p_idx = orc.log_bucket(rel, nb, md)                # [query, key]
+    c2p = np.take_along_axis(q @ Kr.T, c2p_idx, axis=1)
+    p2c_idx = orc.log_bucket(-rel, nb, md)               # the negated relative position matrix
+    g = np.take_along_axis(k @ Qr.T, p2c_idx, axis=1)    # rows of the key-major product
+    p2c = g.T
+    want = tau * (q @ k.T + c2p + p2c)
+    phi = orc.phi_matrix(orc.MapDesc("log_rev", num_buckets=nb, max_distance=md), N)
+    got = orc.head_scores(q, k, Kr, Qr, None, tau, phi, np.ones((N, N), bool))
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
 def test_truncated_identity_closed_forms():
     d = np.arange(-50, 51)
     assert np.array_equal(orc.phi_truncated(d, 16), np.minimum(np.maximum(d, -16), 16) + 16)
