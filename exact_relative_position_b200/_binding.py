@@ -38,7 +38,7 @@ class relpos_fwd_args(ctypes.Structure):
                 ("v", ctypes.c_void_p), ("aq", ctypes.c_void_p), ("ak", ctypes.c_void_p),
                 ("b", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
                 ("dropout_p", ctypes.c_float), ("dropout_offset", ctypes.c_uint32), ("dropout_seed", ctypes.c_uint64),
-                ("projection", ctypes.c_int32)]
+                ("projection", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p), ("total_tokens", ctypes.c_int32)]
 
 
 class relpos_bwd_args(ctypes.Structure):
@@ -172,9 +172,27 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise RelPosError(f"unsupported dtype {dt}")
 
 
+def _shape(q, cu_seqlens=None, max_seqlen=None):
+    """(B, H, N, d): q is [B, H, N, d], or packed [T, H, d] with cu_seqlens [B + 1]
+    and max_seqlen = N (the longest sequence)."""
+    if cu_seqlens is None:
+        return tuple(q.shape)
+    if q.dim() != 3 or max_seqlen is None:
+        raise RelPosError("a packed batch needs q as [total_tokens, H, d] and max_seqlen")
+    if not cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise RelPosError("cu_seqlens must be an int32 CUDA tensor [B + 1]")
+    T, H, d = q.shape
+    return cu_seqlens.numel() - 1, H, int(max_seqlen), d
+
+
+def _lse_shape(q, cu_seqlens=None, max_seqlen=None):
+    B, H, N, _ = _shape(q, cu_seqlens, max_seqlen)
+    return (B, H, N) if cu_seqlens is None else (H, q.shape[0])
+
+
 def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o=None, lse=None,
-              dropout=(0.0, 0, 0), projection="retained"):
-    B, H, N, d = q.shape
+              dropout=(0.0, 0, 0), projection="retained", cu_seqlens=None, max_seqlen=None):
+    B, H, N, d = _shape(q, cu_seqlens, max_seqlen)
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda or not t.is_contiguous() or t.shape != q.shape or t.dtype != q.dtype:
             raise RelPosError(f"{name} must be a contiguous CUDA tensor shaped and typed like q")
@@ -203,12 +221,15 @@ def _fwd_args(q, k, v, aq, ak, b, tau, m: RelPosMap, causal, key_len, out_f32, o
     if projection not in PROJECTION_MODES:
         raise RelPosError(f"projection must be one of {sorted(PROJECTION_MODES)}")
     a.projection = PROJECTION_MODES[projection]
+    if cu_seqlens is not None:
+        a.cu_seqlens, a.total_tokens = cu_seqlens.data_ptr(), q.shape[0]
     return a
 
 
 def workspace_size(q, aq, ak, b, tau, m: RelPosMap, causal=False, key_len=None, out_f32=False,
-                   projection="retained"):
-    a = _fwd_args(q, q, q, aq, ak, b, tau, m, causal, key_len, out_f32, projection=projection)
+                   projection="retained", cu_seqlens=None, max_seqlen=None):
+    a = _fwd_args(q, q, q, aq, ak, b, tau, m, causal, key_len, out_f32, projection=projection,
+                  cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)
     f, bw = ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
     return f.value, bw.value
@@ -221,20 +242,21 @@ def _stream(dev) -> int:
 def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap, causal: bool = False,
                     key_len=None, out_f32: bool = False, workspace=None, o=None, lse=None,
                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0,
-                    projection: str = "retained"):
+                    projection: str = "retained", cu_seqlens=None, max_seqlen=None):
     """Forward through the C ABI.  Returns (O, LSE); O is float32 when out_f32.
     Attention dropout with rate dropout_p uses the Philox mask of (seed, offset);
     the backward needs the same three values.  projection="recompute" projects
-    q.aQ inside every tile instead of storing Z^Q (linear forward memory)."""
-    B, H, N, d = q.shape
+    q.aQ inside every tile instead of storing Z^Q (linear forward memory).
+    Packed variable-length batch: q, k, v [T, H, d] with cu_seqlens (int32
+    CUDA [B + 1]) and max_seqlen; LSE is then [H, T]."""
     if o is None:
         o = torch.empty(q.shape, device=q.device, dtype=torch.float32 if out_f32 else q.dtype)
     if lse is None:
-        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+        lse = torch.empty(_lse_shape(q, cu_seqlens, max_seqlen), device=q.device, dtype=torch.float32)
     if key_len is not None:
         key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse,
-                  (dropout_p, dropout_seed, dropout_offset), projection)
+                  (dropout_p, dropout_seed, dropout_offset), projection, cu_seqlens, max_seqlen)
     f, bw = ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(bw)), "relpos_workspace_size")
     if workspace is None or workspace.numel() < f.value:
@@ -247,7 +269,7 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
 def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: float, map: RelPosMap,
                     causal: bool = False, key_len=None, workspace=None, grads=None, reuse_forward: bool = False,
                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0,
-                    projection: str = "retained"):
+                    projection: str = "retained", cu_seqlens=None, max_seqlen=None):
     """Backward through the C ABI.  Returns (dq, dk, dv, daq, dak, db).
 
     reuse_forward: `workspace` is the one the forward with these same arguments
@@ -259,7 +281,7 @@ def relpos_attn_bwd(dout, q, k, v, o, lse, aq=None, ak=None, b=None, *, tau: flo
     if not dout.is_contiguous() or dout.dtype != q.dtype or dout.shape != q.shape:
         raise RelPosError("dout must be contiguous, shaped and typed like q")
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse,
-                  (dropout_p, dropout_seed, dropout_offset), projection)
+                  (dropout_p, dropout_seed, dropout_offset), projection, cu_seqlens, max_seqlen)
     g = relpos_bwd_args()
     g.fwd = a
     if grads is None:
@@ -341,11 +363,10 @@ def relpos_attn_fwd_noalloc(q, k, v, aq=None, ak=None, b=None, *, tau: float, ma
                             key_len=None, out_f32: bool = False, o=None, lse=None, projection: str = "retained"):
     """Forward through relpos_attn_fwd_noalloc: the library's fixed 32 MiB scratch
     array replaces the workspace, so the call needs no device allocation for it."""
-    B, H, N, d = q.shape
     if o is None:
         o = torch.empty(q.shape, device=q.device, dtype=torch.float32 if out_f32 else q.dtype)
     if lse is None:
-        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+        lse = torch.empty(_lse_shape(q), device=q.device, dtype=torch.float32)
     if key_len is not None:
         key_len = key_len.to(device=q.device, dtype=torch.int32).contiguous()
     a = _fwd_args(q, k, v, aq, ak, b, tau, map, causal, key_len, out_f32, o, lse, projection=projection)

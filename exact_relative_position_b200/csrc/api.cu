@@ -255,6 +255,13 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   p->seed_lo = (uint32_t)(a->dropout_seed & 0xFFFFFFFFull);
   p->seed_hi = (uint32_t)(a->dropout_seed >> 32);
   p->drop_offset = a->dropout_offset;
+  if (a->cu_seqlens) {
+    // packed variable-length batch: the sequence lengths mask the keys
+    if ((a->mask & RELPOS_MASK_KEY_PADDING) || a->total_tokens < 1) return RELPOS_ERR_INVALID_ARG;
+    p->packed = 1;
+    p->T = a->total_tokens;
+    p->cu = a->cu_seqlens;
+  }
   {
     const unsigned long long lim = g_wait_limit_ns.load();
     p->wait_ns = lim ? lim : (unsigned long long)sm100::kTimeoutNs;

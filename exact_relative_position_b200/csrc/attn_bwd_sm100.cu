@@ -48,18 +48,25 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // rows past N (up to a whole tile) get D = 0 and LSE = +inf (so P = 0).  A
 // row whose keys were all masked (LSE = -inf) also gets +inf.
 template <typename OT, typename T>
-__global__ void __launch_bounds__(256) prep_sm100_kernel(const OT* __restrict__ o, const T* __restrict__ dout,
-                                                         const float* __restrict__ lse, float* __restrict__ dsum,
-                                                         float* __restrict__ lse2, int N, int npad, long long BH) {
+__global__ void __launch_bounds__(256) prep_sm100_kernel(const Plan p, const OT* __restrict__ o,
+                                                         const T* __restrict__ dout, const float* __restrict__ lse,
+                                                         float* __restrict__ dsum, float* __restrict__ lse2,
+                                                         int npad, long long BH) {
   const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = gt >> 3;
   const int part = (int)(gt & 7);
   const long long bh = row / npad;
   const int i = (int)(row - bh * npad);
+  const int b = (int)(bh / p.H), h = (int)(bh - (long long)b * p.H);
+  SeqRows sr;
+  sr.row0 = 0;
+  sr.len = 0;
+  if (bh < BH) sr = seq_rows(p, b);
   float acc = 0.f;
-  const bool ok = bh < BH && i < N;
+  // rows past the sequence get D = 0 and LSE = +inf, so P = 0 in both passes
+  const bool ok = bh < BH && i < sr.len;
   if (ok) {
-    const size_t off = ((size_t)bh * N + i) * 64 + part * 8;
+    const size_t off = (size_t)act_row(p, sr, b, h, i) * 64 + part * 8;
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc += (float)o[off + c] * (float)dout[off + c];
   }
@@ -70,7 +77,7 @@ __global__ void __launch_bounds__(256) prep_sm100_kernel(const OT* __restrict__ 
     dsum[row] = acc;
     float l2 = INFINITY;
     if (ok) {
-      const float l = lse[(size_t)bh * N + i];
+      const float l = lse[lse_index(p, sr, b, h, i)];
       if (l != -INFINITY) l2 = l * kLog2e;
     }
     lse2[row] = l2;
@@ -127,10 +134,13 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
   const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, q0 = qt * kT;
   const int npad = p.nT * kT;
-  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
+  const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
+  // keys j >= nkv are masked: the sequence length (packed), or the clamped key length
+  const int nkv = p.packed ? sr.len : (p.padding ? iclamp(p.key_len[b], 0, N) : N);
   int kend = nkv;
   if (p.causal) kend = imin(kend, imin(q0 + kT, N));
-  const int nkt = kend > 0 ? (kend + kT - 1) / kT : 0;
+  // nothing to do for a query tile past the sequence (packed batches)
+  const int nkt = (kend > 0 && q0 < sr.len) ? (kend + kT - 1) / kT : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
@@ -172,8 +182,10 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         prefetch_tmap(&tmV);
         prefetch_tmap(&tmDO);
         mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
-        tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
-        tma_load_3d(sb + kOffDO, &tmDO, bar(kBarQ), 0, q0, bh);
+        int c1, c2;
+        tma_rows(p, sr, bh, h, q0, c1, c2);
+        tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, c1, c2);
+        tma_load_3d(sb + kOffDO, &tmDO, bar(kBarQ), 0, c1, c2);
         int issued = 0;
   #pragma unroll 1
         for (int it = 0; it < nkt; ++it) {
@@ -181,8 +193,9 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag, p.wait_ns)) break;
           const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
           mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
-          tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kT, bh);
-          tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kT, bh);
+          tma_rows(p, sr, bh, h, it * kT, c1, c2);
+          tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, c1, c2);
+          tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, c1, c2);
           if (AK) {
             const float* src = t.zk_sat + (size_t)bh * 2 * npad + (size_t)it * kT;
             bulk_load(dst + 2 * kTileBytes, src, kT * 4, bar(kBarKvFull + s));
@@ -275,7 +288,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     const int cb = 64 * hc;
     const int r = (warp & 3) * 32 + lane;
     const int i = q0 + r;
-    const bool rok = i < N;
+    const bool rok = i < sr.len;
     const uint32_t t_lane = (uint32_t)((warp & 3) * 32) << 16;
     const float sc = p.tau * kLog2e;
     const size_t prow = (size_t)bh * npad + q0 + r;
@@ -324,18 +337,26 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       // P = 2^(S tau log2e + relation terms - LSE log2e)
       if (is_const) {
         const float off = (cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi) - lse2;
+        // paired fp32 arithmetic: one instruction per two scores
+        const float2 sc2 = make_float2(sc, sc), off2 = make_float2(off, off);
         if (AK) {
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
             const float4 v4 = *reinterpret_cast<const float4*>(cv + c);
-            x[c] = fast_exp2(fmaf(x[c], sc, v4.x) + off);
-            x[c + 1] = fast_exp2(fmaf(x[c + 1], sc, v4.y) + off);
-            x[c + 2] = fast_exp2(fmaf(x[c + 2], sc, v4.z) + off);
-            x[c + 3] = fast_exp2(fmaf(x[c + 3], sc, v4.w) + off);
+            const float2 z0 = ffma2(make_float2(x[c], x[c + 1]), sc2, fadd2(make_float2(v4.x, v4.y), off2));
+            const float2 z1 = ffma2(make_float2(x[c + 2], x[c + 3]), sc2, fadd2(make_float2(v4.z, v4.w), off2));
+            x[c] = fast_exp2(z0.x);
+            x[c + 1] = fast_exp2(z0.y);
+            x[c + 2] = fast_exp2(z1.x);
+            x[c + 3] = fast_exp2(z1.y);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = fast_exp2(fmaf(x[c], sc, off));
+          for (int c = 0; c < 64; c += 2) {
+            const float2 z = ffma2(make_float2(x[c], x[c + 1]), sc2, off2);
+            x[c] = fast_exp2(z.x);
+            x[c + 1] = fast_exp2(z.y);
+          }
         }
       } else {
         const float* zk_tile = nullptr;
@@ -349,8 +370,13 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         }
         band_terms_q<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, i, j0, cb, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
                                        imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
+        const float2 nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = fast_exp2(x[c] - lse2);
+        for (int c = 0; c < 64; c += 2) {
+          const float2 z = fadd2(make_float2(x[c], x[c + 1]), nl2);
+          x[c] = fast_exp2(z.x);
+          x[c + 1] = fast_exp2(z.y);
+        }
       }
       const bool need_mask = (j0 + kT > nkv) || (p.causal && j0 + kT - 1 > q0);
       if (need_mask) {
@@ -385,16 +411,19 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           }
         }
         if (!DZQ || is_const) {
-          float ssum[2] = {0.f, 0.f};
+          float2 ssum = make_float2(0.f, 0.f);
+          const float2 nd2 = make_float2(-dval, -dval);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float ds = x[c] * (__uint_as_float(dp[c]) - dval);
-            x[c] = ds;
-            if (DZQ) ssum[c & 1] += ds;
+          for (int c = 0; c < 64; c += 2) {
+            const float2 ds = fmul2(make_float2(x[c], x[c + 1]),
+                                    fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nd2));
+            x[c] = ds.x;
+            x[c + 1] = ds.y;
+            if (DZQ) ssum = fadd2(ssum, ds);
           }
           if (DZQ) {
-            if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
-            else sat_hi += ssum[0] + ssum[1];
+            if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum.x + ssum.y;
+            else sat_hi += ssum.x + ssum.y;
           }
         } else {
           // saturated cells summed here; the interior ones are stored below.
@@ -478,13 +507,13 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       for (int c = 0; c < 32; ++c) dq[c] = __uint_as_float(u[c]) * p.tau;
     }
     if (rok) {
-      const size_t o = ((size_t)bh * N + i) * 64 + 32 * hc;
       if (DQ32) {
-        float* dst = t.dq_acc + o;
+        // the fp32 accumulator keeps the workspace's dense layout
+        float* dst = t.dq_acc + ((size_t)bh * N + i) * 64 + 32 * hc;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dq[c], dq[c + 1], dq[c + 2], dq[c + 3]);
       } else {
-        T* dst = static_cast<T*>(t.dq) + o;
+        T* dst = static_cast<T*>(t.dq) + act_row(p, sr, b, h, i) * 64 + 32 * hc;
 #pragma unroll
         for (int c = 0; c < 32; c += 8) {
           uint4 w;
@@ -558,7 +587,9 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
   const int kt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, k0 = kt * kT;
   const int npad = p.nT * kT;
-  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
+  const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
+  // keys j >= nkv are masked: the sequence length (packed), or the clamped key length
+  const int nkv = p.packed ? sr.len : (p.padding ? iclamp(p.key_len[b], 0, N) : N);
   const int qt0 = p.causal ? kt : 0;            // queries i >= j only under the causal mask
   const int nq = k0 < nkv ? p.nT - qt0 : 0;
 
@@ -602,8 +633,10 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         prefetch_tmap(&tmV);
         prefetch_tmap(&tmDO);
         mbar_expect_tx(bar(kBarKV), 2 * kTileBytes);
-        tma_load_3d(sb + kOffK, &tmK, bar(kBarKV), 0, k0, bh);
-        tma_load_3d(sb + kOffV, &tmV, bar(kBarKV), 0, k0, bh);
+        int c1, c2;
+        tma_rows(p, sr, bh, h, k0, c1, c2);
+        tma_load_3d(sb + kOffK, &tmK, bar(kBarKV), 0, c1, c2);
+        tma_load_3d(sb + kOffV, &tmV, bar(kBarKV), 0, c1, c2);
         int issued = 0;
   #pragma unroll 1
         for (int it = 0; it < nq; ++it) {
@@ -613,8 +646,9 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           const uint32_t dst = sb + kOffQD + (uint32_t)s * kStageBytes;
           const uint32_t fb = bar(kBarQsFull + s);
           mbar_expect_tx(fb, 2 * kTileBytes + ((AQ || BIAS) ? kVecBytes : kVecBytes / 2));
-          tma_load_3d(dst, &tmQ, fb, 0, qb, bh);
-          tma_load_3d(dst + kTileBytes, &tmDO, fb, 0, qb, bh);
+          tma_rows(p, sr, bh, h, qb, c1, c2);
+          tma_load_3d(dst, &tmQ, fb, 0, c1, c2);
+          tma_load_3d(dst + kTileBytes, &tmDO, fb, 0, c1, c2);
           const size_t vo = (size_t)bh * npad + qb;
           bulk_load(dst + 2 * kTileBytes, t.lse2 + vo, kT * 4, fb);
           bulk_load(dst + 2 * kTileBytes + kT * 4, t.dsum + vo, kT * 4, fb);
@@ -717,7 +751,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     const int cb = 64 * hc;
     const int r = (warp & 3) * 32 + lane;
     const int j = k0 + r;
-    const bool jok = j < N;
+    const bool jok = j < sr.len;
     const bool jkeep = j < nkv;                  // keys past key_len are masked for every query
     const uint32_t t_lane = (uint32_t)((warp & 3) * 32) << 16;
     const float sc = p.tau * kLog2e;
@@ -764,18 +798,23 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       // P^T = 2^(S^T tau log2e + relation terms - LSE_i log2e), column c = query qb + cb + c
       if (is_const) {
         const float rowk = cls == RELPOS_TILE_CONST_LO ? rowk_lo : rowk_hi;
+        // paired fp32 arithmetic: one instruction per two scores
+        const float2 sc2 = make_float2(sc, sc), rk2 = make_float2(rowk, rowk);
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
-          float4 w4 = make_float4(-l4.x, -l4.y, -l4.z, -l4.w);
+          float2 w0 = fadd2(rk2, make_float2(-l4.x, -l4.y)), w1 = fadd2(rk2, make_float2(-l4.z, -l4.w));
           if (AQ || BIAS) {
             const float4 c4 = *reinterpret_cast<const float4*>(cvq + c);
-            w4.x += c4.x; w4.y += c4.y; w4.z += c4.z; w4.w += c4.w;
+            w0 = fadd2(w0, make_float2(c4.x, c4.y));
+            w1 = fadd2(w1, make_float2(c4.z, c4.w));
           }
-          x[c] = fast_exp2(fmaf(x[c], sc, w4.x) + rowk);
-          x[c + 1] = fast_exp2(fmaf(x[c + 1], sc, w4.y) + rowk);
-          x[c + 2] = fast_exp2(fmaf(x[c + 2], sc, w4.z) + rowk);
-          x[c + 3] = fast_exp2(fmaf(x[c + 3], sc, w4.w) + rowk);
+          const float2 z0 = ffma2(make_float2(x[c], x[c + 1]), sc2, w0);
+          const float2 z1 = ffma2(make_float2(x[c + 2], x[c + 3]), sc2, w1);
+          x[c] = fast_exp2(z0.x);
+          x[c + 1] = fast_exp2(z0.y);
+          x[c + 2] = fast_exp2(z1.x);
+          x[c + 3] = fast_exp2(z1.y);
         }
       } else {
         const float* zq_tile = nullptr;
@@ -792,10 +831,12 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
-          x[c] = fast_exp2(x[c] - l4.x);
-          x[c + 1] = fast_exp2(x[c + 1] - l4.y);
-          x[c + 2] = fast_exp2(x[c + 2] - l4.z);
-          x[c + 3] = fast_exp2(x[c + 3] - l4.w);
+          const float2 z0 = fadd2(make_float2(x[c], x[c + 1]), make_float2(-l4.x, -l4.y));
+          const float2 z1 = fadd2(make_float2(x[c + 2], x[c + 3]), make_float2(-l4.z, -l4.w));
+          x[c] = fast_exp2(z0.x);
+          x[c + 1] = fast_exp2(z0.y);
+          x[c + 2] = fast_exp2(z1.x);
+          x[c + 3] = fast_exp2(z1.y);
         }
       }
       const bool need_mask = !jkeep || (p.causal && k0 + kT - 1 > qb);
@@ -849,21 +890,22 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
             dp[c] = __float_as_uint(kept(c) ? __uint_as_float(dp[c]) * p.drop_scale : 0.f);
         }
         if (!DZK || is_const) {
-          float ssum[2] = {0.f, 0.f};
+          float2 ssum = make_float2(0.f, 0.f);
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
             const float4 d4 = *reinterpret_cast<const float4*>(dvec + c);
-            const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float ds = x[c + u] * (__uint_as_float(dp[c + u]) - dd[u]);
-              x[c + u] = ds;
-              if (DZK) ssum[u & 1] += ds;
-            }
+            const float2 ds0 = fmul2(make_float2(x[c], x[c + 1]),
+                                     fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                           make_float2(-d4.x, -d4.y)));
+            const float2 ds1 = fmul2(make_float2(x[c + 2], x[c + 3]),
+                                     fadd2(make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
+                                           make_float2(-d4.z, -d4.w)));
+            x[c] = ds0.x; x[c + 1] = ds0.y; x[c + 2] = ds1.x; x[c + 3] = ds1.y;
+            if (DZK) ssum = fadd2(ssum, fadd2(ds0, ds1));
           }
           if (DZK) {
-            if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum[0] + ssum[1];
-            else sat_hi += ssum[0] + ssum[1];
+            if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum.x + ssum.y;
+            else sat_hi += ssum.x + ssum.y;
           }
         } else {
           // column cc = query qb + cc of this key row: kept for
@@ -956,7 +998,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       for (int c = 0; c < 32; ++c) dk[c] = __uint_as_float(u[c]) * p.tau;
     }
     if (jok) {
-      const size_t o = ((size_t)bh * N + j) * 64 + 32 * hc;
+      const size_t o = (size_t)act_row(p, sr, b, h, j) * 64 + 32 * hc;
       T* vdst = static_cast<T*>(t.dv) + o;
 #pragma unroll
       for (int c = 0; c < 32; c += 8) {
@@ -968,7 +1010,8 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         *reinterpret_cast<uint4*>(vdst + c) = w;
       }
       if (DK32) {
-        float* dst = t.dk_acc + o;
+        // the fp32 accumulator keeps the workspace's dense layout
+        float* dst = t.dk_acc + ((size_t)bh * N + j) * 64 + 32 * hc;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dk[c], dk[c + 1], dk[c + 2], dk[c + 3]);
       } else {
@@ -1010,10 +1053,9 @@ struct Maps {
 };
 
 bool make_maps(const Plan& p, const Tensors& t, Maps& m) {
-  const int BH = p.B * p.H;
   const bool bf = t.is_bf16 != 0;
-  return make_rows_map(&m.q, t.q, BH, p.N, bf) && make_rows_map(&m.k, t.k, BH, p.N, bf) &&
-         make_rows_map(&m.v, t.v, BH, p.N, bf) && make_rows_map(&m.dout, t.dout, BH, p.N, bf);
+  return make_rows_map(&m.q, t.q, p, bf) && make_rows_map(&m.k, t.k, p, bf) && make_rows_map(&m.v, t.v, p, bf) &&
+         make_rows_map(&m.dout, t.dout, p, bf);
 }
 
 template <typename T>
@@ -1062,19 +1104,20 @@ cudaError_t launch_bwd_prep(const Plan& p, const Tensors& t, cudaStream_t s) {
   const unsigned blocks = nblocks(BH * npad * 8, 256);
   if (t.is_bf16) {
     if (t.o_f32) {
-      prep_sm100_kernel<float, __nv_bfloat16><<<blocks, 256, 0, s>>>((const float*)t.o, (const __nv_bfloat16*)t.dout,
-                                                                      t.lse, t.dsum, t.lse2, p.N, npad, BH);
+      prep_sm100_kernel<float, __nv_bfloat16><<<blocks, 256, 0, s>>>(p, (const float*)t.o,
+                                                                      (const __nv_bfloat16*)t.dout, t.lse, t.dsum,
+                                                                      t.lse2, npad, BH);
     } else {
       prep_sm100_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(
-          (const __nv_bfloat16*)t.o, (const __nv_bfloat16*)t.dout, t.lse, t.dsum, t.lse2, p.N, npad, BH);
+          p, (const __nv_bfloat16*)t.o, (const __nv_bfloat16*)t.dout, t.lse, t.dsum, t.lse2, npad, BH);
     }
   } else {
     if (t.o_f32) {
-      prep_sm100_kernel<float, __half><<<blocks, 256, 0, s>>>((const float*)t.o, (const __half*)t.dout, t.lse,
-                                                               t.dsum, t.lse2, p.N, npad, BH);
+      prep_sm100_kernel<float, __half><<<blocks, 256, 0, s>>>(p, (const float*)t.o, (const __half*)t.dout, t.lse,
+                                                               t.dsum, t.lse2, npad, BH);
     } else {
-      prep_sm100_kernel<__half, __half><<<blocks, 256, 0, s>>>((const __half*)t.o, (const __half*)t.dout, t.lse,
-                                                                t.dsum, t.lse2, p.N, npad, BH);
+      prep_sm100_kernel<__half, __half><<<blocks, 256, 0, s>>>(p, (const __half*)t.o, (const __half*)t.dout, t.lse,
+                                                                t.dsum, t.lse2, npad, BH);
     }
   }
   note_launch(1);

@@ -112,10 +112,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, q0 = blockIdx.x * (2 * kBQ);
-  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
+  const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
+  // keys j >= nkv are masked: the sequence length (packed), or the clamped key length
+  const int nkv = p.packed ? sr.len : (p.padding ? iclamp(p.key_len[b], 0, N) : N);
   int kend = nkv;
   if (p.causal) kend = imin(kend, imin(q0 + 2 * kBQ, N));
-  const int nkt = kend > 0 ? (kend + kBK - 1) / kBK : 0;
+  // nothing to do for query tiles past the sequence (packed batches)
+  const int nkt = (kend > 0 && q0 < sr.len) ? (kend + kBK - 1) / kBK : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
@@ -153,8 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       mbar_expect_tx(bar(kBarQ), 2 * kTileBytes);
-      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, q0, bh);
-      tma_load_3d(sb + kOffQ + kTileBytes, &tmQ, bar(kBarQ), 0, q0 + kBQ, bh);
+      int c1, c2;
+      tma_rows(p, sr, bh, h, q0, c1, c2);
+      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, c1, c2);
+      tma_rows(p, sr, bh, h, q0 + kBQ, c1, c2);
+      tma_load_3d(sb + kOffQ + kTileBytes, &tmQ, bar(kBarQ), 0, c1, c2);
       int issued = 0;
 #pragma unroll 1
       for (int it = 0; it < nkt; ++it) {
@@ -162,8 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag, p.wait_ns)) break;
         const uint32_t dst = sb + kOffKV + (uint32_t)s * kStageBytes;
         mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes + (AK ? kColvBytes : 0u));
-        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kBK, bh);
-        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kBK, bh);
+        tma_rows(p, sr, bh, h, it * kBK, c1, c2);
+        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, c1, c2);
+        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, c1, c2);
         if (AK) {
           const float* src = t.zk_sat + (size_t)bh * 2 * p.nT * kBK + (size_t)it * kBK;
           bulk_load(dst + 2 * kTileBytes, src, kBK * 4, bar(kBarKvFull + s));
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = wl * 32 + lane;
     const int qtile = (q0 >> 7) + g;
     const int i = q0 + g * kBQ + r;
-    const bool rok = i < N;
+    const bool rok = i < sr.len;
     const uint32_t t_lane = (uint32_t)(wl * 32) << 16;
     const uint32_t tS = tmem + t_lane + (uint32_t)g * 128;
     const uint32_t tO = tmem + t_lane + 256 + (uint32_t)g * 64;
@@ -439,9 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 64; ++c) ov[c] = __uint_as_float(u[c]) * inv;
     }
     if (rok) {
-      OutT* O = static_cast<OutT*>(t.o) + ((size_t)bh * N + i) * 64;
+      OutT* O = static_cast<OutT*>(t.o) + act_row(p, sr, b, h, i) * 64;
       RowStore<OutT>::row(O, ov);
-      t.lse[(size_t)bh * N + i] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      t.lse[lse_index(p, sr, b, h, i)] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
   tc_fence_before();
@@ -468,14 +475,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [BH, N, 64] 16-bit tensor viewed as 3-D for TMA: 128-row boxes, 128-byte
-// swizzle, rows past N read as zero.
-bool make_rows_map(CUtensorMap* m, const void* base, int BH, int N, bool bf16) {
+// A 16-bit activation tensor viewed as 3-D for TMA, 128-row boxes with
+// 128-byte swizzle: dense [B H, N, 64] as {64, N, B H}, rows past N read as
+// zero; packed [T, H, 64] as {64, H, T} (box 64 x 1 x 128, monotonic
+// strides), rows past T read as zero.  Either box lands in shared memory as
+// 128 rows of 128 bytes.  Coordinates: tma_rows.
+bool make_rows_map(CUtensorMap* m, const void* base, const Plan& p, bool bf16) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+  cuuint64_t dims[3] = {64, (cuuint64_t)p.N, (cuuint64_t)p.B * p.H};
+  cuuint64_t strides[2] = {128, (cuuint64_t)p.N * 128};
   cuuint32_t box[3] = {64, 128, 1};
+  if (p.packed) {
+    dims[1] = (cuuint64_t)p.H;
+    dims[2] = (cuuint64_t)p.T;
+    strides[1] = (cuuint64_t)p.H * 128;
+    box[1] = 1;
+    box[2] = 128;
+  }
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -511,8 +528,7 @@ cudaError_t launch_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   const int BH = p.B * p.H;
   const bool bf = t.is_bf16 != 0;
-  if (!make_rows_map(&mq, t.q, BH, p.N, bf) || !make_rows_map(&mk, t.k, BH, p.N, bf) ||
-      !make_rows_map(&mv, t.v, BH, p.N, bf))
+  if (!make_rows_map(&mq, t.q, p, bf) || !make_rows_map(&mk, t.k, p, bf) || !make_rows_map(&mv, t.v, p, bf))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;

@@ -132,10 +132,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, i0 = qt * kT;
-  const int nkv = p.padding ? iclamp(p.key_len[b], 0, N) : N;   // out-of-range lengths clamp into [0, N]
+  const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
+  // keys j >= nkv are masked: the sequence length (packed), or the clamped key length
+  const int nkv = p.packed ? sr.len : (p.padding ? iclamp(p.key_len[b], 0, N) : N);
   int kend = nkv;
   if (p.causal) kend = imin(kend, imin(i0 + kT, N));
-  const int nkt = kend > 0 ? (kend + kT - 1) / kT : 0;
+  // nothing to do for a query tile past the sequence (packed batches)
+  const int nkt = (kend > 0 && i0 < sr.len) ? (kend + kT - 1) / kT : 0;
   const int hq = t.table_per_head ? h : 0;
 
   if (threadIdx.x == 0) {
@@ -173,7 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmV);
       if (AQ) prefetch_tmap(&tmA);
       mbar_expect_tx(bar(kBarQ), kTileBytes);
-      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, i0, bh);
+      int c1, c2;
+      tma_rows(p, sr, bh, h, i0, c1, c2);
+      tma_load_3d(sb + kOffQ, &tmQ, bar(kBarQ), 0, c1, c2);
       int issued = 0, nwin = 0;
 #pragma unroll 1
       for (int it = 0; it < nkt; ++it) {
@@ -181,8 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it >= kStages && !mbar_wait(bar(kBarKvEmpty + s), ((it / kStages) - 1) & 1, abort_flag, p.wait_ns)) break;
         const uint32_t dst = sb + kOffKV + (uint32_t)s * 2 * kTileBytes;
         mbar_expect_tx(bar(kBarKvFull + s), 2 * kTileBytes);
-        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, it * kT, bh);
-        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, it * kT, bh);
+        tma_rows(p, sr, bh, h, it * kT, c1, c2);
+        tma_load_3d(dst, &tmK, bar(kBarKvFull + s), 0, c1, c2);
+        tma_load_3d(dst + kTileBytes, &tmV, bar(kBarKvFull + s), 0, c1, c2);
         issued = it + 1;
         if (AQ && band_tile(p, qt, it, nkv)) {
           // the previous window has been read by its Zt GEMM
@@ -273,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wl = warp & 3;
     const int r = wl * 32 + lane;
     const int i = i0 + r;
-    const bool rok = i < N;
+    const bool rok = i < sr.len;
     const uint32_t t_lane = (uint32_t)(wl * 32) << 16;
     const uint32_t tS = tmem + t_lane + kTmS;
     const uint32_t tO = tmem + t_lane + kTmO;
@@ -281,10 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tZ = tmem + t_lane + kTmZ + (uint32_t)(96 - 32 * wl);   // first column this warp reaches
     const float sc = p.tau * kLog2e;
     // the row's saturated projections q_i.aQ_exp[0] and q_i.aQ_exp[R_exp - 1]
-    // (rows past N use row N - 1, in bounds; their results are discarded)
+    // (rows past the sequence use its last row, in bounds; their results are discarded)
     float zq_lo = 0.f, zq_hi = 0.f;
-    if (AQ) {
-      const T* qrow = static_cast<const T*>(t.q) + ((size_t)bh * N + imin(i, N - 1)) * 64;
+    if (AQ && sr.len > 0) {
+      const T* qrow = static_cast<const T*>(t.q) + act_row(p, sr, b, h, imin(i, sr.len - 1)) * 64;
       const T* alo = static_cast<const T*>(t.aq_exp) + (size_t)hq * t.aq_hs;
       const T* ahi = alo + (size_t)(p.Rexp - 1) * 64;
 #pragma unroll 8
@@ -457,9 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 64; ++c) ov[c] = __uint_as_float(u[c]) * inv;
     }
     if (rok) {
-      OutT* O = static_cast<OutT*>(t.o) + ((size_t)bh * N + i) * 64;
+      OutT* O = static_cast<OutT*>(t.o) + act_row(p, sr, b, h, i) * 64;
       RowStoreRc<OutT>::row(O, ov);
-      t.lse[(size_t)bh * N + i] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      t.lse[lse_index(p, sr, b, h, i)] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
   tc_fence_before();
@@ -506,8 +512,7 @@ cudaError_t launch_rc_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   CUtensorMap mq, mk, mv, ma;
   const int BH = p.B * p.H;
   const bool bf = t.is_bf16 != 0;
-  if (!make_rows_map(&mq, t.q, BH, p.N, bf) || !make_rows_map(&mk, t.k, BH, p.N, bf) ||
-      !make_rows_map(&mv, t.v, BH, p.N, bf))
+  if (!make_rows_map(&mq, t.q, p, bf) || !make_rows_map(&mk, t.k, p, bf) || !make_rows_map(&mv, t.v, p, bf))
     return cudaErrorInvalidValue;
   memset(&ma, 0, sizeof(ma));
   if (t.aq_exp && !make_table_map(&ma, t.aq_exp, t.table_per_head ? p.H : 1, p.Rexp, t.aq_hs, bf))

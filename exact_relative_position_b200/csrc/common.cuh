@@ -109,7 +109,47 @@ struct Plan {
   // limit of every bounded mbarrier wait in the fused kernels (ns); the host
   // lowers it only to exercise the timeout path
   unsigned long long wait_ns;
+  // packed variable-length batch (0: the dense [B, H, N, 64] layout): sequence
+  // b owns token rows cu[b] .. cu[b + 1] - 1 of token-major [T, H, 64] tensors
+  // and of the LSE [H, T]; N is the longest sequence.  The workspace keeps
+  // its dense per-(batch, head) layout of N rows.
+  int packed, T;
+  const int* cu;
 };
+
+// First token row and length of sequence b.  Packed offsets are clamped so
+// that every row a kernel stores stays inside [0, T) and every length inside
+// [0, N], whatever the offsets hold; the dense layout has length N.
+struct SeqRows {
+  int row0, len;
+};
+RP_HD SeqRows seq_rows(const Plan& p, int b) {
+  SeqRows s;
+  if (!p.packed) {
+    s.row0 = 0;
+    s.len = p.N;
+    return s;
+  }
+  s.row0 = iclamp(p.cu[b], 0, p.T);
+  s.len = iclamp(p.cu[b + 1] - s.row0, 0, imin(p.N, p.T - s.row0));
+  return s;
+}
+// Row i of (b, h) of q / k / v / o / dout / dq / dk / dv, in units of 64-element rows.
+RP_HD long long act_row(const Plan& p, const SeqRows& s, int b, int h, int i) {
+  return p.packed ? (long long)(s.row0 + i) * p.H + h : ((long long)b * p.H + h) * p.N + i;
+}
+// Entry of row i of (b, h) in the LSE ([B, H, N] dense, [H, T] packed).
+RP_HD long long lse_index(const Plan& p, const SeqRows& s, int b, int h, int i) {
+  return p.packed ? (long long)h * p.T + s.row0 + i : ((long long)b * p.H + h) * p.N + i;
+}
+// Elements between consecutive rows of one (b, h).
+RP_HD int act_pitch(const Plan& p) { return p.packed ? p.H * 64 : 64; }
+// Coordinates (c1, c2) of row `row` of (b, h) for a TMA map made by
+// make_rows_map: dense maps are {64, N, B H}, packed maps {64, H, T}.
+RP_HD void tma_rows(const Plan& p, const SeqRows& s, int bh, int h, int row, int& c1, int& c2) {
+  if (p.packed) { c1 = h; c2 = s.row0 + row; }
+  else { c1 = row; c2 = bh; }
+}
 
 // Reachable expanded columns of query group g (key_side = 0) or key group g
 // (key_side = 1): a query i reaches delta in [-i, N-1-i], a key j reaches

@@ -59,9 +59,9 @@ cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s, c
 cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream_t s);
 cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t s);
 
-// [BH, N, 64] 16-bit tensor viewed as 3-D for TMA: 128-row boxes, 128-byte
-// swizzle, rows past N read as zero.
-bool make_rows_map(CUtensorMap* m, const void* base, int BH, int N, bool bf16);
+// A 16-bit activation tensor ([B, H, N, 64] dense or [T, H, 64] packed) viewed
+// as 3-D for TMA with 128-row boxes; coordinates from tma_rows (common.cuh).
+bool make_rows_map(CUtensorMap* m, const void* base, const Plan& p, bool bf16);
 cudaError_t launch_forward(const Plan& p, const Tensors& t, cudaStream_t s);
 // Forward with Z^Q recomputed per tile (q.aQ and b terms only).
 cudaError_t launch_forward_recompute(const Plan& p, const Tensors& t, cudaStream_t s);

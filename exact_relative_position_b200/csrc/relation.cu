@@ -80,9 +80,13 @@ __global__ void __launch_bounds__(256) projection_kernel(const Plan p, const int
   if (c0 >= gi.W) return;
   const int r0 = g * kTile;
   const uint32_t sX = smem_u32(smem), sA = sX + 128 * 128;
-  const T* Xh = X + (size_t)bh * p.N * 64;
+  // this sequence's rows of X (dense [B, H, N, 64] or packed [T, H, 64]); rows
+  // past the sequence are zero-filled, so their projections are zero
+  const int b = bh / p.H;
+  const SeqRows sr = seq_rows(p, b);
+  const T* Xh = X + (size_t)act_row(p, sr, b, h, 0) * 64;
   const T* Ah = A + (size_t)h * a_hs + (size_t)(gi.e0 + c0) * 64;
-  load_tile_async<128, 256>(sX, Xh, r0, p.N, tid);
+  load_tile_async<128, 256>(sX, Xh, r0, sr.len, tid, act_pitch(p));
   load_tile_async<64, 256>(sA, Ah, 0, gi.W - c0, tid);
   cp_async_commit();
   cp_async_wait<0>();
@@ -180,10 +184,11 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
   extern __shared__ __align__(16) uint8_t rg_smem[];
   constexpr uint32_t kSB = rg::stage_bytes<T>();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = blockIdx.x, bh = blockIdx.y, h = bh % p.H;
+  const int g = blockIdx.x, bh = blockIdx.y, h = bh % p.H, b = bh / p.H;
   const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
   const int r0 = g * kTile;
-  const int nrows = imin(kTile, p.N - r0);
+  const SeqRows sr = seq_rows(p, b);
+  const int nrows = imin(kTile, sr.len - r0);   // rows of this sequence in the group (may be <= 0)
   const float* Zg = dZ + (size_t)bh * z_head + gi.base;
   const T* Ah = A + (size_t)h * a_hs + (size_t)gi.e0 * 64;
   const int nk = (gi.W + rg::kKC - 1) / rg::kKC;
@@ -242,16 +247,17 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
     }
   }
   cp_async_wait<0>();
-  const size_t off = (size_t)bh * p.N * 64;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
     const int rr = rb + g8 + 8 * hf;
     if (rr >= nrows) continue;
-    const size_t ro = off + (size_t)(r0 + rr) * 64;
+    // the fp32 accumulator keeps the workspace's dense layout; the output is the caller's
+    const size_t ai = ((size_t)bh * p.N + r0 + rr) * 64;
+    const size_t ro = (size_t)act_row(p, sr, b, h, r0 + rr) * 64;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
       const int c = nt * 8 + 2 * tq;
-      const float2 base = *reinterpret_cast<const float2*>(acc_in + ro + c);
+      const float2 base = *reinterpret_cast<const float2*>(acc_in + ai + c);
       *reinterpret_cast<uint32_t*>(out + ro + c) = DT<T>::pack(base.x + acc[nt][2 * hf], base.y + acc[nt][2 * hf + 1]);
     }
   }
@@ -305,24 +311,26 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
       g = (int)(it - (long long)bh * p.nT);
     }
   };
-  auto useful = [&](int g) {
+  // rows of group g that belong to the sequence of (b, h) (all of them in the dense layout)
+  auto item_rows = [&](int bh, int g) { return iclamp(seq_rows(p, bh / p.H).len - g * kTile, 0, kTile); };
+  auto useful = [&](int bh, int g) {
     const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
-    return !(c0 + tp::kEB <= gi.e0 || c0 >= gi.e0 + gi.W);
+    return !(c0 + tp::kEB <= gi.e0 || c0 >= gi.e0 + gi.W) && item_rows(bh, g) > 0;
   };
   // number of chunks of this split (block-uniform)
   int nchunks = 0;
   for (long long it = it0; it < it1; ++it) {
     int bh, g;
     item(it, bh, g);
-    if (useful(g)) nchunks += (imin(kTile, p.N - g * kTile) + tp::kRC - 1) / tp::kRC;
+    if (useful(bh, g)) nchunks += (item_rows(bh, g) + tp::kRC - 1) / tp::kRC;
   }
-  // load cursor: skips items that store none of the block's columns
+  // load cursor: skips items that store none of the block's columns or no rows
   ItemCursor cur{it0, 0};
   auto skip = [&]() {
     while (cur.it < it1) {
       int bh, g;
       item(cur.it, bh, g);
-      if (useful(g)) break;
+      if (useful(bh, g)) break;
       ++cur.it;
     }
   };
@@ -332,9 +340,11 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
     int bh, g;
     item(cur.it, bh, g);
     const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
-    const int r0 = g * kTile, nrows = imin(kTile, p.N - r0);
+    const int r0 = g * kTile, nrows = item_rows(bh, g);
     const float* Zg = dZ + (size_t)bh * z_head + gi.base;
-    const T* Xg = X + ((size_t)bh * p.N + r0) * 64;
+    const int b = bh / p.H;
+    const T* Xg = X + (size_t)act_row(p, seq_rows(p, b), b, bh - b * p.H, r0) * 64;
+    const int xpitch = act_pitch(p);
     const uint32_t zs = sbase + (uint32_t)(q % tp::kStages) * kSB;
     const uint32_t xs = zs + (uint32_t)tp::kRC * tp::kZP * 4u;
     // dZ rows rc .. rc + 31, expanded columns c0 .. c0 + 255 (local column lc = c - e0)
@@ -365,7 +375,7 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
       const int r = tid >> 3, pc = tid & 7;
       const bool ok = cur.rc + r < nrows;
       cp_async16(xs + (uint32_t)(r * tp::kXP + 8 * pc) * (uint32_t)sizeof(T),
-                 ok ? Xg + (size_t)(cur.rc + r) * 64 + 8 * pc : Xg, ok ? 16 : 0);
+                 ok ? Xg + (size_t)(cur.rc + r) * xpitch + 8 * pc : Xg, ok ? 16 : 0);
     }
     cur.rc += tp::kRC;
     if (cur.rc >= nrows) {

@@ -29,17 +29,18 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// Stage rows [r0, r0 + ROWS) of a [*, 64] 16-bit matrix (row pitch 64
+// Stage rows [r0, r0 + ROWS) of a [*, 64] 16-bit matrix (row pitch `pitch`
 // elements) into a swizzled tile; rows >= nrows are zero-filled.
 template <int ROWS, int NTHREADS, typename T>
-__device__ __forceinline__ void load_tile_async(uint32_t sbase, const T* g, int r0, int nrows, int tid) {
+__device__ __forceinline__ void load_tile_async(uint32_t sbase, const T* g, int r0, int nrows, int tid,
+                                                int pitch = 64) {
 #pragma unroll
   for (int it = 0; it < ROWS * 8 / NTHREADS; ++it) {
     const int idx = it * NTHREADS + tid;
     const int r = idx >> 3, c = idx & 7;
     const int gr = r0 + r;
     const bool ok = gr < nrows;
-    const T* src = g + (size_t)(ok ? gr : 0) * 64 + c * 8;
+    const T* src = g + (size_t)(ok ? gr : 0) * pitch + c * 8;
     cp_async16(sbase + swz(r, c), src, ok ? 16 : 0);
   }
 }

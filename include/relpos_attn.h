@@ -136,6 +136,21 @@ typedef struct {
    * the aq and b terms; with ak != NULL it returns UNSUPPORTED.  The backward
    * of a RECOMPUTE forward rebuilds Z^Q in its own part of the workspace. */
   int32_t projection;
+  /* Packed variable-length batch (the pages benchmark padded batches; this is
+   * the layout of FlashAttention's variable-length interface).  NULL: the
+   * dense [B, H, N, d] layout above.  Otherwise cu_seqlens is device int32
+   * [B + 1], non-decreasing from 0: sequence b owns tokens cu_seqlens[b] ..
+   * cu_seqlens[b + 1] - 1, at most N of them (N is the longest sequence and
+   * also sets the identity map's 2N - 1 table rows); q, k, v, o (and dout,
+   * dq, dk, dv) are token-major [total_tokens, H, d] and lse is
+   * [H, total_tokens]; each sequence attends only to its own keys, and no
+   * work is spent on the rows a padded batch would add.  KEY_PADDING must not
+   * be set (INVALID_ARG), total_tokens >= 1.  The kernels clamp offsets into
+   * [0, total_tokens] and lengths into [0, N], so no store leaves the
+   * tensors whatever cu_seqlens holds (inconsistent offsets give meaningless
+   * outputs).  The workspace keeps a dense [B, H, N] layout. */
+  const int32_t* cu_seqlens;
+  int32_t total_tokens;
 } relpos_fwd_args;
 
 typedef enum { RELPOS_PROJECTION_RETAINED = 0, RELPOS_PROJECTION_RECOMPUTE = 1 } relpos_projection_mode;

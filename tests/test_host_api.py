@@ -210,3 +210,21 @@ def test_recompute_projection_forward_workspace_is_linear(lib):
     a = _args()
     a.projection = 2
     assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == -1
+
+
+def test_packed_batch_argument_checks(lib):
+    """A packed batch (cu_seqlens) needs total_tokens >= 1 and excludes the key
+    padding flag (the sequence lengths already mask the keys); its workspace
+    is the dense one of B sequences of N tokens."""
+    f, b = ctypes.c_size_t(), ctypes.c_size_t()
+    a = _args(B=3, N=517)
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == 0
+    dense = (f.value, b.value)
+    a.cu_seqlens, a.total_tokens = 1 << 20, 846
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == 0
+    assert (f.value, b.value) == dense
+    a.total_tokens = 0
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == -1
+    a = _args(B=3, N=517, mask=2)
+    a.cu_seqlens, a.total_tokens = 1 << 20, 846
+    assert lib.relpos_workspace_size(ctypes.byref(a), ctypes.byref(f), ctypes.byref(b)) == -1
