@@ -332,6 +332,9 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--projection", default="retained", choices=["retained", "recompute"],
+                    help="where the forward takes q.aQ from: the stored projection (default) or recomputed in "
+                         "every tile (linear forward memory; q.aQ and bias terms only)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="attention dropout rate for a measurement of its cost (default 0: none)")
     ap.add_argument("--sweep", action="store_true",
@@ -382,10 +385,11 @@ def main():
              None if aq is None else torch.empty(aq.shape, device=dev, dtype=torch.float32),
              None if ak is None else torch.empty(ak.shape, device=dev, dtype=torch.float32),
              None if b is None else torch.empty(b.shape, device=dev, dtype=torch.float32))
-    fws, bws = rp.workspace_size(q, aq, ak, b, w.tau, m, causal=w.causal, key_len=kl, out_f32=out_f32)
+    fws, bws = rp.workspace_size(q, aq, ak, b, w.tau, m, causal=w.causal, key_len=kl, out_f32=out_f32,
+                                 projection=args.projection)
     ws = torch.empty(max(fws, bws), device=dev, dtype=torch.uint8)
     flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)   # 256 MiB > 126 MB L2
-    kw = dict(tau=w.tau, map=m, causal=w.causal, key_len=kl)
+    kw = dict(tau=w.tau, map=m, causal=w.causal, key_len=kl, projection=args.projection)
 
     dkw = dict(dropout_p=args.dropout, dropout_seed=0x5EED, dropout_offset=0)
 
@@ -538,7 +542,8 @@ def main():
             "dtype": "fp16" if w.dtype == torch.float16 else "bf16", "data": "synthetic",
             "config": {"workload": args.workload, **{k_: v_ for k_, v_ in w.describe().items() if k_ != "workload"},
                        "R_exp": R_exp, "l2": "flushed (256 MiB write) before every step",
-                       "dropout": args.dropout,
+                       "dropout": args.dropout, "projection": args.projection,
+                       "workspace_bytes": {"fwd": int(fws), "bwd": int(bws)},
                        "parallelism": f"replicas x{world}"},
             "passes": {
                 "fwd_ms": t_fwd / args.steps, "bwd_ms": t_bwd / args.steps,

@@ -479,10 +479,6 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   const size_t BH = (size_t)a->B * a->H;
   cudaError_t e;
   if (a->aq || a->b) {
-    t.zq_sat = reinterpret_cast<float*>(ws + L.zqsat);
-    if ((e = run_phase(PH_PROJ, s, [&] { return launch_saturated_rows(p, t, s); })) != cudaSuccess) return cuda_fail(e);
-  }
-  if (a->aq || a->b) {
     t.dzq = reinterpret_cast<float*>(ws + L.dzq);
     e = cudaMemsetAsync(t.dzq, 0, sizeof(float) * BH * p.zq_head, s);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -497,6 +493,11 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   if (a->b) t.db_part = reinterpret_cast<float*>(ws + L.dbp);
   t.nsplit_q = L.nsq; t.nsplit_k = L.nsk; t.nsplit_b = L.nsb;
   if ((e = run_phase(PH_PREP, s, [&] { return launch_bwd_prep(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  if (a->aq || a->b) {
+    // the saturated row constants fold in LSE log2e, so they follow the prep
+    t.zq_sat = reinterpret_cast<float*>(ws + L.zqsat);
+    if ((e = run_phase(PH_PROJ, s, [&] { return launch_saturated_rows(p, t, s); })) != cudaSuccess) return cuda_fail(e);
+  }
   const bool terms = a->aq || a->ak || a->b;
   if (terms) {
     e = run_phase(PH_FOLD, s, [&] { return launch_fold_ranges(p, t.phi_exp, L.R, t.fold_lo, t.fold_hi, s); });

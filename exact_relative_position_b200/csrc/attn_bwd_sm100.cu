@@ -131,7 +131,10 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
   auto bar = [&](int slot) { return sb + kOffBar + 8u * (uint32_t)slot; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
+  // causal: query tiles in descending order, the longest rows first (the
+  // K-parallel pass already starts with its longest key tiles)
+  const int qt = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, q0 = qt * kT;
   const int npad = p.nT * kT;
   const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
@@ -294,7 +297,8 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     const size_t prow = (size_t)bh * npad + q0 + r;
     const float lse2 = t.lse2[prow];
     const float dval = t.dsum[prow];
-    // saturated-offset row constants tau log2e (Z^Q[i, sat] + b_sat), zero past N
+    // saturated-offset row constants tau log2e (Z^Q[i, sat] + b_sat) - LSE_i log2e
+    // (-inf for rows without a probability)
     const float crow_lo = (AQ || BIAS) ? t.zq_sat[(size_t)bh * 2 * npad + q0 + r] : 0.f;
     const float crow_hi = (AQ || BIAS) ? t.zq_sat[(size_t)bh * 2 * npad + npad + q0 + r] : 0.f;
     // projection group of this query tile; rows past N use row 0 (in bounds)
@@ -336,7 +340,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       mbar_arrive(bar(kBarSFree));   // S(t + 1) may now be written
       // P = 2^(S tau log2e + relation terms - LSE log2e)
       if (is_const) {
-        const float off = (cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi) - lse2;
+        const float off = (AQ || BIAS) ? (cls == RELPOS_TILE_CONST_LO ? crow_lo : crow_hi) : -lse2;
         // paired fp32 arithmetic: one instruction per two scores
         const float2 sc2 = make_float2(sc, sc), off2 = make_float2(off, off);
         if (AK) {
@@ -802,12 +806,17 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         const float2 sc2 = make_float2(sc, sc), rk2 = make_float2(rowk, rowk);
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
-          float2 w0 = fadd2(rk2, make_float2(-l4.x, -l4.y)), w1 = fadd2(rk2, make_float2(-l4.z, -l4.w));
+          // per query: the staged saturated column already holds its relation terms
+          // minus LSE log2e; without them it is -LSE log2e
+          float2 w0, w1;
           if (AQ || BIAS) {
             const float4 c4 = *reinterpret_cast<const float4*>(cvq + c);
-            w0 = fadd2(w0, make_float2(c4.x, c4.y));
-            w1 = fadd2(w1, make_float2(c4.z, c4.w));
+            w0 = fadd2(rk2, make_float2(c4.x, c4.y));
+            w1 = fadd2(rk2, make_float2(c4.z, c4.w));
+          } else {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
+            w0 = fadd2(rk2, make_float2(-l4.x, -l4.y));
+            w1 = fadd2(rk2, make_float2(-l4.z, -l4.w));
           }
           const float2 z0 = ffma2(make_float2(x[c], x[c + 1]), sc2, w0);
           const float2 z1 = ffma2(make_float2(x[c + 2], x[c + 3]), sc2, w1);

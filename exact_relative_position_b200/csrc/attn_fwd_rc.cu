@@ -130,7 +130,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int slot) { return sb + kOffBar + 8u * (uint32_t)slot; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
+  // causal: query tiles in descending order, the longest rows first
+  const int qt = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, i0 = qt * kT;
   const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
   // keys j >= nkv are masked: the sequence length (packed), or the clamped key length

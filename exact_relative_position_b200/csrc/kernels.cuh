@@ -24,7 +24,7 @@ struct Tensors {
   const void* dout;
   float* dsum;                   // D_i = sum_c dO_ic O_ic, [B*H][nT*128] (0 past N)
   float* lse2;                   // LSE_i log2 e, [B*H][nT*128] (+inf past N and for rows with every key masked)
-  float* zq_sat;                 // [B*H][2][nT*128]: tau log2e (Z^Q[i, sat] + b_sat) for sat = 0, R_exp-1
+  float* zq_sat;                 // [B*H][2][nT*128]: tau log2e (Z^Q[i, sat] + b_sat) - LSE_i log2e, sat = 0, R_exp-1
   float *dzq, *dzk;              // offset-sharded relation gradients (same layout as zq/zk)
   void *dq, *dk, *dv;
   float *dq_acc, *dk_acc;        // fp32 [B,H,N,64] before the relation-GEMM epilogue (or null)

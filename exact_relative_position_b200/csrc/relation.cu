@@ -134,11 +134,12 @@ __global__ void saturated_columns_kernel(const Plan p, const float* __restrict__
   out[(bh * 2 + 1) * npad + j] = hi;
 }
 
-// out[bh][0][i] = tau log2e (Z^Q[i, 0] + b_exp[0]), out[bh][1][i] = the same at
-// R_exp - 1 (each term only when present; zero for i >= N): the row constants
-// of saturated tiles for the backward passes.
+// out[bh][0][i] = tau log2e (Z^Q[i, 0] + b_exp[0]) - LSE_i log2e, out[bh][1][i] =
+// the same at R_exp - 1 (each term only when present; -inf where lse2 is +inf,
+// i.e. past the sequence or for a row without a kept key): the row constants of
+// saturated tiles for the backward passes, with the LSE folded in.
 __global__ void saturated_rows_kernel(const Plan p, const float* __restrict__ zq, const float* __restrict__ b_exp,
-                                      float* __restrict__ out, const float scale) {
+                                      const float* __restrict__ lse2, float* __restrict__ out, const float scale) {
   const int npad = p.nT * kTile;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)p.B * p.H * npad) return;
@@ -158,8 +159,9 @@ __global__ void saturated_rows_kernel(const Plan p, const float* __restrict__ zq
       hi += b_exp[(size_t)h * p.Rexp + p.Rexp - 1];
     }
   }
-  out[(bh * 2 + 0) * npad + i] = lo * scale;
-  out[(bh * 2 + 1) * npad + i] = hi * scale;
+  const float l2 = lse2[bh * npad + i];
+  out[(bh * 2 + 0) * npad + i] = lo * scale - l2;
+  out[(bh * 2 + 1) * npad + i] = hi * scale - l2;
 }
 
 // ------------------------------------------------------------------ relgrad rows
@@ -601,7 +603,7 @@ cudaError_t launch_saturated_columns(const Plan& p, const Tensors& t, cudaStream
 cudaError_t launch_saturated_rows(const Plan& p, const Tensors& t, cudaStream_t s) {
   const long long n = (long long)p.B * p.H * p.nT * kTile;
   {
-    saturated_rows_kernel<<<nblk(n, 256), 256, 0, s>>>(p, t.aq_exp ? t.zq : nullptr, t.b_exp, t.zq_sat,
+    saturated_rows_kernel<<<nblk(n, 256), 256, 0, s>>>(p, t.aq_exp ? t.zq : nullptr, t.b_exp, t.lse2, t.zq_sat,
                                                        p.tau * kLog2e);
     note_launch(1);
   }

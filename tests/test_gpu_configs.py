@@ -37,18 +37,24 @@ def _table(t, h):
     return t[h] if t.ndim == 3 else t
 
 
+def _report(name, errs):
+    print(f"{name}: " + " ".join(f"{k}={v:.2g}" for k, v in errs.items()))
+
+
 def test_config_shaw_clip16_n256_full():
     w = make_workload("shaw_clip16_n256")
     got, want = run_library(w), run_oracle(w)
-    check_forward(got, want, w.name)
-    check_backward(got, want, w.name)
+    o_rel, o_abs = check_forward(got, want, w.name)
+    _report(w.name + " (full)", dict(o_relF=o_rel, o_maxabs=o_abs, lse_maxabs=lse_err(got["lse"], want["lse"]),
+                                     **check_backward(got, want, w.name)))
 
 
 def test_config_deberta_log256_n2048_full():
     w = make_workload("deberta_log256_n2048")
     got, want = run_library(w), run_oracle(w)
-    check_forward(got, want, w.name)
-    check_backward(got, want, w.name)
+    o_rel, o_abs = check_forward(got, want, w.name)
+    _report(w.name + " (full)", dict(o_relF=o_rel, o_maxabs=o_abs, lse_maxabs=lse_err(got["lse"], want["lse"]),
+                                     **check_backward(got, want, w.name)))
 
 
 def _sampled_check(w, got, heads, out_f32_note=""):
@@ -65,12 +71,15 @@ def _sampled_check(w, got, heads, out_f32_note=""):
                                          None if kl is None else kl[bi], rows, cols)
             ctx = f"{w.name} b={bi} h={h}"
             o = got["o"][bi, h][rows]
-            assert relf(o, ref["o"][rows]) <= TOL_O_RELF, ctx
-            assert maxabs(o, ref["o"][rows]) <= TOL_O_MAXABS, ctx
-            assert lse_err(got["lse"][bi, h][rows], ref["lse"][rows]) <= TOL_LSE_MAXABS, ctx
-            assert relf(got["dq"][bi, h][rows], ref["dq"]) <= TOL_GRAD_RELF, ctx + " dq"
-            assert relf(got["dk"][bi, h][cols], ref["dk"]) <= TOL_GRAD_RELF, ctx + " dk"
-            assert relf(got["dv"][bi, h][cols], ref["dv"]) <= TOL_GRAD_RELF, ctx + " dv"
+            errs = dict(o_relF=relf(o, ref["o"][rows]), o_maxabs=maxabs(o, ref["o"][rows]),
+                        lse_maxabs=lse_err(got["lse"][bi, h][rows], ref["lse"][rows]),
+                        dq=relf(got["dq"][bi, h][rows], ref["dq"]), dk=relf(got["dk"][bi, h][cols], ref["dk"]),
+                        dv=relf(got["dv"][bi, h][cols], ref["dv"]))
+            _report(ctx + " (sampled rows)", errs)
+            assert errs["o_relF"] <= TOL_O_RELF and errs["o_maxabs"] <= TOL_O_MAXABS, ctx
+            assert errs["lse_maxabs"] <= TOL_LSE_MAXABS, ctx
+            for n in ("dq", "dk", "dv"):
+                assert errs[n] <= TOL_GRAD_RELF, ctx + " " + n
 
 
 def _table_grads_full(w, heads):
