@@ -246,11 +246,14 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   p->nT = (N + kTile - 1) / kTile;
   p->grouped = p->Rexp > N + kTile - 1;
   p->causal = (a->mask & RELPOS_MASK_CAUSAL) != 0;
+  // causal: the forward and Q-parallel grids take query tiles (pairs) longest first
+  p->qrev = p->causal ? p->nT - 1 : 0;
+  p->qrev_pair = p->causal ? (N + 2 * kTile - 1) / (2 * kTile) - 1 : 0;
   p->padding = (a->mask & RELPOS_MASK_KEY_PADDING) != 0;
   p->tau = a->tau;
   if (!(a->dropout_p >= 0.f && a->dropout_p < 1.f)) return RELPOS_ERR_INVALID_ARG;
   p->dropout = a->dropout_p > 0.f;
-  p->drop_thresh = (uint32_t)ceil((double)a->dropout_p * 16777216.0);
+  p->drop_thresh = (uint32_t)ceil((double)a->dropout_p * 65536.0);   // 16-bit uniforms
   p->drop_scale = p->dropout ? 1.f / (1.f - a->dropout_p) : 1.f;
   p->seed_lo = (uint32_t)(a->dropout_seed & 0xFFFFFFFFull);
   p->seed_hi = (uint32_t)(a->dropout_seed >> 32);

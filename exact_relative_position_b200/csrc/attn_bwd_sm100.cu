@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // causal: query tiles in descending order, the longest rows first (the
   // K-parallel pass already starts with its longest key tiles)
-  const int qt = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int qt = abs(p.qrev - (int)blockIdx.x);
   const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, q0 = qt * kT;
   const int npad = p.nT * kT;

@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   // causal: query tile pairs in descending order, the longest rows (most key
   // tiles) first, so that the last wave holds the shortest ones
-  const int qpair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int qpair = abs(p.qrev_pair - (int)blockIdx.x);
   const int N = p.N, q0 = qpair * (2 * kBQ);
   const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
   // keys j >= nkv are masked: the sequence length (packed), or the clamped key length

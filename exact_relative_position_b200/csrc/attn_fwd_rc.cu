@@ -116,7 +116,9 @@ template <typename T> struct RowStoreRc {
   }
 };
 
-template <typename T, typename OutT, bool AQ, bool BIAS, bool DROP>
+// SAT: a window offset can lie outside [E_lo, E_hi] (every map but the identity
+// map), so saturated cells take the row's saturated values instead of Zt.
+template <typename T, typename OutT, bool AQ, bool BIAS, bool DROP, bool SAT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_rc_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // causal: query tiles in descending order, the longest rows first
-  const int qt = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int qt = abs(p.qrev - (int)blockIdx.x);
   const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
   const int N = p.N, i0 = qt * kT;
   const SeqRows sr = seq_rows(p, b);   // this sequence's rows (the dense layout: all N)
@@ -362,15 +364,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // c - lane + 31 of this lane's row of the skew area
         const int dbase = j0 - i;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int d = dbase + c;
-          float rel = 0.f;
-          if (AQ) {
-            const float zin = sk[lane * kSkPitch + c - lane + 31];
-            rel = d <= p.E_lo ? zq_lo : (d >= p.E_hi ? zq_hi : zin);
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+#pragma unroll
+          for (int c = c0; c < c0 + 32; ++c) {
+            const int d = dbase + c;
+            float rel = 0.f;
+            if (AQ) {
+              const float zin = sk[lane * kSkPitch + c - lane + 31];
+              rel = SAT ? (d <= p.E_lo ? zq_lo : (d >= p.E_hi ? zq_hi : zin)) : zin;
+            }
+            if (BIAS) rel += __ldg(bexp + iclamp(d, p.E_lo, p.E_hi) - p.E_lo);
+            x[c] = (x[c] + rel) * sc;
           }
-          if (BIAS) rel += __ldg(bexp + iclamp(d, p.E_lo, p.E_hi) - p.E_lo);
-          x[c] = (x[c] + rel) * sc;
+          // keep the compiler from hoisting every chunk's loads at once (register pressure)
+          asm volatile("" ::: "memory");
         }
         __syncwarp();   // every lane has read the skew area before the next tile rewrites it
       }
@@ -495,21 +502,21 @@ bool make_table_map(CUtensorMap* m, const void* base, int Hq, int Rexp, long lon
   return r == CUDA_SUCCESS;
 }
 
-template <typename T, typename OutT>
+template <typename T, typename OutT, bool SAT>
 cudaError_t launch_rc_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   using K = void (*)(const Plan, const Tensors, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                      const CUtensorMap);
   const int mask = (t.aq_exp ? 1 : 0) | (t.b_exp ? 2 : 0) | (p.dropout ? 4 : 0);
   K kern = nullptr;
   switch (mask) {
-    case 0: kern = fwd_rc_kernel<T, OutT, false, false, false>; break;
-    case 1: kern = fwd_rc_kernel<T, OutT, true, false, false>; break;
-    case 2: kern = fwd_rc_kernel<T, OutT, false, true, false>; break;
-    case 3: kern = fwd_rc_kernel<T, OutT, true, true, false>; break;
-    case 4: kern = fwd_rc_kernel<T, OutT, false, false, true>; break;
-    case 5: kern = fwd_rc_kernel<T, OutT, true, false, true>; break;
-    case 6: kern = fwd_rc_kernel<T, OutT, false, true, true>; break;
-    default: kern = fwd_rc_kernel<T, OutT, true, true, true>; break;
+    case 0: kern = fwd_rc_kernel<T, OutT, false, false, false, SAT>; break;
+    case 1: kern = fwd_rc_kernel<T, OutT, true, false, false, SAT>; break;
+    case 2: kern = fwd_rc_kernel<T, OutT, false, true, false, SAT>; break;
+    case 3: kern = fwd_rc_kernel<T, OutT, true, true, false, SAT>; break;
+    case 4: kern = fwd_rc_kernel<T, OutT, false, false, true, SAT>; break;
+    case 5: kern = fwd_rc_kernel<T, OutT, true, false, true, SAT>; break;
+    case 6: kern = fwd_rc_kernel<T, OutT, false, true, true, SAT>; break;
+    default: kern = fwd_rc_kernel<T, OutT, true, true, true, SAT>; break;
   }
   CUtensorMap mq, mk, mv, ma;
   const int BH = p.B * p.H;
@@ -528,13 +535,20 @@ cudaError_t launch_rc_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
 
 }  // namespace
 
+template <bool SAT>
+cudaError_t launch_rc_sat(const Plan& p, const Tensors& t, cudaStream_t s) {
+  if (t.is_bf16) {
+    return t.o_f32 ? launch_rc_typed<__nv_bfloat16, float, SAT>(p, t, s)
+                   : launch_rc_typed<__nv_bfloat16, __nv_bfloat16, SAT>(p, t, s);
+  }
+  return t.o_f32 ? launch_rc_typed<__half, float, SAT>(p, t, s) : launch_rc_typed<__half, __half, SAT>(p, t, s);
+}
+
 cudaError_t launch_forward_recompute(const Plan& p, const Tensors& t, cudaStream_t s) {
   if (t.ak_exp) return cudaErrorInvalidValue;   // the key-side term needs the stored projection
-  if (t.is_bf16) {
-    return t.o_f32 ? launch_rc_typed<__nv_bfloat16, float>(p, t, s)
-                   : launch_rc_typed<__nv_bfloat16, __nv_bfloat16>(p, t, s);
-  }
-  return t.o_f32 ? launch_rc_typed<__half, float>(p, t, s) : launch_rc_typed<__half, __half>(p, t, s);
+  // the identity map's expanded range is every reachable offset: no window cell saturates
+  const bool exact_window = p.E_lo == 1 - p.N && p.E_hi == p.N - 1 && p.Rexp == 2 * p.N - 1;
+  return exact_window ? launch_rc_sat<false>(p, t, s) : launch_rc_sat<true>(p, t, s);
 }
 
 }  // namespace relpos

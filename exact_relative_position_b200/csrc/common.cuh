@@ -115,6 +115,10 @@ struct Plan {
   // its dense per-(batch, head) layout of N rows.
   int packed, T;
   const int* cu;
+  // query-tile order of the forward and Q-parallel grids: tile |qrev - blockIdx.x|
+  // (0 in ascending order; under a causal mask the last tile index, so that the
+  // longest rows go first)
+  int qrev, qrev_pair;
 };
 
 // First token row and length of sequence b.  Packed offsets are clamped so
@@ -282,10 +286,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 // "Parallel random numbers: as easy as 1, 2, 3", SC 2011), restated from its
 // definition: ten rounds of (hi0, lo0) = M0 x0, (hi1, lo1) = M1 x2 (32 x 32 ->
 // 64-bit), x = (hi1 ^ x1 ^ k0, lo1, hi0 ^ x3 ^ k1, lo0), the key bumped by
-// (W0, W1) before every round after the first.  Cell (bh, i, j) uses counter
-// (j >> 1, i >> 1, bh, offset) and key (seed_lo, seed_hi) and takes output word
-// 2 (i & 1) + (j & 1): one generator call serves a 2 x 2 block, i.e. a pair of
-// keys of one query row and a pair of queries of one key row alike.
+// (W0, W1) before every round after the first.  One call serves a block of
+// 2 query rows x 4 keys: counter (j >> 2, i >> 1, bh, offset), key (seed_lo,
+// seed_hi); cell k = 4 (i & 1) + (j & 3) reads the 16-bit half k & 1 (low
+// half first) of output word k >> 1 and is kept when it is >= drop_thresh
+// (= ceil(p 2^16)).
 // ---------------------------------------------------------------------------
 #ifdef __CUDACC__
 __device__ __forceinline__ uint4 philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
@@ -306,59 +311,87 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t x0, uint32_t x1, uint32_
   return make_uint4(x0, x1, x2, x3);
 }
 
-__device__ __forceinline__ uint32_t philox_word(const uint4& w, int idx) {
-  return idx == 0 ? w.x : idx == 1 ? w.y : idx == 2 ? w.z : w.w;
+// Keep bits of the two 16-bit uniforms of word w: bit 0 low half, bit 1 high half.
+__device__ __forceinline__ uint32_t keep2(uint32_t w, uint32_t thresh) {
+  return ((w & 0xFFFFu) >= thresh ? 1u : 0u) | ((w >> 16) >= thresh ? 2u : 0u);
 }
 
-// Keep bits of cells (i, j) [bit 0] and (i, j + 1) [bit 1] of slice bh, j even.
-__device__ __forceinline__ uint32_t keep_key_pair(const Plan& p, int bh, int i, int j) {
-  const uint4 w = philox4x32_10((uint32_t)j >> 1, (uint32_t)i >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
-  const int base = 2 * (i & 1);
-  return ((philox_word(w, base) >> 8) >= p.drop_thresh ? 1u : 0u) |
-         ((philox_word(w, base + 1) >> 8) >= p.drop_thresh ? 2u : 0u);
-}
-
-// Keep bits of cells (i, j) [bit 0] and (i + 1, j) [bit 1] of slice bh, i even.
-__device__ __forceinline__ uint32_t keep_query_pair(const Plan& p, int bh, int i, int j) {
-  const uint4 w = philox4x32_10((uint32_t)j >> 1, (uint32_t)i >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
-  const int jb = j & 1;
-  return ((philox_word(w, jb) >> 8) >= p.drop_thresh ? 1u : 0u) |
-         ((philox_word(w, 2 + jb) >> 8) >= p.drop_thresh ? 2u : 0u);
-}
-// Keep bits of 64 consecutive columns c0 .. c0 + 63 (c0 even) for this lane's
-// row, where lane l and lane l ^ 1 own rows 2k and 2k + 1 (row parity = lane
-// parity; the whole warp calls this).  Rows are queries with key columns
-// (row_is_query) or keys with query columns.  Each lane draws every other
-// 2 x 2 block and passes its partner the two words of the partner's row, so a
-// lane makes 16 generator calls for its 64 cells.  Bit c of km[c >> 5] keeps
-// column c0 + c.
+// Keep bits of 64 consecutive columns c0 .. c0 + 63 (c0 a multiple of 4) of
+// this lane's row; bit c of km[c >> 5] keeps column c0 + c.  The whole warp
+// calls this.
+//  row_is_query: rows are queries i (lane parity = i & 1), columns keys.  A
+//    block is the 2 rows of a lane pair x 4 columns; each lane draws every
+//    other block and hands its partner the partner's 4 bits of each (one
+//    shuffle), so a lane makes 8 generator calls for its 64 cells.
+//  otherwise: rows are keys j (lane & 3 = j & 3), columns queries.  A block is
+//    2 columns x the 4 keys of a lane quad; each lane of the quad draws every
+//    fourth block and hands each other lane its 2 bits of each (three
+//    shuffles), again 8 generator calls per lane.
 __device__ __forceinline__ void keep_mask64(const Plan& p, int bh, int row, int c0, bool row_is_query,
                                             uint32_t (&km)[2]) {
-  const int par = row & 1;
   km[0] = km[1] = 0u;
+  const uint32_t th = p.drop_thresh;
+  if (row_is_query) {
+    const int par = row & 1;
+    uint32_t give = 0u;                          // the partner's 4 bits of each block this lane draws
 #pragma unroll
-  for (int w2 = 0; w2 < 16; ++w2) {
-    const int wm = 2 * w2 + par;              // block this lane draws: columns c0 + 2 wm, + 1
-    const uint32_t col = (uint32_t)(c0 + 2 * wm);
-    const uint4 r = row_is_query
-                        ? philox4x32_10(col >> 1, (uint32_t)row >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi)
-                        : philox4x32_10((uint32_t)row >> 1, col >> 1, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
-    // block words: x (i even, j even), y (i even, j odd), z (i odd, j even), w (i odd, j odd);
-    // a row's two cells of the block, in column order, and the partner row's
-    uint32_t m0, m1, o0, o1;
-    if (row_is_query) {        // row = i, columns j
-      m0 = par ? r.z : r.x; m1 = par ? r.w : r.y;
-      o0 = par ? r.x : r.z; o1 = par ? r.y : r.w;
-    } else {                   // row = j, columns i
-      m0 = par ? r.y : r.x; m1 = par ? r.w : r.z;
-      o0 = par ? r.x : r.y; o1 = par ? r.z : r.w;
+    for (int t = 0; t < 8; ++t) {
+      const int blk = 2 * t + par;              // block: columns c0 + 4 blk .. + 3
+      const uint4 r = philox4x32_10((uint32_t)(c0 + 4 * blk) >> 2, (uint32_t)row >> 1, (uint32_t)bh, p.drop_offset,
+                                    p.seed_lo, p.seed_hi);
+      // cells of row parity 0 are words x, y; of parity 1 words z, w
+      const uint32_t even = keep2(r.x, th) | (keep2(r.y, th) << 2);
+      const uint32_t odd = keep2(r.z, th) | (keep2(r.w, th) << 2);
+      km[blk >> 3] |= (par ? odd : even) << (4 * (blk & 7));
+      give |= (par ? even : odd) << (4 * t);
     }
-    const uint32_t g0 = __shfl_xor_sync(0xFFFFFFFFu, o0, 1), g1 = __shfl_xor_sync(0xFFFFFFFFu, o1, 1);
-    const int wp = 2 * w2 + (par ^ 1);         // block the partner drew for this row
-    const uint32_t bm = ((m0 >> 8) >= p.drop_thresh ? 1u : 0u) | ((m1 >> 8) >= p.drop_thresh ? 2u : 0u);
-    const uint32_t bp = ((g0 >> 8) >= p.drop_thresh ? 1u : 0u) | ((g1 >> 8) >= p.drop_thresh ? 2u : 0u);
-    km[wm >> 4] |= bm << (2 * (wm & 15));
-    km[wp >> 4] |= bp << (2 * (wp & 15));
+    const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, give, 1);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int blk = 2 * t + (par ^ 1);        // the blocks the partner drew
+      km[blk >> 3] |= ((got >> (4 * t)) & 0xFu) << (4 * (blk & 7));
+    }
+  } else {
+    const int q4 = row & 3;                     // this lane's key within its quad
+    uint32_t give[4] = {0u, 0u, 0u, 0u};        // 2 bits per drawn block for each key of the quad
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int blk = 4 * t + q4;               // block: columns c0 + 2 blk, + 1 (queries)
+      const uint4 r = philox4x32_10((uint32_t)row >> 2, (uint32_t)(c0 + 2 * blk) >> 1, (uint32_t)bh, p.drop_offset,
+                                    p.seed_lo, p.seed_hi);
+      // key jj: query parity 0 reads cell jj (word jj >> 1), parity 1 cell 4 + jj (word 2 + (jj >> 1))
+      const uint32_t lo01 = keep2(r.x, th), lo23 = keep2(r.y, th), hi01 = keep2(r.z, th), hi23 = keep2(r.w, th);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const uint32_t q0b = ((jj < 2 ? lo01 : lo23) >> (jj & 1)) & 1u;
+        const uint32_t q1b = ((jj < 2 ? hi01 : hi23) >> (jj & 1)) & 1u;
+        give[jj] |= (q0b | (q1b << 1)) << (2 * t);
+      }
+    }
+    // own bits, then the three partners' bits for this key
+    uint32_t mine = give[0];
+    if (q4 == 1) mine = give[1];
+    if (q4 == 2) mine = give[2];
+    if (q4 == 3) mine = give[3];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int blk = 4 * t + q4;
+      km[blk >> 4] |= ((mine >> (2 * t)) & 3u) << (2 * (blk & 15));
+    }
+#pragma unroll
+    for (int d = 1; d < 4; ++d) {
+      const int dst = q4 ^ d;                   // the partner lane's key; it sends this lane's bits
+      uint32_t send = give[0];
+      if (dst == 1) send = give[1];
+      if (dst == 2) send = give[2];
+      if (dst == 3) send = give[3];
+      const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, d);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int blk = 4 * t + dst;            // a block the partner drew
+        km[blk >> 4] |= ((got >> (2 * t)) & 3u) << (2 * (blk & 15));
+      }
+    }
   }
 }
 #endif

@@ -304,15 +304,21 @@ def philox4x32_10(ctr, key):
 
 
 def dropout_keep(bh, rows, N, p, seed, offset):
-    """Kept cells [len(rows), N] (bool) of slice bh = b * H + h."""
+    """Kept cells [len(rows), N] (bool) of slice bh = b * H + h.
+
+    One Philox4x32-10 call serves a block of 2 query rows x 4 keys: counter
+    (j >> 2, i >> 1, bh, offset), key (low, high 32 bits of seed).  Cell
+    k = 4 (i & 1) + (j & 3) of the block reads the 16-bit half k & 1 (low half
+    first) of output word k >> 1 as a uniform u in [0, 2^16); the cell is kept
+    when u 2^-16 >= p."""
     i = np.asarray(rows, dtype=np.uint64)[:, None]
     j = np.arange(N, dtype=np.uint64)[None, :]
-    w = philox4x32_10((j >> np.uint64(1), i >> np.uint64(1), np.uint64(bh), np.uint64(offset & 0xFFFFFFFF)),
+    w = philox4x32_10((j >> np.uint64(2), i >> np.uint64(1), np.uint64(bh), np.uint64(offset & 0xFFFFFFFF)),
                       (np.uint64(seed & 0xFFFFFFFF), np.uint64((seed >> 32) & 0xFFFFFFFF)))
-    sel = (i & np.uint64(1)) * np.uint64(2) + (j & np.uint64(1))
-    word = np.choose(sel.astype(np.int64) + np.zeros(w[0].shape, dtype=np.int64), w)
-    u = (word >> np.uint64(8)).astype(np.float64) * 2.0 ** -24
-    return u >= p
+    k = (i & np.uint64(1)) * np.uint64(4) + (j & np.uint64(3))
+    word = np.choose((k >> np.uint64(1)).astype(np.int64) + np.zeros(w[0].shape, dtype=np.int64), w)
+    u16 = (word >> (np.uint64(16) * (k & np.uint64(1)))) & np.uint64(0xFFFF)
+    return u16.astype(np.float64) * 2.0 ** -16 >= p
 
 
 def head_scores(q, k, aq, ak, bvec, tau, phi, allowed):

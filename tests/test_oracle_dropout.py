@@ -44,6 +44,22 @@ def test_keep_rate(p):
     assert abs(keep.mean() - (1 - p)) < 6 * sd
 
 
+def test_block_cells_use_distinct_uniforms():
+    """Each Philox call serves 2 x 4 cells with eight distinct 16-bit uniforms:
+    every pair of cell positions within a block agrees about half the time at
+    p = 0.5 (two cells reading the same half would always agree), and so do
+    cells of neighbouring blocks."""
+    keep = orc.dropout_keep(2, np.arange(512), 512, 0.5, seed=0xDEADBEEF, offset=3)
+    blocks = keep.reshape(256, 2, 128, 4).transpose(0, 2, 1, 3).reshape(-1, 8)   # [block, 4 (i & 1) + (j & 3)]
+    n = blocks.shape[0]
+    for a in range(8):
+        for b in range(a + 1, 8):
+            agree = np.mean(blocks[:, a] == blocks[:, b])
+            assert abs(agree - 0.5) < 6 * 0.5 / np.sqrt(n), (a, b, agree)
+    agree_next = np.mean(keep[:, 3::4][:, :-1] == keep[:, 4::4])   # last key of a block vs first of the next
+    assert abs(agree_next - 0.5) < 6 * 0.5 / np.sqrt(keep[:, 4::4].size)
+
+
 def test_mask_rows_are_independent_of_the_row_subset():
     full = orc.dropout_keep(3, np.arange(40), 40, 0.3, seed=9, offset=4)
     rows = np.array([0, 7, 8, 33])
