@@ -347,6 +347,9 @@ def main():
                          "their replays (the short-N points are launch-bound when called eagerly)")
     ap.add_argument("--ncu", action="store_true",
                     help="one forward + backward only (for an ncu capture of each kernel's first launch)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (e.g. --ncu --batch 4: inputs larger than L2 for a "
+                         "one-kernel ncu capture)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -370,7 +373,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", device_id=dev)
 
-    w = make_workload(args.workload, seed=rank)
+    w = make_workload(args.workload, seed=rank, **({"B": args.batch} if args.batch > 0 else {}))
     m = rp.RelPosMap(w.map_kind, w.clip, w.num_buckets, w.max_distance, w.bidirectional)
     elo, ehi = rp.expanded_bounds(m, w.N)
     R_exp = ehi - elo + 1

@@ -314,7 +314,10 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   };
   L->nsq = pick(148LL / ((long long)nE * L->Hq), items);   // one table-gradient CTA per SM
   L->nsk = L->nsq;
-  L->nsb = pick(592LL / ((long long)((p->Rexp + 255) / 256) * a->H), (long long)a->B * p->nT);
+  // with per-head aQ tables the bias gradient comes out of the aQ table-gradient
+  // pass, on its splits
+  L->nsb = (aq && a->table_per_head) ? L->nsq
+                                     : pick(592LL / ((long long)((p->Rexp + 255) / 256) * a->H), (long long)a->B * p->nT);
   L->daqp = aq ? take(sizeof(float) * (size_t)L->nsq * L->Hq * p->Rexp * 64) : 0;
   L->dakp = ak ? take(sizeof(float) * (size_t)L->nsk * L->Hq * p->Rexp * 64) : 0;
   L->dbp = bb ? take(sizeof(float) * (size_t)L->nsb * a->H * p->Rexp) : 0;

@@ -429,6 +429,17 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
             if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum.x + ssum.y;
             else sat_hi += ssum.x + ssum.y;
           }
+        } else if (j0 + cb - (i - lane) - 31 > p.E_lo && j0 + cb + 63 - (i - lane) < p.E_hi) {
+          // every offset of the warp's 32 rows x 64 keys interior (warp-uniform):
+          // nothing saturated to sum, all entries stored below
+          const float2 nd2 = make_float2(-dval, -dval);
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float2 ds = fmul2(make_float2(x[c], x[c + 1]),
+                                    fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nd2));
+            x[c] = ds.x;
+            x[c + 1] = ds.y;
+          }
         } else {
           // saturated cells summed here; the interior ones are stored below.
           // Kept keys are cc <= ckeep (cc = key - j0); low-saturated cc <= clo, high cc >= chi.
@@ -915,6 +926,19 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           if (DZK) {
             if (cls == RELPOS_TILE_CONST_LO) sat_lo += ssum.x + ssum.y;
             else sat_hi += ssum.x + ssum.y;
+          }
+        } else if ((j - lane) - (qb + cb + 63) > p.E_lo && (j - lane) + 31 - (qb + cb) < p.E_hi) {
+          // every offset of the warp's 32 keys x 64 queries interior (warp-uniform)
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + c);
+            const float2 ds0 = fmul2(make_float2(x[c], x[c + 1]),
+                                     fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                           make_float2(-d4.x, -d4.y)));
+            const float2 ds1 = fmul2(make_float2(x[c + 2], x[c + 3]),
+                                     fadd2(make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
+                                           make_float2(-d4.z, -d4.w)));
+            x[c] = ds0.x; x[c + 1] = ds0.y; x[c + 2] = ds1.x; x[c + 3] = ds1.y;
           }
         } else {
           // column cc = query qb + cc of this key row: kept for

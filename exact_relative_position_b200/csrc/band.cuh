@@ -78,15 +78,32 @@ template <typename T>
 __device__ __forceinline__ void dz_band_store(const T* stage16, int rbase, int lane, bool key_rows, int row0, int col0,
                                               int cbeg, int nrows, int nkv, int N, int causal, int E_lo, int E_hi,
                                               float* dz_base, long long S, int e0, float tau) {
-#pragma unroll 4
-  for (int rr = 0; rr < 32; ++rr) {
-    const int row = rbase + rr;
-    if (row >= nrows) break;
-    float* dz_row = dz_base + (long long)row * S - e0 - E_lo;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int c = lane + 32 * q;
-      const int col = col0 + cbeg + c;
+  for (int q = 0; q < 2; ++q) {
+    const int c = lane + 32 * q;
+    const int col = col0 + cbeg + c;
+    // the warp's 32 rows x this 32-column chunk: when every cell is kept and
+    // interior (warp-uniform), the entries of a lane form a line of slope
+    // S -+ 1 through dZ, walked with one pointer step per row
+    const int r0 = row0 + rbase, c0 = col0 + cbeg + 32 * q;
+    const int dmin = key_rows ? r0 - (c0 + 31) : c0 - (r0 + 31);
+    const int dmax = key_rows ? r0 + 31 - c0 : c0 + 31 - r0;
+    const int imx = key_rows ? c0 + 31 : r0 + 31, jmx = key_rows ? r0 + 31 : c0 + 31;
+    if (rbase + 31 < nrows && dmin > E_lo && dmax < E_hi && imx < N && jmx < nkv && !(causal && dmax > 0)) {
+      float* ptr = dz_base + (long long)rbase * S + (key_rows ? r0 - col : col - r0) - E_lo - e0;
+      const long long step = key_rows ? S + 1 : S - 1;
+#pragma unroll 8
+      for (int rr = 0; rr < 32; ++rr) {
+        *ptr = tau * DT<T>::to_f(stage16[rr * kDsPitch + c]);
+        ptr += step;
+      }
+      continue;
+    }
+#pragma unroll 4
+    for (int rr = 0; rr < 32; ++rr) {
+      const int row = rbase + rr;
+      if (row >= nrows) break;
+      float* dz_row = dz_base + (long long)row * S - e0 - E_lo;
       const int i = key_rows ? col : row0 + row;
       const int j = key_rows ? row0 + row : col;
       const int d = j - i;

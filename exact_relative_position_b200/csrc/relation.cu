@@ -14,6 +14,8 @@
 //                 pass that sums the splits in order and folds the copy
 //                 columns of a bucket back into that bucket in ascending
 //                 offset order.  No atomics.
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "warp_mma.cuh"
 
@@ -275,7 +277,10 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
 // m16 tiles), so every X fragment feeds two MMAs.  dZ is copied in 16-byte
 // pieces when the item's first column lines up with the block (the common
 // case: e0 = 0 for every group of a map whose groups reach all offsets), else
-// in 4-byte pieces.
+// in 4-byte pieces.  With db_part (per-head tables on the query side, with a
+// bias) the block also sums its dZ columns in fp32 from the same staged chunks,
+// db_part[s][h][c0 + m] = sum over the split's items of column c0 + m of dZ^Q,
+// so the bias gradient needs no pass of its own over dZ^Q.
 namespace tp {
 constexpr int kEB = 256;       // expanded rows per block
 constexpr int kRC = 32;        // positions per chunk
@@ -295,7 +300,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
                                                          const long long z_head, const T* __restrict__ X,
                                                          const int per_head, const int nsplit,
-                                                         float* __restrict__ part) {
+                                                         float* __restrict__ part, float* __restrict__ db_part) {
   extern __shared__ __align__(16) uint8_t tp_smem[];
   constexpr uint32_t kSB = tp::stage_bytes<T>();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -392,6 +397,10 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[mt][i][0] = acc[mt][i][1] = acc[mt][i][2] = acc[mt][i][3] = 0.f;
+  // column sums of dZ for db_part: rows m0 and m0 + 8 of each m16 tile, over this
+  // lane's positions tq and tq + 4 of every k8 step
+  const bool with_db = db_part != nullptr;   // block-uniform
+  float dbs[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
   for (int q = 0; q < tp::kStages - 1; ++q) {
     if (q < nchunks) load(q);
@@ -412,10 +421,16 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         const int m0 = eb + 16 * mt + g8;
-        a[mt][0] = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + m0]);
-        a[mt][1] = to_tf32(Zs[(ks * 8 + tq) * tp::kZP + m0 + 8]);
-        a[mt][2] = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + m0]);
-        a[mt][3] = to_tf32(Zs[(ks * 8 + tq + 4) * tp::kZP + m0 + 8]);
+        const float z0 = Zs[(ks * 8 + tq) * tp::kZP + m0], z1 = Zs[(ks * 8 + tq) * tp::kZP + m0 + 8];
+        const float z2 = Zs[(ks * 8 + tq + 4) * tp::kZP + m0], z3 = Zs[(ks * 8 + tq + 4) * tp::kZP + m0 + 8];
+        a[mt][0] = to_tf32(z0);
+        a[mt][1] = to_tf32(z1);
+        a[mt][2] = to_tf32(z2);
+        a[mt][3] = to_tf32(z3);
+        if (with_db) {
+          dbs[mt][0] += z0 + z2;
+          dbs[mt][1] += z1 + z3;
+        }
       }
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
@@ -427,6 +442,19 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
     }
   }
   cp_async_wait<0>();
+  if (with_db) {
+    // the quad's four lanes hold the four position classes of the same rows
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float v = dbs[mt][hf];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        const int e = c0 + eb + 16 * mt + g8 + 8 * hf;
+        if (tq == 0 && e < p.Rexp) db_part[((size_t)s * p.H + hq) * p.Rexp + e] = v;
+      }
+  }
   float* P = part + ((size_t)s * Hq + hq) * (size_t)p.Rexp * 64;
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt) {
@@ -490,6 +518,25 @@ __global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const floa
 #pragma unroll
     for (int w = 0; w < 8; ++w) sum += red[w][tid];
     part[((size_t)s * p.H + h) * p.Rexp + e] = sum;
+  }
+}
+
+// The fold below for maps whose every table row is one expanded row (R = R_exp:
+// the identity and truncated maps) and with many rows: out[hq][r][c] = the sum
+// over splits s, in order, of part[s][hq][fold_lo[r]][c], as a grid-stride
+// pass over the output (one block per row would mostly schedule blocks).
+__global__ void __launch_bounds__(256) fold_rows_kernel(const float* __restrict__ part, const int nsplit, const int Hq,
+                                                        const int Rexp, const int R, const int C,
+                                                        const int* __restrict__ fold_lo, float* __restrict__ out) {
+  const long long n = (long long)Hq * R * C;
+  for (long long idx = blockIdx.x * 256LL + threadIdx.x; idx < n; idx += (long long)gridDim.x * 256) {
+    const int c = (int)(idx % C);
+    const long long hr = idx / C;
+    const int r = (int)(hr % R), hq = (int)(hr / R);
+    const int e = fold_lo[r];
+    float acc = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) acc += part[(((size_t)sp * Hq + hq) * Rexp + e) * C + c];
+    out[idx] = acc;
   }
 }
 
@@ -614,6 +661,19 @@ cudaError_t launch_projection(const Plan& p, const Tensors& t, cudaStream_t s, c
   return t.is_bf16 ? projection_typed<__nv_bfloat16>(p, t, s, key_stream) : projection_typed<__half>(p, t, s, key_stream);
 }
 
+// Table-gradient fold: the grid-stride pass when every row folds one expanded
+// row and there are many rows, else one block per (row, head).
+static void launch_fold(const float* part, int nsplit, int Hq, int Rexp, int R, int C, const int* fold_lo,
+                        const int* fold_hi, float* out, cudaStream_t s) {
+  if (R == Rexp && (long long)R * Hq >= 4096) {
+    const long long n = (long long)Hq * R * C;
+    const int blocks = (int)std::min<long long>((n + 255) / 256, 148LL * 8);
+    { fold_rows_kernel<<<blocks, 256, 0, s>>>(part, nsplit, Hq, Rexp, R, C, fold_lo, out); note_launch(1); }
+  } else {
+    { fold_kernel<<<dim3(R, Hq), 256, 0, s>>>(part, nsplit, Hq, Rexp, R, C, fold_lo, fold_hi, out); note_launch(1); }
+  }
+}
+
 // side 0: the query side (aQ rows, aQ table, bias); side 1: the key side (aK).
 template <typename T>
 static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cudaStream_t s, cudaStream_t sr) {
@@ -625,26 +685,29 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cuda
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(table_part_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPartSmem);
   if (e != cudaSuccess) return e;
+  // per-head aQ tables with a bias: the aQ table-gradient pass also sums the
+  // bias gradient's columns (its splits are the workspace's bias splits)
+  const bool fuse_db = t.aq_exp && t.b_exp && t.table_per_head && t.nsplit_b == t.nsplit_q;
   if (side == 0 && t.aq_exp) {
     { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
                                                                         t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
     { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
-                                                                           t.table_per_head, t.nsplit_q, t.daq_part); note_launch(1); }
-    { fold_kernel<<<dim3(t.R, Hq), 256, 0, s>>>(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64,
-                                                                     t.fold_lo, t.fold_hi, t.daq); note_launch(1); }
+                                                                           t.table_per_head, t.nsplit_q, t.daq_part,
+                                                                           fuse_db ? t.db_part : nullptr); note_launch(1); }
+    launch_fold(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64, t.fold_lo, t.fold_hi, t.daq, s);
   }
   if (side == 1 && t.ak_exp) {
     { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
                                                                         t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
     { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
-                                                                           t.table_per_head, t.nsplit_k, t.dak_part); note_launch(1); }
-    { fold_kernel<<<dim3(t.R, Hq), 256, 0, s>>>(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64,
-                                                                     t.fold_lo, t.fold_hi, t.dak); note_launch(1); }
+                                                                           t.table_per_head, t.nsplit_k, t.dak_part,
+                                                                           nullptr); note_launch(1); }
+    launch_fold(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64, t.fold_lo, t.fold_hi, t.dak, s);
   }
   if (side == 0 && t.b_exp) {
+    if (!fuse_db)
     { bias_part_kernel<<<dim3((p.Rexp + 255) / 256, p.H, t.nsplit_b), 256, 0, s>>>(p, t.dzq, p.zq_head, t.nsplit_b, t.db_part); note_launch(1); }
-    { fold_kernel<<<dim3(t.R, p.H), 256, 0, s>>>(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1,
-                                                                 t.fold_lo, t.fold_hi, t.db); note_launch(1); }
+    launch_fold(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1, t.fold_lo, t.fold_hi, t.db, s);
   }
   return cudaGetLastError();
 }
