@@ -216,7 +216,7 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
   size_t status, zksat, gq, gk, phi, fold_lo, fold_hi, bexp, aqe, ake, zq, zk, fwd_end;
-  size_t dsum, lse2, zqsat, dzq, dzk, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
+  size_t dsum, lse2, zqsat, dzq, dzk, dzqs, dzks, dqacc, dkacc, daqp, dakp, dbp, bwd_end;
   int R, Hq, expand, nsq, nsk, nsb;
   int recompute;   // projection = RECOMPUTE: Z^Q lives in the backward-only part
 };
@@ -300,8 +300,11 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   L->dsum = take(sizeof(float) * BH * npad);
   L->lse2 = take(sizeof(float) * BH * npad);
   L->zqsat = (aq || bb) ? take(sizeof(float) * BH * 2 * npad) : 0;
-  L->dzq = (aq || bb) ? take(sizeof(float) * BH * p->zq_head) : 0;
-  L->dzk = ak ? take(sizeof(float) * BH * p->zk_head) : 0;
+  // relation gradients: 16-bit interior entries, fp32 saturated-offset sums per row
+  L->dzq = (aq || bb) ? take(2 * BH * p->zq_head) : 0;
+  L->dzk = ak ? take(2 * BH * p->zk_head) : 0;
+  L->dzqs = (aq || bb) ? take(sizeof(float) * BH * npad * 2) : 0;
+  L->dzks = ak ? take(sizeof(float) * BH * npad * 2) : 0;
   L->dqacc = aq ? take(sizeof(float) * BH * N * 64) : 0;
   L->dkacc = ak ? take(sizeof(float) * BH * N * 64) : 0;
   const int nE = (p->Rexp + 255) / 256;   // expanded-row blocks of the table-gradient kernel
@@ -485,13 +488,15 @@ RELPOS_EXPORT int relpos_attn_bwd(const relpos_bwd_args* g, void* workspace, siz
   const size_t BH = (size_t)a->B * a->H;
   cudaError_t e;
   if (a->aq || a->b) {
-    t.dzq = reinterpret_cast<float*>(ws + L.dzq);
-    e = cudaMemsetAsync(t.dzq, 0, sizeof(float) * BH * p.zq_head, s);
+    t.dzq = ws + L.dzq;
+    t.dzq_sat = reinterpret_cast<float*>(ws + L.dzqs);
+    e = cudaMemsetAsync(t.dzq, 0, 2 * BH * p.zq_head, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   if (a->ak) {
-    t.dzk = reinterpret_cast<float*>(ws + L.dzk);
-    e = cudaMemsetAsync(t.dzk, 0, sizeof(float) * BH * p.zk_head, s);
+    t.dzk = ws + L.dzk;
+    t.dzk_sat = reinterpret_cast<float*>(ws + L.dzks);
+    e = cudaMemsetAsync(t.dzk, 0, 2 * BH * p.zk_head, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   if (a->aq) { t.dq_acc = reinterpret_cast<float*>(ws + L.dqacc); t.daq_part = reinterpret_cast<float*>(ws + L.daqp); }

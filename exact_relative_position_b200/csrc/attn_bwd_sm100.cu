@@ -304,8 +304,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
     // projection group of this query tile; rows past N use row 0 (in bounds)
     const GroupInfo gi = p.gq[qt];
     const int rrow = rok ? r : 0;
-    float* dzq_base = DZQ ? t.dzq + (size_t)bh * p.zq_head + gi.base : nullptr;
-    float* dzq_row = DZQ ? dzq_base + (long long)rrow * gi.S - gi.e0 : nullptr;
+    T* dzq_base = DZQ ? static_cast<T*>(t.dzq) + (size_t)bh * p.zq_head + gi.base : nullptr;
     const int nrows_q = imin(kT, N - q0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
     T* stg = reinterpret_cast<T*>(sg + kOffStage + (uint32_t)(warp - 4) * kStageWarpBytes);
@@ -482,7 +481,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
       if (DZQ && !is_const) {
         __syncwarp();
         dz_band_store<T>(stg, (warp & 3) * 32, lane, false, q0, j0, cb, nrows_q, nkv, N,
-                         p.causal, p.E_lo, p.E_hi, dzq_base, gi.S, gi.e0, p.tau);
+                         p.causal, p.E_lo, p.E_hi, dzq_base, gi.S, gi.e0);
       }
       tc_fence_before();
       mbar_arrive(bar(kBarDsReady + (it & 1)));
@@ -496,16 +495,8 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         sat[2 * r + 1] = sat_hi;
       }
       named_bar_sync(1, 256);
-      if (hc == 0 && rok) {
-        sat_lo += sat[2 * r];
-        sat_hi += sat[2 * r + 1];
-        if (p.Rexp == 1) {
-          dzq_row[0] = p.tau * (sat_lo + sat_hi);
-        } else {
-          if (gi.e0 == 0) dzq_row[0] = p.tau * sat_lo;
-          if (p.Rexp - 1 < gi.e0 + gi.W) dzq_row[p.Rexp - 1] = p.tau * sat_hi;
-        }
-      }
+      if (hc == 0 && rok)
+        *reinterpret_cast<float2*>(t.dzq_sat + 2 * prow) = make_float2(sat_lo + sat[2 * r], sat_hi + sat[2 * r + 1]);
     }
     // dQ: half hc stores head-dim columns [32 hc, 32 hc + 32) of its row
     float dq[32];
@@ -776,8 +767,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
     // projection group of this key tile; keys past N use row 0 (in bounds)
     const GroupInfo gk = p.gk[kt];
     const int krow = jok ? r : 0;
-    float* dzk_base = DZK ? t.dzk + (size_t)bh * p.zk_head + gk.base : nullptr;
-    float* dzk_row = DZK ? dzk_base + (long long)krow * gk.S - gk.e0 : nullptr;
+    T* dzk_base = DZK ? static_cast<T*>(t.dzk) + (size_t)bh * p.zk_head + gk.base : nullptr;
     const int nrows_k = imin(kT, N - k0);
     const float* bexp = BIAS ? t.b_exp + (size_t)h * p.Rexp : nullptr;
     T* stg = reinterpret_cast<T*>(sg + kOffStage + (uint32_t)(warp - 4) * kStageWarpBytes);
@@ -988,7 +978,7 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       if (DZK && !is_const) {
         __syncwarp();
         dz_band_store<T>(stg, (warp & 3) * 32, lane, true, k0, qb, cb, nrows_k, nkv, N,
-                         p.causal, p.E_lo, p.E_hi, dzk_base, gk.S, gk.e0, p.tau);
+                         p.causal, p.E_lo, p.E_hi, dzk_base, gk.S, gk.e0);
       }
       tc_fence_before();
       mbar_arrive(bar(kBarDsReady));
@@ -1002,16 +992,9 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         sat[2 * r + 1] = sat_hi;
       }
       named_bar_sync(1, 256);
-      if (hc == 0 && jok) {
-        sat_lo += sat[2 * r];
-        sat_hi += sat[2 * r + 1];
-        if (p.Rexp == 1) {
-          dzk_row[0] = p.tau * (sat_lo + sat_hi);
-        } else {
-          if (gk.e0 == 0) dzk_row[0] = p.tau * sat_lo;
-          if (p.Rexp - 1 < gk.e0 + gk.W) dzk_row[p.Rexp - 1] = p.tau * sat_hi;
-        }
-      }
+      if (hc == 0 && jok)
+        *reinterpret_cast<float2*>(t.dzk_sat + 2 * ((size_t)bh * npad + k0 + r)) =
+            make_float2(sat_lo + sat[2 * r], sat_hi + sat[2 * r + 1]);
     }
     // dV and dK: half hc stores head-dim columns [32 hc, 32 hc + 32) of its key
     float dv[32], dk[32];

@@ -67,7 +67,7 @@ __device__ __forceinline__ void band_terms_k(float* x, int E_lo, int E_hi, int j
 
 // Interior relation-gradient entries of one BAND tile, stored by offset from
 // the warp's 16-bit dS rows (rows = this side's positions, 64 columns = the
-// other side's).  Warp-cooperative and coalesced: the warp walks its 32 rows
+// other side's) as those 16-bit values (the consumers apply tau).  Warp-cooperative and coalesced: the warp walks its 32 rows
 // and its lanes cover the columns, whose offsets are consecutive.  Interior
 // offsets E_lo < d < E_hi have exactly one cell per (row, offset), so every
 // entry has one writer; the two saturated offsets are summed by the caller.
@@ -77,7 +77,7 @@ __device__ __forceinline__ void band_terms_k(float* x, int E_lo, int E_hi, int j
 template <typename T>
 __device__ __forceinline__ void dz_band_store(const T* stage16, int rbase, int lane, bool key_rows, int row0, int col0,
                                               int cbeg, int nrows, int nkv, int N, int causal, int E_lo, int E_hi,
-                                              float* dz_base, long long S, int e0, float tau) {
+                                              T* dz_base, long long S, int e0) {
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int c = lane + 32 * q;
@@ -90,11 +90,11 @@ __device__ __forceinline__ void dz_band_store(const T* stage16, int rbase, int l
     const int dmax = key_rows ? r0 + 31 - c0 : c0 + 31 - r0;
     const int imx = key_rows ? c0 + 31 : r0 + 31, jmx = key_rows ? r0 + 31 : c0 + 31;
     if (rbase + 31 < nrows && dmin > E_lo && dmax < E_hi && imx < N && jmx < nkv && !(causal && dmax > 0)) {
-      float* ptr = dz_base + (long long)rbase * S + (key_rows ? r0 - col : col - r0) - E_lo - e0;
+      T* ptr = dz_base + (long long)rbase * S + (key_rows ? r0 - col : col - r0) - E_lo - e0;
       const long long step = key_rows ? S + 1 : S - 1;
 #pragma unroll 8
       for (int rr = 0; rr < 32; ++rr) {
-        *ptr = tau * DT<T>::to_f(stage16[rr * kDsPitch + c]);
+        *ptr = stage16[rr * kDsPitch + c];
         ptr += step;
       }
       continue;
@@ -103,12 +103,12 @@ __device__ __forceinline__ void dz_band_store(const T* stage16, int rbase, int l
     for (int rr = 0; rr < 32; ++rr) {
       const int row = rbase + rr;
       if (row >= nrows) break;
-      float* dz_row = dz_base + (long long)row * S - e0 - E_lo;
+      T* dz_row = dz_base + (long long)row * S - e0 - E_lo;
       const int i = key_rows ? col : row0 + row;
       const int j = key_rows ? row0 + row : col;
       const int d = j - i;
       const bool kept = i < N && j < nkv && !(causal && j > i) && d > E_lo && d < E_hi;
-      if (kept) dz_row[d] = tau * DT<T>::to_f(stage16[rr * kDsPitch + c]);
+      if (kept) dz_row[d] = stage16[rr * kDsPitch + c];
     }
   }
 }

@@ -27,7 +27,9 @@ constexpr double kGuard = 1e-9;      // exact integer crossings of the log formu
 RP_HD int imin(int a, int b) { return a < b ? a : b; }
 RP_HD int imax(int a, int b) { return a > b ? a : b; }
 RP_HD int iclamp(int x, int lo, int hi) { return imin(imax(x, lo), hi); }
-RP_HD int round_up4(int x) { return (x + 3) & ~3; }
+// Row stride of a projection group: a multiple of 8 elements, so that rows of
+// the fp32 projection and of the 16-bit relation gradient both start on 16 bytes.
+RP_HD int round_up8(int x) { return (x + 7) & ~7; }
 
 // ---------------------------------------------------------------------------
 // Offset maps phi(delta), delta = j - i.
@@ -179,10 +181,10 @@ RP_HD GroupInfo group_info(const Plan& p, int key_side, int g) {
   for (int t = 0; t < g; ++t) {
     int e0, W;
     group_columns(p, key_side, t, &e0, &W);
-    base += (long long)imin(kTile, p.N - t * kTile) * round_up4(W);
+    base += (long long)imin(kTile, p.N - t * kTile) * round_up8(W);
   }
   group_columns(p, key_side, g, &gi.e0, &gi.W);
-  gi.S = round_up4(gi.W);
+  gi.S = round_up8(gi.W);
   gi.pad = 0;
   gi.base = base;
   return gi;

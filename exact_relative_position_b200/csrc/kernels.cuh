@@ -25,7 +25,10 @@ struct Tensors {
   float* dsum;                   // D_i = sum_c dO_ic O_ic, [B*H][nT*128] (0 past N)
   float* lse2;                   // LSE_i log2 e, [B*H][nT*128] (+inf past N and for rows with every key masked)
   float* zq_sat;                 // [B*H][2][nT*128]: tau log2e (Z^Q[i, sat] + b_sat) - LSE_i log2e, sat = 0, R_exp-1
-  float *dzq, *dzk;              // offset-sharded relation gradients (same layout as zq/zk)
+  void *dzq, *dzk;               // offset-sharded relation gradients: the 16-bit dS of each interior
+                                 // offset (tau not applied), same layout as zq/zk, zero elsewhere
+  float *dzq_sat, *dzk_sat;      // [B*H][nT*128][2]: each row's sums of dS over its cells at the low /
+                                 // high saturated offset (tau not applied)
   void *dq, *dk, *dv;
   float *dq_acc, *dk_acc;        // fp32 [B,H,N,64] before the relation-GEMM epilogue (or null)
   float *daq_part, *dak_part;    // [nsplit][Hq][Rexp][64] partial table gradients

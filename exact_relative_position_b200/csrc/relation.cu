@@ -167,24 +167,28 @@ __global__ void saturated_rows_kernel(const Plan p, const float* __restrict__ zq
 }
 
 // ------------------------------------------------------------------ relgrad rows
-// out[rows of group g] = acc_in[rows] + dZ_g[rows, :W] A_exp[e0 .. e0 + W)   (tf32 tensor cores)
+// out[rows of group g] = acc_in[rows] + tau (dS_g[rows, :W] A_exp[e0 .. e0 + W)
+//                        + s_lo A_exp[0] + s_hi A_exp[R_exp - 1])     (16-bit tensor cores)
+// dS_g: the group's stored 16-bit relation gradient (interior offsets; zero at
+// the saturated ones), (s_lo, s_hi): the row's fp32 saturated-offset sums.
 // One CTA per (group, batch x head).  The reduction runs over the group's W
 // stored columns, streamed in chunks of 32 columns through a 3-stage cp.async
-// ring; warp w owns rows 16w .. 16w + 15 and all 64 output columns.
+// ring; warp w owns rows 16w .. 16w + 15 and all 64 output columns
+// (mma m16n8k16, operands by ldmatrix).
 namespace rg {
-constexpr int kKC = 32;        // columns of dZ (rows of the table) per chunk
+constexpr int kKC = 32;        // columns of dS (rows of the table) per chunk
 constexpr int kStages = 3;
-constexpr int kZP = 36;        // floats per row of a dZ chunk [128][32]: conflict-free fragment reads
-constexpr int kAP = 72;        // elements per row of a table chunk [32][64]
+constexpr int kZP = 40;        // elements per row of a dS chunk [128][32] (80 bytes: conflict-free ldmatrix)
+constexpr int kAP = 72;        // elements per row of a table chunk [32][64] (144 bytes)
 template <typename T>
-constexpr uint32_t stage_bytes() { return 128u * kZP * 4u + (uint32_t)(kKC * kAP * sizeof(T)); }
+constexpr uint32_t stage_bytes() { return (uint32_t)(128 * kZP + kKC * kAP) * (uint32_t)sizeof(T); }
 }  // namespace rg
 
 template <typename T>
-__global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
-                                                           const long long z_head, const T* __restrict__ A,
-                                                           const long long a_hs, const float* __restrict__ acc_in,
-                                                           T* __restrict__ out) {
+__global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const int key_side, const T* __restrict__ dZ,
+                                                           const long long z_head, const float* __restrict__ dz_sat,
+                                                           const T* __restrict__ A, const long long a_hs,
+                                                           const float* __restrict__ acc_in, T* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t rg_smem[];
   constexpr uint32_t kSB = rg::stage_bytes<T>();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -193,24 +197,26 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
   const int r0 = g * kTile;
   const SeqRows sr = seq_rows(p, b);
   const int nrows = imin(kTile, sr.len - r0);   // rows of this sequence in the group (may be <= 0)
-  const float* Zg = dZ + (size_t)bh * z_head + gi.base;
-  const T* Ah = A + (size_t)h * a_hs + (size_t)gi.e0 * 64;
+  const T* Zg = dZ + (size_t)bh * z_head + gi.base;
+  const T* Ah0 = A + (size_t)h * a_hs;
+  const T* Ah = Ah0 + (size_t)gi.e0 * 64;
   const int nk = (gi.W + rg::kKC - 1) / rg::kKC;
   const uint32_t sbase = smem_u32(rg_smem);
   auto load = [&](int kc) {
     const uint32_t zs = sbase + (uint32_t)(kc % rg::kStages) * kSB;
-    const uint32_t as = zs + 128u * rg::kZP * 4u;
+    const uint32_t as = zs + 128u * rg::kZP * (uint32_t)sizeof(T);
     const int c0 = kc * rg::kKC;
-    // dZ: 128 rows x 8 pieces of 4 columns; a piece at or past the row stride
-    // S (a multiple of 4) or a row past the group is zero-filled.  Columns in
-    // [W, S) are stored zeros.
+    // dS: 128 rows x 4 pieces of 8 columns (rows start on 16 bytes: S and the
+    // group base are multiples of 8); a piece at or past the row stride S or
+    // a row past the group is zero-filled.  Columns in [W, S) are stored zeros.
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int idx = u * 256 + tid;
-      const int r = idx >> 3, pc = idx & 7;
-      const int col = c0 + 4 * pc;
+      const int r = idx >> 2, pc = idx & 3;
+      const int col = c0 + 8 * pc;
       const bool ok = r < nrows && col < gi.S;
-      cp_async16(zs + (uint32_t)(r * rg::kZP + 4 * pc) * 4u, ok ? Zg + (long long)r * gi.S + col : Zg, ok ? 16 : 0);
+      cp_async16(zs + (uint32_t)(r * rg::kZP + 8 * pc) * (uint32_t)sizeof(T), ok ? Zg + (long long)r * gi.S + col : Zg,
+                 ok ? 16 : 0);
     }
     // table rows e0 + c0 .. + 31 (8 pieces of 8 elements each); rows past W are zero-filled
     const int r = tid >> 3, pc = tid & 7;
@@ -227,34 +233,37 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
     if (s < nk) load(s);
     cp_async_commit();
   }
+  // ldmatrix lane addresses: A (dS rows) and B (table, transposed)
+  const int mi = lane >> 3;
+  const uint32_t a_off = (uint32_t)((rb + (lane & 15)) * rg::kZP + (lane >> 4) * 8) * (uint32_t)sizeof(T);
+  const uint32_t b_off = (uint32_t)(((mi & 1) * 8 + (lane & 7)) * rg::kAP + (mi >> 1) * 8) * (uint32_t)sizeof(T);
   for (int kc = 0; kc < nk; ++kc) {
     cp_async_wait<rg::kStages - 2>();
     __syncthreads();   // chunk kc visible to all; the stage of chunk kc - 1 is free again
     if (kc + rg::kStages - 1 < nk) load(kc + rg::kStages - 1);
     cp_async_commit();
-    const uint8_t* st = rg_smem + (uint32_t)(kc % rg::kStages) * kSB;
-    const float* Zs = reinterpret_cast<const float*>(st);
-    const T* As = reinterpret_cast<const T*>(st + 128u * rg::kZP * 4u);
+    const uint32_t zs = sbase + (uint32_t)(kc % rg::kStages) * kSB;
+    const uint32_t as = zs + 128u * rg::kZP * (uint32_t)sizeof(T);
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t a0 = to_tf32(Zs[(rb + g8) * rg::kZP + ks * 8 + tq]);
-      const uint32_t a1 = to_tf32(Zs[(rb + g8 + 8) * rg::kZP + ks * 8 + tq]);
-      const uint32_t a2 = to_tf32(Zs[(rb + g8) * rg::kZP + ks * 8 + tq + 4]);
-      const uint32_t a3 = to_tf32(Zs[(rb + g8 + 8) * rg::kZP + ks * 8 + tq + 4]);
+    for (int ks = 0; ks < rg::kKC / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(zs + a_off + (uint32_t)(ks * 16) * (uint32_t)sizeof(T), a[0], a[1], a[2], a[3]);
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        // a 16-bit value is exact in tf32
-        const uint32_t b0 = __float_as_uint(DT<T>::to_f(As[(ks * 8 + tq) * rg::kAP + nt * 8 + g8]));
-        const uint32_t b1 = __float_as_uint(DT<T>::to_f(As[(ks * 8 + tq + 4) * rg::kAP + nt * 8 + g8]));
-        mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(as + b_off + (uint32_t)(ks * 16 * rg::kAP + np * 16) * (uint32_t)sizeof(T), b0, b1, b2, b3);
+        MmaOp<T>::run(acc[2 * np], a, b0, b1);
+        MmaOp<T>::run(acc[2 * np + 1], a, b2, b3);
       }
     }
   }
   cp_async_wait<0>();
+  const size_t npad = (size_t)p.nT * kTile;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
     const int rr = rb + g8 + 8 * hf;
     if (rr >= nrows) continue;
+    const float2 sat = *reinterpret_cast<const float2*>(dz_sat + 2 * ((size_t)bh * npad + r0 + rr));
     // the fp32 accumulator keeps the workspace's dense layout; the output is the caller's
     const size_t ai = ((size_t)bh * p.N + r0 + rr) * 64;
     const size_t ro = (size_t)act_row(p, sr, b, h, r0 + rr) * 64;
@@ -262,33 +271,39 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
     for (int nt = 0; nt < 8; ++nt) {
       const int c = nt * 8 + 2 * tq;
       const float2 base = *reinterpret_cast<const float2*>(acc_in + ai + c);
-      *reinterpret_cast<uint32_t*>(out + ro + c) = DT<T>::pack(base.x + acc[nt][2 * hf], base.y + acc[nt][2 * hf + 1]);
+      const float lo0 = DT<T>::to_f(Ah0[c]), lo1 = DT<T>::to_f(Ah0[c + 1]);
+      const float hi0 = DT<T>::to_f(Ah0[(size_t)(p.Rexp - 1) * 64 + c]), hi1 = DT<T>::to_f(Ah0[(size_t)(p.Rexp - 1) * 64 + c + 1]);
+      const float v0 = acc[nt][2 * hf] + sat.x * lo0 + sat.y * hi0;
+      const float v1 = acc[nt][2 * hf + 1] + sat.x * lo1 + sat.y * hi1;
+      *reinterpret_cast<uint32_t*>(out + ro + c) = DT<T>::pack(fmaf(p.tau, v0, base.x), fmaf(p.tau, v1, base.y));
     }
   }
 }
 
 // ------------------------------------------------------------------ table partials
-// part[s][hq][c0 + m][:] = sum over the split's (batch, head, group) items, in
-// order, of dZ_g[rows, c0 + m - e0] X[rows, :]   (tf32 tensor cores)
+// part[s][hq][c0 + m][:] = tau x the sum over the split's (batch, head, group)
+// items, in order, of dS_g[rows, c0 + m - e0] X[rows, :]   (16-bit tensor cores)
+// plus, at the saturated offsets m = 0 and R_exp - 1, tau x the sum of the
+// rows' fp32 saturated-offset sums times X[rows, :].
 // Block (e-block of 256 expanded rows, table, split).  The split's positions
-// are streamed in chunks of 32 rows of (dZ, X) through a 3-stage cp.async
-// ring that runs across item boundaries; items whose group stores none of the
-// block's columns are skipped.  Warp w owns expanded rows 32w .. 32w + 31 (two
-// m16 tiles), so every X fragment feeds two MMAs.  dZ is copied in 16-byte
-// pieces when the item's first column lines up with the block (the common
-// case: e0 = 0 for every group of a map whose groups reach all offsets), else
-// in 4-byte pieces.  With db_part (per-head tables on the query side, with a
-// bias) the block also sums its dZ columns in fp32 from the same staged chunks,
-// db_part[s][h][c0 + m] = sum over the split's items of column c0 + m of dZ^Q,
-// so the bias gradient needs no pass of its own over dZ^Q.
+// are streamed in chunks of 32 rows of (dS, X, saturated sums) through a
+// 3-stage cp.async ring that runs across item boundaries; items whose group
+// stores none of the block's columns are skipped.  Warp w owns expanded rows
+// 32w .. 32w + 31 (two m16 tiles), so every X fragment feeds two MMAs.  dS is
+// copied in 16-byte pieces when the item's first column lines up with the
+// block to 8 elements (every group of a map whose groups reach all offsets),
+// else element by element.  With db_part (per-head tables on the query side,
+// with a bias) the block also sums its dS columns in fp32 from the same staged
+// chunks: db_part[s][h][c0 + m] = tau x (column sums + saturated sums), so the
+// bias gradient needs no pass of its own over dS^Q.
 namespace tp {
 constexpr int kEB = 256;       // expanded rows per block
 constexpr int kRC = 32;        // positions per chunk
 constexpr int kStages = 3;
-constexpr int kZP = 264;       // floats per row of a dZ chunk [32][256]: conflict-free transposed fragment reads
+constexpr int kZP = 264;       // elements per row of a dS chunk [32][256] (528 bytes: conflict-free ldmatrix)
 constexpr int kXP = 72;        // elements per row of an X chunk [32][64]
 template <typename T>
-constexpr uint32_t stage_bytes() { return (uint32_t)kRC * kZP * 4u + (uint32_t)(kRC * kXP * sizeof(T)); }
+constexpr uint32_t stage_bytes() { return (uint32_t)(kRC * kZP + kRC * kXP) * (uint32_t)sizeof(T) + kRC * 8u; }
 }  // namespace tp
 
 struct ItemCursor {
@@ -297,17 +312,20 @@ struct ItemCursor {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int key_side, const float* __restrict__ dZ,
-                                                         const long long z_head, const T* __restrict__ X,
-                                                         const int per_head, const int nsplit,
+__global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int key_side, const T* __restrict__ dZ,
+                                                         const long long z_head, const float* __restrict__ dz_sat,
+                                                         const T* __restrict__ X, const int per_head, const int nsplit,
                                                          float* __restrict__ part, float* __restrict__ db_part) {
   extern __shared__ __align__(16) uint8_t tp_smem[];
   constexpr uint32_t kSB = tp::stage_bytes<T>();
+  constexpr uint32_t kXOff = (uint32_t)tp::kRC * tp::kZP * (uint32_t)sizeof(T);
+  constexpr uint32_t kSOff = kXOff + (uint32_t)tp::kRC * tp::kXP * (uint32_t)sizeof(T);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c0 = blockIdx.x * tp::kEB, hq = blockIdx.y, s = blockIdx.z;
   const int Hq = per_head ? p.H : 1;
   const long long nitems = per_head ? (long long)p.B * p.nT : (long long)p.B * p.H * p.nT;
   const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
+  const size_t npad = (size_t)p.nT * kTile;
   auto item = [&](long long it, int& bh, int& g) {
     if (per_head) {
       const int b = (int)(it / p.nT);
@@ -348,41 +366,49 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
     item(cur.it, bh, g);
     const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
     const int r0 = g * kTile, nrows = item_rows(bh, g);
-    const float* Zg = dZ + (size_t)bh * z_head + gi.base;
+    const T* Zg = dZ + (size_t)bh * z_head + gi.base;
     const int b = bh / p.H;
     const T* Xg = X + (size_t)act_row(p, seq_rows(p, b), b, bh - b * p.H, r0) * 64;
     const int xpitch = act_pitch(p);
     const uint32_t zs = sbase + (uint32_t)(q % tp::kStages) * kSB;
-    const uint32_t xs = zs + (uint32_t)tp::kRC * tp::kZP * 4u;
-    // dZ rows rc .. rc + 31, expanded columns c0 .. c0 + 255 (local column lc = c - e0)
-    if (((c0 - gi.e0) & 3) == 0) {
-      // 16-byte pieces: lc is a multiple of 4 and the row stride S too; the
+    // dS rows rc .. rc + 31, expanded columns c0 .. c0 + 255 (local column lc = c - e0)
+    if (((c0 - gi.e0) & 7) == 0) {
+      // 16-byte pieces: lc is a multiple of 8 and the row stride S too; the
       // columns [W, S) are stored zeros
-#pragma unroll 4
-      for (int u = 0; u < tp::kRC * tp::kEB / 4 / 256; ++u) {
+#pragma unroll
+      for (int u = 0; u < tp::kRC * tp::kEB / 8 / 256; ++u) {
         const int idx = u * 256 + tid;
-        const int r = idx >> 6, c = (idx & 63) * 4;
+        const int r = idx >> 5, c = (idx & 31) * 8;
         const int lc = c0 + c - gi.e0;
         const bool ok = cur.rc + r < nrows && lc >= 0 && lc < gi.S;
-        cp_async16(zs + (uint32_t)(r * tp::kZP + c) * 4u, ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg,
-                   ok ? 16 : 0);
+        cp_async16(zs + (uint32_t)(r * tp::kZP + c) * (uint32_t)sizeof(T),
+                   ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg, ok ? 16 : 0);
       }
     } else {
+      // a window not aligned to 8 elements (ragged N): plain 16-bit copies,
+      // visible to the block after the barrier that makes the stage current
+      T* zp = reinterpret_cast<T*>(tp_smem + (uint32_t)(q % tp::kStages) * kSB);
 #pragma unroll 4
       for (int u = 0; u < tp::kRC * tp::kEB / 256; ++u) {
         const int idx = u * 256 + tid;
         const int r = idx >> 8, c = idx & 255;
         const int lc = c0 + c - gi.e0;
         const bool ok = cur.rc + r < nrows && lc >= 0 && lc < gi.W;
-        cp_async4(zs + (uint32_t)(r * tp::kZP + c) * 4u, ok ? Zg + (long long)(cur.rc + r) * gi.S + lc : Zg,
-                  ok ? 4 : 0);
+        zp[r * tp::kZP + c] = ok ? Zg[(long long)(cur.rc + r) * gi.S + lc] : DT<T>::from_f(0.f);
       }
     }
     {
       const int r = tid >> 3, pc = tid & 7;
       const bool ok = cur.rc + r < nrows;
-      cp_async16(xs + (uint32_t)(r * tp::kXP + 8 * pc) * (uint32_t)sizeof(T),
+      cp_async16(zs + kXOff + (uint32_t)(r * tp::kXP + 8 * pc) * (uint32_t)sizeof(T),
                  ok ? Xg + (size_t)(cur.rc + r) * xpitch + 8 * pc : Xg, ok ? 16 : 0);
+    }
+    if (tid < tp::kRC / 2) {
+      // the rows' saturated-offset sums (s_lo, s_hi), two rows per piece
+      const int r = 2 * tid;
+      const bool ok = cur.rc + r < nrows;
+      const float* src = dz_sat + 2 * ((size_t)bh * npad + r0 + cur.rc + r);
+      cp_async16(zs + kSOff + (uint32_t)r * 8u, ok ? src : dz_sat, ok ? (cur.rc + r + 1 < nrows ? 16 : 8) : 0);
     }
     cur.rc += tp::kRC;
     if (cur.rc >= nrows) {
@@ -397,64 +423,68 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[mt][i][0] = acc[mt][i][1] = acc[mt][i][2] = acc[mt][i][3] = 0.f;
-  // column sums of dZ for db_part: rows m0 and m0 + 8 of each m16 tile, over this
-  // lane's positions tq and tq + 4 of every k8 step
+  // column sums of dS for db_part: rows g8 and g8 + 8 of each m16 tile
   const bool with_db = db_part != nullptr;   // block-uniform
   float dbs[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  // the saturated offsets 0 / R_exp - 1 in this block: sums over the rows of
+  // s x X (thread: column sc, rows sr, sr + 4, ...) and, for db, of s
+  const bool sat_lo_here = c0 == 0, sat_hi_here = c0 <= p.Rexp - 1 && p.Rexp - 1 < c0 + tp::kEB;
+  const int sc = tid & 63, srg = tid >> 6;
+  float sx_lo = 0.f, sx_hi = 0.f, ss_lo = 0.f, ss_hi = 0.f;
 #pragma unroll
   for (int q = 0; q < tp::kStages - 1; ++q) {
     if (q < nchunks) load(q);
     cp_async_commit();
   }
+  // ldmatrix lane addresses (both operands transposed from [position][.] rows)
+  const int mi = lane >> 3;
+  const uint32_t a_off = (uint32_t)(((mi >> 1) * 8 + (lane & 7)) * tp::kZP + eb + (mi & 1) * 8) * (uint32_t)sizeof(T);
+  const uint32_t b_off = (uint32_t)(((mi & 1) * 8 + (lane & 7)) * tp::kXP + (mi >> 1) * 8) * (uint32_t)sizeof(T);
   for (int q = 0; q < nchunks; ++q) {
     cp_async_wait<tp::kStages - 2>();
     __syncthreads();   // chunk q visible to all; the stage of chunk q - 1 is free again
     if (q + tp::kStages - 1 < nchunks) load(q + tp::kStages - 1);
     cp_async_commit();
-    const uint8_t* st = tp_smem + (uint32_t)(q % tp::kStages) * kSB;
-    const float* Zs = reinterpret_cast<const float*>(st);
-    const T* Xs = reinterpret_cast<const T*>(st + (uint32_t)tp::kRC * tp::kZP * 4u);
+    const uint32_t zs = sbase + (uint32_t)(q % tp::kStages) * kSB;
 #pragma unroll
-    for (int ks = 0; ks < tp::kRC / 8; ++ks) {
-      // A = dZ^T: rows = expanded offsets, columns = positions
+    for (int ks = 0; ks < tp::kRC / 16; ++ks) {
+      // A = dS^T: rows = expanded offsets, columns = positions
       uint32_t a[2][4];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        const int m0 = eb + 16 * mt + g8;
-        const float z0 = Zs[(ks * 8 + tq) * tp::kZP + m0], z1 = Zs[(ks * 8 + tq) * tp::kZP + m0 + 8];
-        const float z2 = Zs[(ks * 8 + tq + 4) * tp::kZP + m0], z3 = Zs[(ks * 8 + tq + 4) * tp::kZP + m0 + 8];
-        a[mt][0] = to_tf32(z0);
-        a[mt][1] = to_tf32(z1);
-        a[mt][2] = to_tf32(z2);
-        a[mt][3] = to_tf32(z3);
+        ldsm_x4_t(zs + a_off + (uint32_t)(ks * 16 * tp::kZP + 16 * mt) * (uint32_t)sizeof(T), a[mt][0], a[mt][1],
+                  a[mt][2], a[mt][3]);
         if (with_db) {
-          dbs[mt][0] += z0 + z2;
-          dbs[mt][1] += z1 + z3;
+          dbs[mt][0] += DT<T>::pair_sum(a[mt][0]) + DT<T>::pair_sum(a[mt][2]);
+          dbs[mt][1] += DT<T>::pair_sum(a[mt][1]) + DT<T>::pair_sum(a[mt][3]);
         }
       }
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const uint32_t b0 = __float_as_uint(DT<T>::to_f(Xs[(ks * 8 + tq) * tp::kXP + nt * 8 + g8]));
-        const uint32_t b1 = __float_as_uint(DT<T>::to_f(Xs[(ks * 8 + tq + 4) * tp::kXP + nt * 8 + g8]));
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(zs + kXOff + b_off + (uint32_t)(ks * 16 * tp::kXP + np * 16) * (uint32_t)sizeof(T), b0, b1, b2, b3);
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) mma_tf32(acc[mt][nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+        for (int mt = 0; mt < 2; ++mt) {
+          MmaOp<T>::run(acc[mt][2 * np], a[mt], b0, b1);
+          MmaOp<T>::run(acc[mt][2 * np + 1], a[mt], b2, b3);
+        }
+      }
+    }
+    if (sat_lo_here || sat_hi_here) {   // block-uniform
+      const T* Xs = reinterpret_cast<const T*>(tp_smem + (uint32_t)(q % tp::kStages) * kSB + kXOff);
+      const float2* Ss = reinterpret_cast<const float2*>(tp_smem + (uint32_t)(q % tp::kStages) * kSB + kSOff);
+#pragma unroll
+      for (int rr = srg; rr < tp::kRC; rr += 4) {
+        const float2 sv = Ss[rr];
+        const float xv = DT<T>::to_f(Xs[rr * tp::kXP + sc]);
+        sx_lo = fmaf(sv.x, xv, sx_lo);
+        sx_hi = fmaf(sv.y, xv, sx_hi);
+        ss_lo += sv.x;
+        ss_hi += sv.y;
       }
     }
   }
   cp_async_wait<0>();
-  if (with_db) {
-    // the quad's four lanes hold the four position classes of the same rows
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v = dbs[mt][hf];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        const int e = c0 + eb + 16 * mt + g8 + 8 * hf;
-        if (tq == 0 && e < p.Rexp) db_part[((size_t)s * p.H + hq) * p.Rexp + e] = v;
-      }
-  }
   float* P = part + ((size_t)s * Hq + hq) * (size_t)p.Rexp * 64;
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt) {
@@ -465,32 +495,76 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int d = nt * 8 + 2 * tq;
-        *reinterpret_cast<float2*>(P + (size_t)e * 64 + d) = make_float2(acc[mt][nt][2 * hf], acc[mt][nt][2 * hf + 1]);
+        *reinterpret_cast<float2*>(P + (size_t)e * 64 + d) =
+            make_float2(p.tau * acc[mt][nt][2 * hf], p.tau * acc[mt][nt][2 * hf + 1]);
+      }
+    }
+  }
+  float* DB = with_db ? db_part + ((size_t)s * p.H + hq) * p.Rexp : nullptr;
+  if (with_db) {
+    // the quad's four lanes hold the four position classes of the same rows
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float v = dbs[mt][hf];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        const int e = c0 + eb + 16 * mt + g8 + 8 * hf;
+        if (tq == 0 && e < p.Rexp) DB[e] = p.tau * v;
+      }
+  }
+  if (sat_lo_here || sat_hi_here) {
+    // saturated offsets: the four row classes added in order on top of the
+    // (zero) stored columns 0 / R_exp - 1 written above
+    __shared__ float sred[4][64][2];
+    __shared__ float sdb[4][2];
+    __syncthreads();
+    sred[srg][sc][0] = sx_lo;
+    sred[srg][sc][1] = sx_hi;
+    if (sc == 0) { sdb[srg][0] = ss_lo; sdb[srg][1] = ss_hi; }
+    __syncthreads();
+    if (srg == 0) {
+      const float lo = ((sred[0][sc][0] + sred[1][sc][0]) + sred[2][sc][0]) + sred[3][sc][0];
+      const float hi = ((sred[0][sc][1] + sred[1][sc][1]) + sred[2][sc][1]) + sred[3][sc][1];
+      if (sat_lo_here) P[sc] += p.tau * lo;
+      if (sat_hi_here) P[(size_t)(p.Rexp - 1) * 64 + sc] += p.tau * hi;
+      if (with_db && sc == 0) {
+        if (sat_lo_here) DB[0] += p.tau * (((sdb[0][0] + sdb[1][0]) + sdb[2][0]) + sdb[3][0]);
+        if (sat_hi_here) DB[p.Rexp - 1] += p.tau * (((sdb[0][1] + sdb[1][1]) + sdb[2][1]) + sdb[3][1]);
       }
     }
   }
 }
 
-// db_part[s][h][e] = sum over the split's (batch, group) items of column e of
-// dZ^Q, for the block's 256 expanded columns.  Warp w takes the rows r = w
-// (mod 8) of every item, lane l the columns l + 32 k; the eight warp sums are
-// added in warp order at the end.
-__global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const float* __restrict__ dZ, const long long z_head,
-                                                        const int nsplit, float* __restrict__ part) {
+// db_part[s][h][e] = tau x the sum over the split's (batch, group) items of
+// column e of dS^Q (plus, at e = 0 and R_exp - 1, of the rows' fp32
+// saturated-offset sums), for the block's 256 expanded columns.  Warp w takes
+// the rows r = w (mod 8) of every item, lane l the columns l + 32 k; the eight
+// warp sums are added in warp order at the end.
+template <typename T>
+__global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const T* __restrict__ dZ, const long long z_head,
+                                                        const float* __restrict__ dz_sat, const int nsplit,
+                                                        float* __restrict__ part) {
   __shared__ float red[8][256];
+  __shared__ float sred[8][2];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c0 = blockIdx.x * 256, h = blockIdx.y, s = blockIdx.z;
   const long long nitems = (long long)p.B * p.nT;
   const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
+  const size_t npad = (size_t)p.nT * kTile;
+  const bool sat_lo_here = c0 == 0, sat_hi_here = c0 <= p.Rexp - 1 && p.Rexp - 1 < c0 + 256;
   float acc[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  float ss_lo = 0.f, ss_hi = 0.f;
   for (long long it = it0; it < it1; ++it) {
     const int b = (int)(it / p.nT), g = (int)(it - (long long)b * p.nT);
     const GroupInfo gi = p.gq[g];
     if (c0 + 256 <= gi.e0 || c0 >= gi.e0 + gi.W) continue;   // block-uniform
-    const int nrows = imin(kTile, p.N - g * kTile);
-    const float* Zg = dZ + (size_t)(b * p.H + h) * z_head + gi.base;
+    const int bh = b * p.H + h;
+    const int nrows = iclamp(seq_rows(p, b).len - g * kTile, 0, kTile);
+    const T* Zg = dZ + (size_t)bh * z_head + gi.base;
     int lc[8];
     bool okc[8];
 #pragma unroll
@@ -501,23 +575,33 @@ __global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const floa
     }
 #pragma unroll 4
     for (int r = warp; r < nrows; r += 8) {
-      const float* zr = Zg + (long long)r * gi.S;
+      const T* zr = Zg + (long long)r * gi.S;
       float v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = okc[k] ? __ldg(zr + lc[k]) : 0.f;
+      for (int k = 0; k < 8; ++k) v[k] = okc[k] ? DT<T>::to_f(zr[lc[k]]) : 0.f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) acc[k] += v[k];
+      if ((sat_lo_here || sat_hi_here) && lane == 0) {
+        const float2 sv = *reinterpret_cast<const float2*>(dz_sat + 2 * ((size_t)bh * npad + g * kTile + r));
+        ss_lo += sv.x;
+        ss_hi += sv.y;
+      }
     }
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) red[warp][lane + 32 * k] = acc[k];
+  if (lane == 0) { sred[warp][0] = ss_lo; sred[warp][1] = ss_hi; }
   __syncthreads();
   const int e = c0 + tid;
   if (e < p.Rexp) {
     float sum = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) sum += red[w][tid];
-    part[((size_t)s * p.H + h) * p.Rexp + e] = sum;
+    if (sat_lo_here && e == 0)
+      for (int w = 0; w < 8; ++w) sum += sred[w][0];
+    if (sat_hi_here && e == p.Rexp - 1)
+      for (int w = 0; w < 8; ++w) sum += sred[w][1];
+    part[((size_t)s * p.H + h) * p.Rexp + e] = p.tau * sum;
   }
 }
 
@@ -689,24 +773,29 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cuda
   // bias gradient's columns (its splits are the workspace's bias splits)
   const bool fuse_db = t.aq_exp && t.b_exp && t.table_per_head && t.nsplit_b == t.nsplit_q;
   if (side == 0 && t.aq_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 0, t.dzq, p.zq_head, (const T*)t.aq_exp,
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 0, (const T*)t.dzq, p.zq_head, t.dzq_sat,
+                                                                        (const T*)t.aq_exp,
                                                                         t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
-    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, t.dzq, p.zq_head, (const T*)t.q,
+    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, (const T*)t.dzq, p.zq_head,
+                                                                           t.dzq_sat, (const T*)t.q,
                                                                            t.table_per_head, t.nsplit_q, t.daq_part,
                                                                            fuse_db ? t.db_part : nullptr); note_launch(1); }
     launch_fold(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64, t.fold_lo, t.fold_hi, t.daq, s);
   }
   if (side == 1 && t.ak_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 1, t.dzk, p.zk_head, (const T*)t.ak_exp,
+    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 1, (const T*)t.dzk, p.zk_head, t.dzk_sat,
+                                                                        (const T*)t.ak_exp,
                                                                         t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
-    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, t.dzk, p.zk_head, (const T*)t.k,
+    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, (const T*)t.dzk, p.zk_head,
+                                                                           t.dzk_sat, (const T*)t.k,
                                                                            t.table_per_head, t.nsplit_k, t.dak_part,
                                                                            nullptr); note_launch(1); }
     launch_fold(t.dak_part, t.nsplit_k, Hq, p.Rexp, t.R, 64, t.fold_lo, t.fold_hi, t.dak, s);
   }
   if (side == 0 && t.b_exp) {
     if (!fuse_db)
-    { bias_part_kernel<<<dim3((p.Rexp + 255) / 256, p.H, t.nsplit_b), 256, 0, s>>>(p, t.dzq, p.zq_head, t.nsplit_b, t.db_part); note_launch(1); }
+    { bias_part_kernel<T><<<dim3((p.Rexp + 255) / 256, p.H, t.nsplit_b), 256, 0, s>>>(p, (const T*)t.dzq, p.zq_head,
+                                                                                     t.dzq_sat, t.nsplit_b, t.db_part); note_launch(1); }
     launch_fold(t.db_part, t.nsplit_b, p.H, p.Rexp, t.R, 1, t.fold_lo, t.fold_hi, t.db, s);
   }
   return cudaGetLastError();
