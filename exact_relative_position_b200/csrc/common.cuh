@@ -104,7 +104,7 @@ struct Plan {
   const GroupInfo* gq;          // device [nT]
   const GroupInfo* gk;          // device [nT]
   const int* key_len;           // device [B] or null
-  // attention dropout (0 = off): keep cell when (Philox word >> 8) >= drop_thresh
+  // attention dropout (0 = off): keep a cell when its 16-bit Philox uniform is >= drop_thresh
   int dropout;
   uint32_t drop_thresh, seed_lo, seed_hi, drop_offset;
   float drop_scale;             // 1 / (1 - p)
