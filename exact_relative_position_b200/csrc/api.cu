@@ -367,9 +367,11 @@ int prepare(const relpos_fwd_args* a, Plan& p, const Layout& L, uint8_t* ws, Ten
   t.fold_hi = reinterpret_cast<int*>(ws + L.fold_hi);
   if (a->b) t.b_exp = reinterpret_cast<float*>(ws + L.bexp);
   // expanded-table row e <-> offset E_lo + e
+  // truncated / identity maps use the caller's table in place: expanded row e is
+  // table row phi(E_lo) + e (consecutive rows; for clip 0 the single row 0)
   long long row0 = 0;
-  if (a->map.kind == RELPOS_MAP_TRUNCATED) row0 = (long long)p.E_lo + a->map.clip;
-  else if (a->map.kind == RELPOS_MAP_IDENTITY) row0 = (long long)p.E_lo + a->N - 1;
+  if (a->map.kind == RELPOS_MAP_TRUNCATED || a->map.kind == RELPOS_MAP_IDENTITY)
+    row0 = phi_of(a->map, a->N, p.E_lo);
   const size_t esz = 2;
   if (a->aq) {
     if (L.expand) { t.aq_exp = ws + L.aqe; t.aq_hs = (long long)p.Rexp * 64; }

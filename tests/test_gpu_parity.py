@@ -19,6 +19,7 @@ pytestmark = pytest.mark.gpu
 MAPS = {
     "trunc16": dict(map_kind="truncated", clip=16),
     "trunc200": dict(map_kind="truncated", clip=200),
+    "trunc0": dict(map_kind="truncated", clip=0),   # one table row: R_exp = 1, every tile saturated
     "identity": dict(map_kind="identity"),
     "t5": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=1),
     "t5uni": dict(map_kind="t5", num_buckets=32, max_distance=128, bidirectional=0),
@@ -90,6 +91,43 @@ def test_small_parity(case):
     want = run_oracle(w)
     check_forward(got, want, str(case))
     check_backward(got, want, str(case))
+
+
+@pytest.mark.parametrize("N,terms,causal,key_len,dtype,per_head", [
+    (300, ("aQ", "aK", "b"), False, [300, 177], torch.float16, False),
+    (257, ("aQ", "b"), True, None, torch.bfloat16, True)])
+def test_single_row_map(N, terms, causal, key_len, dtype, per_head):
+    """Clip 0: one table row, R_exp = 1, every tile saturated (both saturated-sum
+    sides of a row land on the one row).  Every score of a row gets the same q.aQ_0 +
+    b_0 shift, so by the softmax's shift invariance the exact daQ and db vanish
+    (sum_j dS_ij = 0).  The library's values are the rounding residue of
+    D_i = sum_c dO_ic O_ic with O (and P) rounded to 16 bits: per row about
+    eps sum_c |dO_ic O_ic|, eps the dtype's relative rounding; summed over the rows as
+    independent errors, with a factor 4."""
+    B = 1 if key_len is None else len(key_len)
+    w = small_workload(N=N, B=B, H=2, terms=terms, causal=causal, key_len=key_len, dtype=dtype,
+                       per_head_tables=per_head, tau=_tau(terms, dtype), **MAPS["trunc0"])
+    got = run_library(w, out_f32=(dtype == torch.bfloat16))
+    want = run_oracle(w)
+    check_forward(got, want, "trunc0")
+    for n in ("dq", "dk", "dv"):
+        assert relf(got[n], want[n]) <= 1e-2, n
+    assert np.max(np.abs(want["daq"])) < 1e-12
+    eps = 2.0 ** -10 if dtype == torch.float16 else 2.0 ** -8
+    q, do = w.q.double().numpy(), w.do.double().numpy()
+    dabs = np.sum(np.abs(do * want["o"]), axis=-1)                      # [B, H, N]
+    rowq = (dabs[..., None] * q) ** 2                                    # [B, H, N, 64]
+    if per_head:
+        bq = 4 * w.tau * eps * np.sqrt(rowq.sum(axis=(0, 2)))[:, None, :]   # [H, 1, 64]
+    else:
+        bq = 4 * w.tau * eps * np.sqrt(rowq.sum(axis=(0, 1, 2)))[None, :]   # [1, 64]
+    assert np.all(np.abs(got["daq"]) <= bq), (np.max(np.abs(got["daq"])), np.min(bq))
+    if got.get("db") is not None:
+        bb = 4 * w.tau * eps * np.sqrt((dabs ** 2).sum(axis=(0, 2)))[:, None]   # [H, 1]
+        assert np.all(np.abs(got["db"]) <= bb), (np.max(np.abs(got["db"])), np.min(bb))
+    if got.get("dak") is not None:
+        # k.aK_0 varies with the key: a genuine gradient
+        assert relf(got["dak"], want["dak"]) <= 1e-2
 
 
 def test_fully_masked_rows():
