@@ -505,7 +505,9 @@ def main():
         torch.cuda.synchronize()
         return t0, t1
 
-    e2e_steps = max(3, min(args.steps, 20))
+    # up to 100 pipelined steps: the pipeline's fill (the first upload) and drain (the
+    # last download) are paid once per run, so a longer run measures the steady state
+    e2e_steps = max(3, min(args.steps, 100))
     e2e_run(3)                                              # warm-up of the pipeline
     t0, t1 = e2e_run(e2e_steps)
     e2e_ms = t0.elapsed_time(t1) / e2e_steps
