@@ -1,5 +1,5 @@
 // warp_mma.cuh -- warp-level tensor-core helpers (mma.sync m16n8k16 for
-// 16-bit inputs, m16n8k8 for tf32), ldmatrix and cp.async staging with a
+// 16-bit inputs), ldmatrix and cp.async staging with a
 // 128-byte XOR swizzle for [rows x 64] 16-bit tiles.
 #pragma once
 
@@ -71,19 +71,6 @@ template <> struct MmaOp<__nv_bfloat16> {
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
   }
 };
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ void mma_tf32(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // A fragments (16 rows x 64 cols, 4 k16 steps) of a swizzled [rows x 64] tile.
 __device__ __forceinline__ void load_a_frags(uint32_t sbase, int row0, int lane, uint32_t (&a)[4][4]) {
