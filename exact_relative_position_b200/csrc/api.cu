@@ -316,6 +316,10 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
     return (int)std::max(1LL, s);
   };
   L->nsq = pick(148LL / ((long long)nE * L->Hq), items);   // one table-gradient CTA per SM
+  // a grouped map (the identity map) gives the table-gradient blocks very uneven
+  // work: an offset block near the diagonal is stored by every query group, one
+  // far from it by a few.  Eight splits spread the long blocks' items.
+  if (p->grouped) L->nsq = std::max(L->nsq, pick(8, items));
   L->nsk = L->nsq;
   // with per-head aQ tables the bias gradient comes out of the aQ table-gradient
   // pass, on its splits
