@@ -350,6 +350,9 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (e.g. --ncu --batch 4: inputs larger than L2 for a "
                          "one-kernel ncu capture)")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (e.g. a smaller case of the same map for a "
+                         "one-kernel ncu capture)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -373,7 +376,12 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", device_id=dev)
 
-    w = make_workload(args.workload, seed=rank, **({"B": args.batch} if args.batch > 0 else {}))
+    over = {}
+    if args.batch > 0:
+        over["B"] = args.batch
+    if args.seqlen > 0:
+        over["N"] = args.seqlen
+    w = make_workload(args.workload, seed=rank, **over)
     m = rp.RelPosMap(w.map_kind, w.clip, w.num_buckets, w.max_distance, w.bidirectional)
     elo, ehi = rp.expanded_bounds(m, w.N)
     R_exp = ehi - elo + 1
