@@ -371,8 +371,12 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
           ek0 = gk.e0;
           ek1 = gk.e0 + gk.W - 1;
         }
-        band_terms_q<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, i, j0, cb, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
-                                       imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
+        if (AQ)
+          band_terms_q_vec<AK, BIAS, 64>(x, p.E_lo, p.E_hi, i, lane, j0, cb, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile,
+                                         zS, imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
+        else
+          band_terms_q<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, i, j0, cb, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
+                                         imin(kT, N - j0) - 1, ek0, ek1, bexp, sc);
         const float2 nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
@@ -575,7 +579,11 @@ constexpr int kBarKV = 0, kBarQsFull = 1, kBarQsEmpty = kBarQsFull + kStages, kB
               kBarDsFree = kBarDsReady + 1, kBarDrain = kBarDsFree + 1;
 }  // namespace kp
 
-template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32, bool DROP>
+// VEC (with aK, for a wide interior band): the BAND tiles' k.aK gathers of a
+// key's own Z^K row read aligned float4 pieces where a chunk is all interior
+// (band_terms_k_vec); a narrow band, as Shaw clip 64's, has few such chunks and
+// keeps the plain gather (a separate instantiation, chosen by the host).
+template <typename T, bool AQ, bool AK, bool BIAS, bool DZK, bool DK32, bool DROP, bool VEC>
 __global__ void __launch_bounds__(kp::kThreads, 1)
     dkdv_sm100_kernel(const Plan p, const Tensors t, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -836,8 +844,12 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
           eq0 = gq.e0;
           eq1 = gq.e0 + gq.W - 1;
         }
-        band_terms_k<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, j, qb, cb, zk_row, gk.e0, gk.e0 + gk.W - 1, zq_tile, zS,
-                                       imin(kT, N - qb) - 1, eq0, eq1, bexp, sc);
+        if (AK && VEC)
+          band_terms_k_vec<AQ, BIAS, 64>(x, p.E_lo, p.E_hi, j, qb, cb, zk_row, gk.e0, gk.e0 + gk.W - 1, zq_tile, zS,
+                                         imin(kT, N - qb) - 1, eq0, eq1, bexp, sc);
+        else
+          band_terms_k<AQ, AK, BIAS, 64>(x, p.E_lo, p.E_hi, j, qb, cb, zk_row, gk.e0, gk.e0 + gk.W - 1, zq_tile, zS,
+                                         imin(kT, N - qb) - 1, eq0, eq1, bexp, sc);
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2v + c);
@@ -1098,12 +1110,20 @@ cudaError_t dk_typed(const Plan& p, const Tensors& t, cudaStream_t s) {
   if (!make_maps(p, t, m)) return cudaErrorInvalidValue;
   const bool aq = t.aq_exp, ak = t.ak_exp, bb = t.b_exp;
   const dim3 grid(p.nT, p.B * p.H);
-#define RP_DK(A, K_, B_)                                                                                         \
-  if (aq == A && ak == K_ && bb == B_)                                                                           \
-    return p.dropout ? launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, true>, grid, kp::kThreads, kp::kSmemBytes, \
-                               p, t, m.q, m.k, m.v, m.dout, s)                                                   \
-                     : launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, false>, grid, kp::kThreads, kp::kSmemBytes, \
-                               p, t, m.q, m.k, m.v, m.dout, s);
+  // the float4 k.aK gather for an interior band wider than two tiles
+  const bool wide = p.E_hi - p.E_lo + 1 > 2 * kT;
+#define RP_DK(A, K_, B_)                                                                                           \
+  if (aq == A && ak == K_ && bb == B_) {                                                                           \
+    if (K_ && wide)                                                                                                \
+      return p.dropout ? launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, true, K_>, grid, kp::kThreads,          \
+                                 kp::kSmemBytes, p, t, m.q, m.k, m.v, m.dout, s)                                 \
+                       : launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, false, K_>, grid, kp::kThreads,         \
+                                 kp::kSmemBytes, p, t, m.q, m.k, m.v, m.dout, s);                                \
+    return p.dropout ? launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, true, false>, grid, kp::kThreads,         \
+                               kp::kSmemBytes, p, t, m.q, m.k, m.v, m.dout, s)                                   \
+                     : launch4(dkdv_sm100_kernel<T, A, K_, B_, K_, K_, false, false>, grid, kp::kThreads,        \
+                               kp::kSmemBytes, p, t, m.q, m.k, m.v, m.dout, s);                                  \
+  }
   RP_DK(false, false, false) RP_DK(true, false, false) RP_DK(false, true, false) RP_DK(true, true, false)
   RP_DK(false, false, true) RP_DK(true, false, true) RP_DK(false, true, true) RP_DK(true, true, true)
 #undef RP_DK

@@ -344,8 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ek0 = gk.e0;
           ek1 = gk.e0 + gk.W - 1;
         }
-        band_terms_q<AQ, AK, BIAS, 128>(x, p.E_lo, p.E_hi, i, j0, 0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
-                                        imin(kBK, N - j0) - 1, ek0, ek1, bexp, sc);
+        // the float4 gather pays in the forward where q.aQ is the only per-row
+        // gather (the identity map's Transformer-XL layer); beside the aK gather
+        // its extra registers cost more than it saves
+        if (AQ && !AK)
+          band_terms_q_vec<AK, BIAS, 128>(x, p.E_lo, p.E_hi, i, lane, j0, 0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile,
+                                          zS, imin(kBK, N - j0) - 1, ek0, ek1, bexp, sc);
+        else
+          band_terms_q<AQ, AK, BIAS, 128>(x, p.E_lo, p.E_hi, i, j0, 0, zq_row, gi.e0, gi.e0 + gi.W - 1, zk_tile, zS,
+                                          imin(kBK, N - j0) - 1, ek0, ek1, bexp, sc);
       }
       const bool need_mask = (j0 + kBK > nkv) || (p.causal && j0 + kBK - 1 > q0 + g * kBQ);
       if (need_mask) {
