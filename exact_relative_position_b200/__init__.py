@@ -57,7 +57,8 @@ def relpos_attention(q, k, v, aq=None, ak=None, b=None, *, tau, map, causal=Fals
                      dropout_p=0.0, dropout_seed=0, dropout_offset=0, projection="retained",
                      cu_seqlens=None, max_seqlen=None):
     """Differentiable exact relative-position attention (CUDA only); optional
-    attention dropout with the Philox mask of (seed, offset); projection
+    attention dropout with the Philox mask of (seed, offset) at dropout_p rounded
+    up to a multiple of 1/256; projection
     "recompute" keeps the forward's memory linear (q.aQ projected per tile);
     a packed variable-length batch passes q, k, v as [T, H, d] with cu_seqlens
     (int32 CUDA [B + 1]) and max_seqlen."""

@@ -244,8 +244,8 @@ def relpos_attn_fwd(q, k, v, aq=None, ak=None, b=None, *, tau: float, map: RelPo
                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0,
                     projection: str = "retained", cu_seqlens=None, max_seqlen=None):
     """Forward through the C ABI.  Returns (O, LSE); O is float32 when out_f32.
-    Attention dropout with rate dropout_p uses the Philox mask of (seed, offset);
-    the backward needs the same three values.  projection="recompute" projects
+    Attention dropout with rate dropout_p (rounded up to a multiple of 1/256) uses
+    the Philox mask of (seed, offset); the backward needs the same three values.  projection="recompute" projects
     q.aQ inside every tile instead of storing Z^Q (linear forward memory).
     Packed variable-length batch: q, k, v [T, H, d] with cu_seqlens (int32
     CUDA [B + 1]) and max_seqlen; LSE is then [H, T]."""

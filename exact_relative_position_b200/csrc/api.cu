@@ -253,8 +253,10 @@ int make_plan(const relpos_fwd_args* a, Plan* p, Layout* L) {
   p->tau = a->tau;
   if (!(a->dropout_p >= 0.f && a->dropout_p < 1.f)) return RELPOS_ERR_INVALID_ARG;
   p->dropout = a->dropout_p > 0.f;
-  p->drop_thresh = (uint32_t)ceil((double)a->dropout_p * 65536.0);   // 16-bit uniforms
-  p->drop_scale = p->dropout ? 1.f / (1.f - a->dropout_p) : 1.f;
+  // 8-bit uniforms: the realised rate is p rounded up to a multiple of 1/256,
+  // and the kept cells are scaled by the reciprocal of its keep probability
+  p->drop_thresh = (uint32_t)ceil((double)a->dropout_p * 256.0);
+  p->drop_scale = p->dropout ? (float)(256.0 / (256.0 - (double)p->drop_thresh)) : 1.f;
   p->seed_lo = (uint32_t)(a->dropout_seed & 0xFFFFFFFFull);
   p->seed_hi = (uint32_t)(a->dropout_seed >> 32);
   p->drop_offset = a->dropout_offset;

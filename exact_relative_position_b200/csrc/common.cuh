@@ -104,10 +104,10 @@ struct Plan {
   const GroupInfo* gq;          // device [nT]
   const GroupInfo* gk;          // device [nT]
   const int* key_len;           // device [B] or null
-  // attention dropout (0 = off): keep a cell when its 16-bit Philox uniform is >= drop_thresh
+  // attention dropout (0 = off): keep a cell when its 8-bit Philox uniform is >= drop_thresh
   int dropout;
   uint32_t drop_thresh, seed_lo, seed_hi, drop_offset;
-  float drop_scale;             // 1 / (1 - p)
+  float drop_scale;             // 1 / (1 - drop_thresh / 256)
   // limit of every bounded mbarrier wait in the fused kernels (ns); the host
   // lowers it only to exercise the timeout path
   unsigned long long wait_ns;
@@ -289,10 +289,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 // definition: ten rounds of (hi0, lo0) = M0 x0, (hi1, lo1) = M1 x2 (32 x 32 ->
 // 64-bit), x = (hi1 ^ x1 ^ k0, lo1, hi0 ^ x3 ^ k1, lo0), the key bumped by
 // (W0, W1) before every round after the first.  One call serves a block of
-// 2 query rows x 4 keys: counter (j >> 2, i >> 1, bh, offset), key (seed_lo,
-// seed_hi); cell k = 4 (i & 1) + (j & 3) reads the 16-bit half k & 1 (low
-// half first) of output word k >> 1 and is kept when it is >= drop_thresh
-// (= ceil(p 2^16)).
+// 4 query rows x 4 keys: counter (j >> 2, i >> 2, bh, offset), key (seed_lo,
+// seed_hi); query row i & 3 reads output word i & 3, key j & 3 its byte j & 3
+// (least significant first), and the cell is kept when that byte is
+// >= drop_thresh (= ceil(256 p)).
 // ---------------------------------------------------------------------------
 #ifdef __CUDACC__
 __device__ __forceinline__ uint4 philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
@@ -313,86 +313,76 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t x0, uint32_t x1, uint32_
   return make_uint4(x0, x1, x2, x3);
 }
 
-// Keep bits of the two 16-bit uniforms of word w: bit 0 low half, bit 1 high half.
-__device__ __forceinline__ uint32_t keep2(uint32_t w, uint32_t thresh) {
-  return ((w & 0xFFFFu) >= thresh ? 1u : 0u) | ((w >> 16) >= thresh ? 2u : 0u);
+// Keep bits of the four 8-bit uniforms of word w (bit b: byte b >= thresh).
+// Bytes 0 / 2 and 1 / 3 are added, as 16-bit lanes, to 256 - thresh: the carry
+// into bit 8 of a lane is the comparison (thresh <= 256, so no lane overflows).
+__device__ __forceinline__ uint32_t keep4(uint32_t w, uint32_t thresh) {
+  const uint32_t c = (256u - thresh) * 0x00010001u;
+  const uint32_t e = ((w & 0x00FF00FFu) + c) & 0x01000100u;          // bytes 0, 2 -> bits 8, 24
+  const uint32_t o = (((w >> 8) & 0x00FF00FFu) + c) & 0x01000100u;   // bytes 1, 3 -> bits 8, 24
+  const uint32_t m = e | (o << 1);                                   // bits 8, 9, 24, 25
+  return ((m >> 8) & 3u) | ((m >> 22) & 12u);
 }
 
 // Keep bits of 64 consecutive columns c0 .. c0 + 63 (c0 a multiple of 4) of
 // this lane's row; bit c of km[c >> 5] keeps column c0 + c.  The whole warp
-// calls this.
-//  row_is_query: rows are queries i (lane parity = i & 1), columns keys.  A
-//    block is the 2 rows of a lane pair x 4 columns; each lane draws every
-//    other block and hands its partner the partner's 4 bits of each (one
-//    shuffle), so a lane makes 8 generator calls for its 64 cells.
-//  otherwise: rows are keys j (lane & 3 = j & 3), columns queries.  A block is
-//    2 columns x the 4 keys of a lane quad; each lane of the quad draws every
-//    fourth block and hands each other lane its 2 bits of each (three
-//    shuffles), again 8 generator calls per lane.
+// calls this, with rows = 32 consecutive indices, lane = row & 31.
+//  row_is_query: rows are queries i, columns keys; a block is the 4 rows of a
+//    lane quad (i & 3) x 4 keys and gives row i & 3 the 4 bits of word i & 3.
+//  otherwise: rows are keys j, columns queries; a block is 4 queries x the 4
+//    keys of a lane quad (j & 3) and gives key j & 3 byte j & 3 of each word.
+// Either way the quad's 16 blocks over the 64 columns are split so that each
+// lane draws every fourth one (4 generator calls per lane for its 64 cells)
+// and hands each of the other three lanes its 4 bits of each (three shuffles).
 __device__ __forceinline__ void keep_mask64(const Plan& p, int bh, int row, int c0, bool row_is_query,
                                             uint32_t (&km)[2]) {
   km[0] = km[1] = 0u;
   const uint32_t th = p.drop_thresh;
-  if (row_is_query) {
-    const int par = row & 1;
-    uint32_t give = 0u;                          // the partner's 4 bits of each block this lane draws
+  const int q4 = row & 3;                       // this lane's place in its quad
+  uint32_t give[4] = {0u, 0u, 0u, 0u};          // 4 bits per drawn block for each lane of the quad
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int blk = 2 * t + par;              // block: columns c0 + 4 blk .. + 3
-      const uint4 r = philox4x32_10((uint32_t)(c0 + 4 * blk) >> 2, (uint32_t)row >> 1, (uint32_t)bh, p.drop_offset,
-                                    p.seed_lo, p.seed_hi);
-      // cells of row parity 0 are words x, y; of parity 1 words z, w
-      const uint32_t even = keep2(r.x, th) | (keep2(r.y, th) << 2);
-      const uint32_t odd = keep2(r.z, th) | (keep2(r.w, th) << 2);
-      km[blk >> 3] |= (par ? odd : even) << (4 * (blk & 7));
-      give |= (par ? even : odd) << (4 * t);
+  for (int t = 0; t < 4; ++t) {
+    const int blk = 4 * t + q4;                 // block: columns c0 + 4 blk .. + 3
+    const uint32_t cb = (uint32_t)(c0 + 4 * blk) >> 2, rb = (uint32_t)row >> 2;
+    const uint4 r = row_is_query ? philox4x32_10(cb, rb, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi)
+                                 : philox4x32_10(rb, cb, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi);
+    const uint32_t k0 = keep4(r.x, th), k1 = keep4(r.y, th), k2 = keep4(r.z, th), k3 = keep4(r.w, th);
+    if (row_is_query) {
+      // lane q of the quad is query row q: word q, its 4 bits are the block's 4 keys
+      give[0] |= k0 << (4 * t);
+      give[1] |= k1 << (4 * t);
+      give[2] |= k2 << (4 * t);
+      give[3] |= k3 << (4 * t);
+    } else {
+      // lane q of the quad is key q: bit q of every word, one per query of the block
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        give[q] |= (((k0 >> q) & 1u) | (((k1 >> q) & 1u) << 1) | (((k2 >> q) & 1u) << 2) | (((k3 >> q) & 1u) << 3))
+                   << (4 * t);
     }
-    const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, give, 1);
+  }
+  // own bits first, then each partner's bits for this lane
+  uint32_t mine = give[0];
+  if (q4 == 1) mine = give[1];
+  if (q4 == 2) mine = give[2];
+  if (q4 == 3) mine = give[3];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int blk = 2 * t + (par ^ 1);        // the blocks the partner drew
+  for (int t = 0; t < 4; ++t) {
+    const int blk = 4 * t + q4;
+    km[blk >> 3] |= ((mine >> (4 * t)) & 0xFu) << (4 * (blk & 7));
+  }
+#pragma unroll
+  for (int d = 1; d < 4; ++d) {
+    const int src = q4 ^ d;                     // the partner lane; it drew blocks 4 t + src
+    uint32_t send = give[0];
+    if (src == 1) send = give[1];
+    if (src == 2) send = give[2];
+    if (src == 3) send = give[3];
+    const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, d);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int blk = 4 * t + src;
       km[blk >> 3] |= ((got >> (4 * t)) & 0xFu) << (4 * (blk & 7));
-    }
-  } else {
-    const int q4 = row & 3;                     // this lane's key within its quad
-    uint32_t give[4] = {0u, 0u, 0u, 0u};        // 2 bits per drawn block for each key of the quad
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int blk = 4 * t + q4;               // block: columns c0 + 2 blk, + 1 (queries)
-      const uint4 r = philox4x32_10((uint32_t)row >> 2, (uint32_t)(c0 + 2 * blk) >> 1, (uint32_t)bh, p.drop_offset,
-                                    p.seed_lo, p.seed_hi);
-      // key jj: query parity 0 reads cell jj (word jj >> 1), parity 1 cell 4 + jj (word 2 + (jj >> 1))
-      const uint32_t lo01 = keep2(r.x, th), lo23 = keep2(r.y, th), hi01 = keep2(r.z, th), hi23 = keep2(r.w, th);
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const uint32_t q0b = ((jj < 2 ? lo01 : lo23) >> (jj & 1)) & 1u;
-        const uint32_t q1b = ((jj < 2 ? hi01 : hi23) >> (jj & 1)) & 1u;
-        give[jj] |= (q0b | (q1b << 1)) << (2 * t);
-      }
-    }
-    // own bits, then the three partners' bits for this key
-    uint32_t mine = give[0];
-    if (q4 == 1) mine = give[1];
-    if (q4 == 2) mine = give[2];
-    if (q4 == 3) mine = give[3];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int blk = 4 * t + q4;
-      km[blk >> 4] |= ((mine >> (2 * t)) & 3u) << (2 * (blk & 15));
-    }
-#pragma unroll
-    for (int d = 1; d < 4; ++d) {
-      const int dst = q4 ^ d;                   // the partner lane's key; it sends this lane's bits
-      uint32_t send = give[0];
-      if (dst == 1) send = give[1];
-      if (dst == 2) send = give[2];
-      if (dst == 3) send = give[3];
-      const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, d);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int blk = 4 * t + dst;            // a block the partner drew
-        km[blk >> 4] |= ((got >> (2 * t)) & 3u) << (2 * (blk & 15));
-      }
     }
   }
 }

@@ -117,14 +117,14 @@ typedef struct {
   float* lse;                /* device [B,H,N] float32, natural log: output (fwd) / input (bwd);
                                 -inf for a row whose keys are all masked (its O row is 0) */
   /* Attention dropout (no counterpart on the paper's pages: the standard form).
-   * O = (P o M / (1 - p)) V with P = softmax(S) (LSE is that of S) and M_ij in
-   * {0, 1} drawn by Philox4x32-10 (Salmon et al., SC 2011), one call per block
-   * of 2 query rows x 4 keys: cell (b*H + h, i, j) uses counter (j >> 2, i >> 1,
-   * b*H + h, dropout_offset) and key (low, high 32 bits of dropout_seed); with
-   * k = 4 (i & 1) + (j & 3), u = 16-bit half k & 1 (low half first) of output
-   * word k >> 1, and M_ij = 1 when u >= ceil(p 2^16).  The backward regenerates
-   * the same mask, so pass the same three values to both calls.  dropout_p in
-   * [0, 1); 0 = no dropout. */
+   * O = (P o M / (1 - p')) V with P = softmax(S) (LSE is that of S), M_ij in
+   * {0, 1} drawn by Philox4x32-10 (Salmon et al., SC 2011), and p' = ceil(256 p)
+   * / 256 the rate the mask realises.  One generator call per block of 4 query
+   * rows x 4 keys: cell (b*H + h, i, j) uses counter (j >> 2, i >> 2, b*H + h,
+   * dropout_offset) and key (low, high 32 bits of dropout_seed); u = byte j & 3
+   * (least significant first) of output word i & 3, and M_ij = 1 when
+   * u >= ceil(256 p).  The backward regenerates the same mask, so pass the same
+   * three values to both calls.  dropout_p in [0, 1); 0 = no dropout. */
   float dropout_p;
   uint32_t dropout_offset;
   uint64_t dropout_seed;

@@ -268,17 +268,16 @@ def _f64(x):
 
 # ----------------------------------------------------------------------------
 # Attention dropout (the scope table's next row f3; not on the pages, the
-# standard attention-dropout semantics): O = (P o M / (1 - p)) V with P the
-# softmax of S (so LSE is that of S), M_ij in {0, 1}.  The mask is drawn by
-# the counter-based generator Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
-# "Parallel random numbers: as easy as 1, 2, 3", SC 2011), restated here from
-# that definition: ten rounds of
+# standard attention-dropout semantics): O = (P o M / (1 - p')) V with P the
+# softmax of S (so LSE is that of S), M_ij in {0, 1}, and p' the rate p
+# rounded up to a multiple of 2^-8 (the mask compares 8-bit uniforms).  The
+# mask is drawn by the counter-based generator Philox4x32-10 (Salmon, Moraes,
+# Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011),
+# restated here from that definition: ten rounds of
 #     (hi0, lo0) = M0 * x0,  (hi1, lo1) = M1 * x2   (32 x 32 -> 64-bit products)
 #     x = (hi1 ^ x1 ^ k0, lo1, hi0 ^ x3 ^ k1, lo0)
-# with the key bumped by (W0, W1) before every round after the first.
-# Cell (bh, i, j): counter (j >> 1, i >> 1, bh, offset), key (seed low 32
-# bits, seed high 32 bits); output word 2 (i & 1) + (j & 1) as w; kept when
-# (w >> 8) 2^-24 >= p.
+# with the key bumped by (W0, W1) before every round after the first.  The
+# cell layout (which output byte serves which cell) is in dropout_keep.
 # ----------------------------------------------------------------------------
 
 PHILOX_M0, PHILOX_M1 = 0xD2511F53, 0xCD9E8D57
@@ -303,22 +302,27 @@ def philox4x32_10(ctr, key):
     return x
 
 
+def dropout_rate(p):
+    """The rate the mask realises: p rounded up to a multiple of 2^-8 (a cell is
+    dropped when its 8-bit uniform u has u 2^-8 < p, i.e. u < ceil(256 p))."""
+    return np.ceil(np.float64(p) * 256.0) / 256.0
+
+
 def dropout_keep(bh, rows, N, p, seed, offset):
     """Kept cells [len(rows), N] (bool) of slice bh = b * H + h.
 
-    One Philox4x32-10 call serves a block of 2 query rows x 4 keys: counter
-    (j >> 2, i >> 1, bh, offset), key (low, high 32 bits of seed).  Cell
-    k = 4 (i & 1) + (j & 3) of the block reads the 16-bit half k & 1 (low half
-    first) of output word k >> 1 as a uniform u in [0, 2^16); the cell is kept
-    when u 2^-16 >= p."""
+    One Philox4x32-10 call serves a block of 4 query rows x 4 keys: counter
+    (j >> 2, i >> 2, bh, offset), key (low, high 32 bits of seed).  Query row
+    i & 3 of the block reads output word i & 3, key j & 3 its byte j & 3 (least
+    significant byte first), as a uniform u in [0, 256); the cell is kept when
+    u 2^-8 >= p."""
     i = np.asarray(rows, dtype=np.uint64)[:, None]
     j = np.arange(N, dtype=np.uint64)[None, :]
-    w = philox4x32_10((j >> np.uint64(2), i >> np.uint64(1), np.uint64(bh), np.uint64(offset & 0xFFFFFFFF)),
+    w = philox4x32_10((j >> np.uint64(2), i >> np.uint64(2), np.uint64(bh), np.uint64(offset & 0xFFFFFFFF)),
                       (np.uint64(seed & 0xFFFFFFFF), np.uint64((seed >> 32) & 0xFFFFFFFF)))
-    k = (i & np.uint64(1)) * np.uint64(4) + (j & np.uint64(3))
-    word = np.choose((k >> np.uint64(1)).astype(np.int64) + np.zeros(w[0].shape, dtype=np.int64), w)
-    u16 = (word >> (np.uint64(16) * (k & np.uint64(1)))) & np.uint64(0xFFFF)
-    return u16.astype(np.float64) * 2.0 ** -16 >= p
+    word = np.choose((i & np.uint64(3)).astype(np.int64) + np.zeros(w[0].shape, dtype=np.int64), w)
+    u8 = (word >> (np.uint64(8) * (j & np.uint64(3)))) & np.uint64(0xFF)
+    return u8.astype(np.float64) * 2.0 ** -8 >= p
 
 
 def head_scores(q, k, aq, ak, bvec, tau, phi, allowed):
@@ -352,7 +356,8 @@ def head_softmax(S):
 
 
 def head_forward(q, k, v, aq, ak, bvec, tau, phi, allowed, keep=None, p=0.0):
-    """O, LSE, P of one slice; with `keep` (bool [n, N]) O uses P o keep / (1 - p)."""
+    """O, LSE, P of one slice; with `keep` (bool [n, N]) O uses P o keep / (1 - p)
+    (p: the realised rate, dropout_rate of the requested one)."""
     S = head_scores(q, k, aq, ak, bvec, tau, phi, allowed)
     P, lse = head_softmax(S)
     Pv = P if keep is None else np.where(keep, P / (1.0 - p), 0.0)
@@ -363,7 +368,7 @@ def head_backward(q, k, v, do, aq, ak, bvec, tau, phi, allowed, R, keep=None, p=
     """Gradients of one full (b, h) slice for the upstream gradient dO.
 
     Returns dict: dq, dk, dv, dzq [N,R], dzk [N,R], daq [R,d], dak [R,d], db [R],
-    plus o, lse.  With dropout (`keep`), O = (P o M s) V, s = 1 / (1 - p):
+    plus o, lse.  With dropout (`keep`), O = (P o M s) V, s = 1 / (1 - p) (p the realised rate):
     dV = (P o M s)^T dO, dS = P o (M s o dO V^T - D), D_i = sum_c dO_ic O_ic."""
     N, d = q.shape
     O, lse, P = head_forward(q, k, v, aq, ak, bvec, tau, phi, allowed, keep, p)
@@ -425,7 +430,8 @@ def forward(q, k, v, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None, row
             keep = None if dropout_p == 0 else dropout_keep(bi * H + h, rows, N, dropout_p, dropout_seed,
                                                              dropout_offset)
             o, lse, _ = head_forward(q[bi, h, rows], k[bi, h], v[bi, h], _table(aq, h),
-                                     _table(ak, h), None if b is None else b[h], tau, phi, allowed, keep, dropout_p)
+                                     _table(ak, h), None if b is None else b[h], tau, phi, allowed, keep,
+                                     dropout_rate(dropout_p))
             O[bi, h], L[bi, h] = o, lse
     return O, L
 
@@ -453,7 +459,8 @@ def backward(q, k, v, do, aq, ak, b, tau, m: MapDesc, causal=False, key_len=None
             keep = None if dropout_p == 0 else dropout_keep(bi * H + h, np.arange(N), N, dropout_p, dropout_seed,
                                                              dropout_offset)
             g = head_backward(q[bi, h], k[bi, h], v[bi, h], do[bi, h], _table(aq, h),
-                              _table(ak, h), None if b is None else b[h], tau, phi, allowed, R, keep, dropout_p)
+                              _table(ak, h), None if b is None else b[h], tau, phi, allowed, R, keep,
+                              dropout_rate(dropout_p))
             for n in ("o", "dq", "dk", "dv", "lse"):
                 res[n][bi, h] = g[n]
             if aq is not None:

@@ -1,7 +1,8 @@
 """Pins of the oracle's attention dropout (scope-table next row f3).
 
 The Philox4x32-10 generator against its published known-answer vectors
-(tests/golden/philox4x32_10_kat.json); the keep rate; the p = 0 case against
+(tests/golden/philox4x32_10_kat.json); the keep rate and its rounding to
+multiples of 2^-8; sixteen distinct uniforms per call; the p = 0 case against
 the dropout-free oracle; and the dropout backward against central finite
 differences of sum(dO o O) with the mask held fixed (the mask depends only on
 (seed, offset, b, h, i, j), never on the inputs)."""
@@ -40,24 +41,60 @@ def test_philox_vectorised_matches_scalar():
 def test_keep_rate(p):
     keep = orc.dropout_keep(5, np.arange(512), 512, p, seed=0x1234_5678_9ABC_DEF0, offset=77)
     n = keep.size
-    sd = np.sqrt(p * (1 - p) / n)
-    assert abs(keep.mean() - (1 - p)) < 6 * sd
+    q = orc.dropout_rate(p)
+    assert q >= p and q - p < 2.0 ** -8
+    sd = np.sqrt(q * (1 - q) / n)
+    assert abs(keep.mean() - (1 - q)) < 6 * sd
+
+
+def test_rate_is_rounded_up_to_eighth_bit_steps():
+    """A rate between two multiples of 2^-8 masks exactly like the next one up;
+    the cells a step of 2^-8 adds are those whose uniform equals the step's
+    numerator, about 1 / 256 of them, and the masks are nested."""
+    kw = dict(seed=0x0F0F_1234, offset=11)
+    for p in (0.1, 0.3, 0.77):
+        q = np.ceil(256 * p) / 256
+        assert orc.dropout_rate(p) == q
+        assert np.array_equal(orc.dropout_keep(1, np.arange(256), 256, p, **kw),
+                              orc.dropout_keep(1, np.arange(256), 256, q, **kw))
+    lo = orc.dropout_keep(1, np.arange(256), 256, 26 / 256, **kw)
+    hi = orc.dropout_keep(1, np.arange(256), 256, 27 / 256, **kw)
+    assert np.all(lo >= hi)                          # dropped at 26/256 => dropped at 27/256
+    frac = np.mean(lo & ~hi)
+    assert abs(frac - 1 / 256) < 6 * np.sqrt(1 / 256 / lo.size)
+    assert orc.dropout_rate(0.0) == 0.0 and orc.dropout_rate(1.0) == 1.0
+    assert orc.dropout_rate(2.0 ** -12) == 2.0 ** -8
 
 
 def test_block_cells_use_distinct_uniforms():
-    """Each Philox call serves 2 x 4 cells with eight distinct 16-bit uniforms:
+    """Each Philox call serves 4 x 4 cells with sixteen distinct 8-bit uniforms:
     every pair of cell positions within a block agrees about half the time at
-    p = 0.5 (two cells reading the same half would always agree), and so do
-    cells of neighbouring blocks."""
+    p = 0.5 (two cells reading the same byte would always agree), and so do
+    cells of neighbouring blocks along both axes."""
     keep = orc.dropout_keep(2, np.arange(512), 512, 0.5, seed=0xDEADBEEF, offset=3)
-    blocks = keep.reshape(256, 2, 128, 4).transpose(0, 2, 1, 3).reshape(-1, 8)   # [block, 4 (i & 1) + (j & 3)]
+    blocks = keep.reshape(128, 4, 128, 4).transpose(0, 2, 1, 3).reshape(-1, 16)   # [block, 4 (i & 3) + (j & 3)]
     n = blocks.shape[0]
-    for a in range(8):
-        for b in range(a + 1, 8):
+    for a in range(16):
+        for b in range(a + 1, 16):
             agree = np.mean(blocks[:, a] == blocks[:, b])
             assert abs(agree - 0.5) < 6 * 0.5 / np.sqrt(n), (a, b, agree)
     agree_next = np.mean(keep[:, 3::4][:, :-1] == keep[:, 4::4])   # last key of a block vs first of the next
     assert abs(agree_next - 0.5) < 6 * 0.5 / np.sqrt(keep[:, 4::4].size)
+    agree_down = np.mean(keep[3::4][:-1] == keep[4::4])             # last row of a block vs first of the next
+    assert abs(agree_down - 0.5) < 6 * 0.5 / np.sqrt(keep[4::4].size)
+
+
+def test_mask_is_the_published_generator_bytes():
+    """Cell (i, j) of slice bh is byte j & 3 of word i & 3 of the generator's
+    output for counter (j >> 2, i >> 2, bh, offset), computed here for single
+    cells with the scalar generator (a transposed word / byte choice or a
+    wrong counter component fails it)."""
+    seed, off, bh = 0x0123_4567_89AB_CDEF, 9, 6
+    keep = orc.dropout_keep(bh, np.arange(24), 24, 0.5, seed, off)
+    for (i, j) in [(0, 0), (1, 2), (2, 1), (3, 3), (5, 9), (7, 4), (13, 22), (22, 13), (23, 23)]:
+        w = orc.philox4x32_10([j >> 2, i >> 2, bh, off], [seed & 0xFFFFFFFF, seed >> 32])
+        u = (int(w[i & 3]) >> (8 * (j & 3))) & 0xFF
+        assert keep[i, j] == (u >= 128), (i, j)
 
 
 def test_mask_rows_are_independent_of_the_row_subset():
