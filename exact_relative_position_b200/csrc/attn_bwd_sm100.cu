@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(qp::kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(kBarDpFree));     // dP(t + 1) may now be written
         if (DROP) {
-          // dropout: dS = P o (M / (1 - p) o dP - D)
+          // dropout: dS = P o (M / (1 - p') o dP - D)
           uint32_t km[2];
           keep_mask64(p, bh, i, j0 + cb, true, km);
 #pragma unroll
@@ -882,9 +882,8 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          if (DROP)   // dV sees P^T o M / (1 - p)
-            pk[u] = DT<T>::pack(kept(2 * u) ? x[2 * u] * p.drop_scale : 0.f,
-                                kept(2 * u + 1) ? x[2 * u + 1] * p.drop_scale : 0.f);
+          if (DROP)   // dV sees P^T o M; the epilogue scales dV by 1 / (1 - p')
+            pk[u] = DT<T>::pack(kept(2 * u) ? x[2 * u] : 0.f, kept(2 * u + 1) ? x[2 * u + 1] : 0.f);
           else
             pk[u] = DT<T>::pack(x[2 * u], x[2 * u + 1]);
         }
@@ -1018,8 +1017,9 @@ __global__ void __launch_bounds__(kp::kThreads, 1)
       uint32_t u[32];
       tmem_ld32(tmem + t_lane + kTmDV + 32 * hc, u);
       tmem_wait_ld();
+      const float vs = DROP ? p.drop_scale : 1.f;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) dv[c] = __uint_as_float(u[c]);
+      for (int c = 0; c < 32; ++c) dv[c] = __uint_as_float(u[c]) * vs;
       tmem_ld32(tmem + t_lane + kTmDK + 32 * hc, u);
       tmem_wait_ld();
 #pragma unroll

@@ -423,9 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (DT<T>::kCoarse) ps[w & 1] += DT<T>::pair_sum(pk[w]);
         else ps2[w & 1] = fadd2(ps2[w & 1], e);
         if (DROP) {
-          // PV sees P o M / (1 - p)
+          // PV sees P o M; the epilogue scales O by 1 / (1 - p')
           const uint32_t kb = (km[w >> 4] >> (2 * (w & 15))) & 3u;
-          pk[w] = DT<T>::pack((kb & 1u) ? e.x * p.drop_scale : 0.f, (kb & 2u) ? e.y * p.drop_scale : 0.f);
+          pk[w] = DT<T>::pack((kb & 1u) ? e.x : 0.f, (kb & 2u) ? e.y : 0.f);
         }
       }
       l_run += DT<T>::kCoarse ? ps[0] + ps[1] : (ps2[0].x + ps2[1].x) + (ps2[0].y + ps2[1].y);
@@ -451,7 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tO + 0, u);
       tmem_ld32(tO + 32, u + 32);
       tmem_wait_ld();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      // dropout: the kept P went to PV unscaled (the same 16-bit values the row
+      // sum holds); 1 / (1 - p') is applied here
+      const float inv = l_run > 0.f ? (DROP ? p.drop_scale : 1.f) / l_run : 0.f;
 #pragma unroll
       for (int c = 0; c < 64; ++c) ov[c] = __uint_as_float(u[c]) * inv;
     }

@@ -192,7 +192,10 @@ __global__ void __launch_bounds__(256) relgrad_rows_kernel(const Plan p, const i
   extern __shared__ __align__(16) uint8_t rg_smem[];
   constexpr uint32_t kSB = rg::stage_bytes<T>();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = blockIdx.x, bh = blockIdx.y, h = bh % p.H, b = bh / p.H;
+  // grid (batch x heads, groups), the groups launched from the last one down:
+  // under a causal mask a later group's rows reach more offsets, so the launch
+  // ends on the shortest groups
+  const int bh = blockIdx.x, g = (int)(gridDim.y - 1 - blockIdx.y), h = bh % p.H, b = bh / p.H;
   const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
   const int r0 = g * kTile;
   const SeqRows sr = seq_rows(p, b);
@@ -321,7 +324,10 @@ __global__ void __launch_bounds__(256) table_part_kernel(const Plan p, const int
   constexpr uint32_t kXOff = (uint32_t)tp::kRC * tp::kZP * (uint32_t)sizeof(T);
   constexpr uint32_t kSOff = kXOff + (uint32_t)tp::kRC * tp::kXP * (uint32_t)sizeof(T);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c0 = blockIdx.x * tp::kEB, hq = blockIdx.y, s = blockIdx.z;
+  // grid (splits, heads, expanded-row blocks), the blocks launched from the last
+  // one down: under a causal identity map the blocks next to the diagonal carry
+  // the most rows, and the launch then ends on the lightest ones
+  const int s = blockIdx.x, hq = blockIdx.y, c0 = (int)(gridDim.z - 1 - blockIdx.z) * tp::kEB;
   const int Hq = per_head ? p.H : 1;
   const long long nitems = per_head ? (long long)p.B * p.nT : (long long)p.B * p.H * p.nT;
   const long long it0 = nitems * s / nsplit, it1 = nitems * (s + 1) / nsplit;
@@ -773,20 +779,20 @@ static cudaError_t relgrad_typed(const Plan& p, const Tensors& t, int side, cuda
   // bias gradient's columns (its splits are the workspace's bias splits)
   const bool fuse_db = t.aq_exp && t.b_exp && t.table_per_head && t.nsplit_b == t.nsplit_q;
   if (side == 0 && t.aq_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 0, (const T*)t.dzq, p.zq_head, t.dzq_sat,
+    { relgrad_rows_kernel<T><<<dim3(p.B * p.H, p.nT), 256, kRowsSmem, sr>>>(p, 0, (const T*)t.dzq, p.zq_head, t.dzq_sat,
                                                                         (const T*)t.aq_exp,
                                                                         t.table_per_head ? t.aq_hs : 0, t.dq_acc, (T*)t.dq); note_launch(1); }
-    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_q), 256, kPartSmem, s>>>(p, 0, (const T*)t.dzq, p.zq_head,
+    { table_part_kernel<T><<<dim3(t.nsplit_q, Hq, nE), 256, kPartSmem, s>>>(p, 0, (const T*)t.dzq, p.zq_head,
                                                                            t.dzq_sat, (const T*)t.q,
                                                                            t.table_per_head, t.nsplit_q, t.daq_part,
                                                                            fuse_db ? t.db_part : nullptr); note_launch(1); }
     launch_fold(t.daq_part, t.nsplit_q, Hq, p.Rexp, t.R, 64, t.fold_lo, t.fold_hi, t.daq, s);
   }
   if (side == 1 && t.ak_exp) {
-    { relgrad_rows_kernel<T><<<dim3(p.nT, p.B * p.H), 256, kRowsSmem, sr>>>(p, 1, (const T*)t.dzk, p.zk_head, t.dzk_sat,
+    { relgrad_rows_kernel<T><<<dim3(p.B * p.H, p.nT), 256, kRowsSmem, sr>>>(p, 1, (const T*)t.dzk, p.zk_head, t.dzk_sat,
                                                                         (const T*)t.ak_exp,
                                                                         t.table_per_head ? t.ak_hs : 0, t.dk_acc, (T*)t.dk); note_launch(1); }
-    { table_part_kernel<T><<<dim3(nE, Hq, t.nsplit_k), 256, kPartSmem, s>>>(p, 1, (const T*)t.dzk, p.zk_head,
+    { table_part_kernel<T><<<dim3(t.nsplit_k, Hq, nE), 256, kPartSmem, s>>>(p, 1, (const T*)t.dzk, p.zk_head,
                                                                            t.dzk_sat, (const T*)t.k,
                                                                            t.table_per_head, t.nsplit_k, t.dak_part,
                                                                            nullptr); note_launch(1); }

@@ -44,6 +44,19 @@ def test_dropout_matches_oracle(case, p):
     check_backward(got, want, f"case {case} p {p}")
 
 
+@pytest.mark.parametrize("case", [0, 4])
+def test_dropout_rate_between_eighth_bit_steps(case):
+    """p = 0.1 is not a multiple of 1/256: both sides mask at ceil(25.6) = 26 /
+    256 and scale the kept cells by 256 / 230."""
+    w = _wl(CASES[case])
+    drop = (0.1, 0x0BAD_F00D + case, 17)
+    bf16 = str(w.dtype).endswith("bfloat16")
+    got = run_library(w, out_f32=bf16, dropout=drop)
+    want = run_oracle(w, dropout=drop)
+    check_forward(got, want, f"case {case} p 0.1")
+    check_backward(got, want, f"case {case} p 0.1")
+
+
 def test_dropout_is_deterministic_and_keyed():
     w = _wl(CASES[0])
     a = run_library(w, dropout=(0.25, 99, 5))
