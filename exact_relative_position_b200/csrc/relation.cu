@@ -618,6 +618,29 @@ __global__ void __launch_bounds__(256) bias_part_kernel(const Plan p, const T* _
 __global__ void __launch_bounds__(256) fold_rows_kernel(const float* __restrict__ part, const int nsplit, const int Hq,
                                                         const int Rexp, const int R, const int C,
                                                         const int* __restrict__ fold_lo, float* __restrict__ out) {
+  if (C == 64 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+    // a table row as 16 float4: the row, its head and its fold source are found once
+    // per four columns; the splits are added in the same order as below
+    const float4* src4 = reinterpret_cast<const float4*>(part);
+    const size_t split_stride = (size_t)Hq * Rexp * 16;
+    const long long n4 = (long long)Hq * R * 16;
+    for (long long idx = blockIdx.x * 256LL + threadIdx.x; idx < n4; idx += (long long)gridDim.x * 256) {
+      const long long hr = idx >> 4;
+      const int hq = (int)(hr / R), r = (int)(hr - (long long)hq * R);
+      const float4* src = src4 + ((size_t)hq * Rexp + fold_lo[r]) * 16 + (idx & 15);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float4 v = __ldg(src + sp * split_stride);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      reinterpret_cast<float4*>(out)[idx] = acc;
+    }
+    return;
+  }
   const long long n = (long long)Hq * R * C;
   for (long long idx = blockIdx.x * 256LL + threadIdx.x; idx < n; idx += (long long)gridDim.x * 256) {
     const int c = (int)(idx % C);
