@@ -66,8 +66,11 @@ __global__ void fold_mark_kernel(const int* __restrict__ phi_exp, const int Rexp
 }
 
 // ------------------------------------------------------------------ projection
-// Z[b,h, group g rows, columns e0 + [c0, c0 + 64)] = X_rows A_exp[e0 + c0 ..]^T
-constexpr int kProjSmem = 128 * 128 + 64 * 128;
+// Z[b,h, group g rows, columns e0 + [c0, c0 + 64)] = X_rows A_exp[e0 + c0 ..]^T for
+// kProjChunks consecutive 64-column chunks per CTA: the group's X rows are loaded
+// once, and the next chunk's A rows arrive while the current chunk is stored.
+constexpr int kProjChunks = 4;
+constexpr int kProjSmem = 128 * 128 + 2 * 64 * 128;
 
 template <typename T>
 __global__ void __launch_bounds__(256) projection_kernel(const Plan p, const int key_side, const T* __restrict__ X,
@@ -75,42 +78,56 @@ __global__ void __launch_bounds__(256) projection_kernel(const Plan p, const int
                                                          float* __restrict__ Z, const long long z_head) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
+  const int g = blockIdx.y, bh = blockIdx.z;
   const int h = bh % p.H;
   const GroupInfo gi = key_side ? p.gk[g] : p.gq[g];
-  const int c0 = chunk * 64;
-  if (c0 >= gi.W) return;
+  const int cfirst = blockIdx.x * kProjChunks * 64;
+  if (cfirst >= gi.W) return;
+  const int nch = imin(kProjChunks, (gi.W - cfirst + 63) / 64);
   const int r0 = g * kTile;
-  const uint32_t sX = smem_u32(smem), sA = sX + 128 * 128;
+  const uint32_t sX = smem_u32(smem), sA0 = sX + 128 * 128;
   // this sequence's rows of X (dense [B, H, N, 64] or packed [T, H, 64]); rows
   // past the sequence are zero-filled, so their projections are zero
   const int b = bh / p.H;
   const SeqRows sr = seq_rows(p, b);
   const T* Xh = X + (size_t)act_row(p, sr, b, h, 0) * 64;
-  const T* Ah = A + (size_t)h * a_hs + (size_t)(gi.e0 + c0) * 64;
+  const T* Ah = A + (size_t)h * a_hs + (size_t)gi.e0 * 64;
   load_tile_async<128, 256>(sX, Xh, r0, sr.len, tid, act_pitch(p));
-  load_tile_async<64, 256>(sA, Ah, 0, gi.W - c0, tid);
+  load_tile_async<64, 256>(sA0, Ah + (size_t)cfirst * 64, 0, gi.W - cfirst, tid);
   cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  uint32_t xa[4][4];
-  load_a_frags(sX, warp * 16, lane, xa);
-  float acc[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  mma_abt<T, 8>(acc, xa, sA, 0, lane);
   const int g8 = lane >> 2, tq = lane & 3;
   float* Zg = Z + (size_t)bh * z_head + gi.base;
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    const int rr = warp * 16 + g8 + 8 * hf;
-    if (r0 + rr >= p.N) continue;
-    float* zrow = Zg + (long long)rr * gi.S;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int col = c0 + nt * 8 + 2 * tq;
-      if (col < gi.W) *reinterpret_cast<float2*>(zrow + col) = make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+  uint32_t xa[4][4];
+#pragma unroll 1
+  for (int k = 0; k < nch; ++k) {
+    const int c0 = cfirst + 64 * k;
+    if (k + 1 < nch) {
+      // buffer (k + 1) & 1 was last read in iteration k - 1, which ended with a barrier
+      load_tile_async<64, 256>(sA0 + (uint32_t)((k + 1) & 1) * 64 * 128, Ah + (size_t)(c0 + 64) * 64, 0,
+                               gi.W - c0 - 64, tid);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
+    __syncthreads();
+    if (k == 0) load_a_frags(sX, warp * 16, lane, xa);
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    mma_abt<T, 8>(acc, xa, sA0 + (uint32_t)(k & 1) * 64 * 128, 0, lane);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int rr = warp * 16 + g8 + 8 * hf;
+      if (r0 + rr >= p.N) continue;
+      float* zrow = Zg + (long long)rr * gi.S;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int col = c0 + nt * 8 + 2 * tq;
+        if (col < gi.W) *reinterpret_cast<float2*>(zrow + col) = make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+      }
+    }
+    __syncthreads();   // every warp has read buffer k & 1 before iteration k + 1 refills it
   }
 }
 
@@ -742,12 +759,12 @@ static cudaError_t projection_typed(const Plan& p, const Tensors& t, cudaStream_
   if (!p.grouped) { wq = wk = p.Rexp; }
   else { wq = wk = p.N + kTile - 1; }
   if (t.zq && t.aq_exp) {
-    dim3 grid((wq + 63) / 64, p.nT, p.B * p.H);
+    dim3 grid((wq + 64 * kProjChunks - 1) / (64 * kProjChunks), p.nT, p.B * p.H);
     { projection_kernel<T><<<grid, 256, kProjSmem, s>>>(p, 0, (const T*)t.q, (const T*)t.aq_exp,
                                                       t.table_per_head ? t.aq_hs : 0, t.zq, p.zq_head); note_launch(1); }
   }
   if (t.zk && t.ak_exp) {
-    dim3 grid((wk + 63) / 64, p.nT, p.B * p.H);
+    dim3 grid((wk + 64 * kProjChunks - 1) / (64 * kProjChunks), p.nT, p.B * p.H);
     { projection_kernel<T><<<grid, 256, kProjSmem, sk>>>(p, 1, (const T*)t.k, (const T*)t.ak_exp,
                                                       t.table_per_head ? t.ak_hs : 0, t.zk, p.zk_head); note_launch(1); }
   }
